@@ -1,0 +1,94 @@
+"""Chunkwise form of the KDA recurrence in float64 (test infrastructure only).
+
+This restates, in plain numpy, the chunk algebra that follows from the
+token-by-token definition (see ``ref.py``). The pages name the technique --
+chunk-parallel prefill with a WY representation, chunk size 64 (KimiLinear
+KDA/MLA tutorial (icman.com.cn), sec. 3 config and sec. 6 tuning notes) -- but
+print no formula, so the steps below are derived here from the definition.
+
+Within one chunk of L <= C tokens (rows r = 0..L-1), with S the state entering
+the chunk and all products per key channel c:
+
+  g_r      = sum_{j<=r} log_alpha_j                   (cumulative log-decay)
+  Kt_r     = k_r * exp(g_r)         Kh_r = k_r * exp(-g_r)
+  Qt_r     = q_r * exp(g_r)         Kend_r = k_r * exp(g_{L-1} - g_r)
+  A        = StrictLower(diag(beta) Kt Kh^T)          (A_ri = beta_r sum_c k_rc k_ic exp(g_rc - g_ic), i < r)
+  Tm       = (I + A)^{-1}                             (unit lower triangular)
+  W        = Tm diag(beta) Kt ,   U' = Tm diag(beta) V
+  U        = U' - W S                                 (the per-token delta-rule writes u_r)
+  O        = Qt S + tril(Qt Kh^T) U                   (diagonal included)
+  S_next   = Diag(exp(g_{L-1})) S + Kend^T U
+
+Derivation sketch: unrolling the recurrence inside the chunk gives
+S_r = Diag(e^{g_r}) S + sum_{i<=r} Diag(e^{g_r - g_i}) k_i u_i^T with
+u_r = beta_r (v_r - (Diag(alpha_r) S_{r-1})^T k_r); collecting the u_r gives the
+unit lower-triangular system (I + A) U = diag(beta)(V - Kt S).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def _chunk(S, q, k, v, la, be):
+    L = q.shape[0]
+    g = np.cumsum(la, axis=0)
+    Kt = k * np.exp(g)
+    Kh = k * np.exp(-g)
+    Qt = q * np.exp(g)
+    Kend = k * np.exp(g[L - 1][None, :] - g)
+    A = np.tril(be[:, None] * (Kt @ Kh.T), -1)
+    Tm = np.linalg.inv(np.eye(L) + A)
+    W = Tm @ (be[:, None] * Kt)
+    Up = Tm @ (be[:, None] * v)
+    U = Up - W @ S
+    O = Qt @ S + np.tril(Qt @ Kh.T) @ U
+    S_next = np.exp(g[L - 1])[:, None] * S + Kend.T @ U
+    return O, S_next
+
+
+def forward(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, chunk=64):
+    """Same arguments and results as ``ref.forward_numpy``, computed chunk by chunk."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    la = np.asarray(log_alpha, dtype=np.float64)
+    be = np.asarray(beta, dtype=np.float64)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is None:
+        spans = [(b, 0, T) for b in range(B)]
+    else:
+        cu = [int(x) for x in cu_seqlens]
+        spans = [(0, cu[n], cu[n + 1]) for n in range(len(cu) - 1)]
+    out = np.zeros((B, T, H, dv))
+    Sf = np.zeros((len(spans), H, dk, dv))
+    for n, (b, t0, t1) in enumerate(spans):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if S0 is None else np.array(S0[n, h], dtype=np.float64)
+            for s in range(t0, t1, chunk):
+                e = min(s + chunk, t1)
+                O, S = _chunk(S, q[b, s:e, h], k[b, s:e, h], v[b, s:e, h], la[b, s:e, h], be[b, s:e, h])
+                out[b, s:e, h] = O
+            Sf[n, h] = S
+    return out, Sf
+
+
+def decode_step(S, q, k, v, log_alpha, beta):
+    """One token per (sequence, head): the chunk form with L = 1.
+
+    S: [N, H, dk, dv]; q, k, log_alpha: [N, H, dk]; v: [N, H, dv]; beta: [N, H].
+    S' = Diag(alpha) S; w = S'^T k; u = beta (v - w); S_new = S' + k u^T;
+    o = S'^T q + (q . k) u. Returns (o, S_new).
+    """
+    S = np.asarray(S, dtype=np.float64)
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    a = np.exp(np.asarray(log_alpha, dtype=np.float64))
+    be = np.asarray(beta, dtype=np.float64)
+    Sp = a[..., :, None] * S
+    w = np.einsum("nhi,nhij->nhj", k, Sp)
+    u = be[..., None] * (v - w)
+    S_new = Sp + k[..., :, None] * u[..., None, :]
+    o = np.einsum("nhi,nhij->nhj", q, Sp) + np.einsum("nhi,nhi->nh", q, k)[..., None] * u
+    return o, S_new
