@@ -1,0 +1,351 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA hot path on B200: chunkwise prefill (headline) and the decode step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+A step is one ``kda_chunk_fwd`` over the 128K-token, 32-head bf16 workload (B=1, T=131072,
+H=32, d_k=d_v=128, chunk 64, fp32 state, S0 ~ N(0, 0.1^2)); the decode step (256 sequences x 32
+heads, 512 MiB fp32 state, 1000 consecutive steps) is measured in the same run and reported
+under ``decode``. Inputs are synthetic (``kda_inputs``), resident in HBM before timing; one step
+reads 6.5 GB, far more than the 126 MB L2, so no flush is needed between steps.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own copy of the workload: the
+heads and sequences are independent, so there is no collective on the data path (weak scaling);
+only the timing uses a MAX all-reduce. ``--impl reference`` times the float64 CPU oracle on a
+bounded sample of the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kda_inputs as K  # noqa: E402
+
+METRIC = "KDA prefill Mtok/s @T=128K,H=32 (% TC peak); decode-step HBM GB/s vs peak"
+WORKLOAD = "bf16_t128k_h32"
+DECODE = "decode_n256_h32"
+C = 64
+D = 128
+# algorithmic HBM bytes per token*head of the prefill: q, k, v bf16 (3 x 256 B), out fp32
+# (512 B), log_alpha fp32 (512 B), beta fp32 (4 B)
+PREFILL_BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 4 + D * 4 + 4
+# useful tensor flops per token*head (chunk C): 6 d^2 (W.S, Q.S, Kend^T.U) + 5 C d (triangular
+# K K^T, Q K^T, T.(beta K), T.(beta V), M.U) + C^2 / 3 (triangular inverse)
+PREFILL_FLOPS_PER_TOKEN_HEAD = 6 * D * D + 5 * C * D + C * C // 3
+# decode: state read + written once per step
+DECODE_STATE_BYTES_PER_HEAD = 2 * D * D * 4
+DECODE_IO_BYTES_PER_HEAD = 3 * D * 2 + D * 4 + 4 + D * 4
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return dict(hbm=float(j["hbm_gbs"]), bf16=float(j["bf16_tflops"]),
+                    bf16_sus=float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+class Clocks:
+    """Samples SM clocks and throttle reasons with nvidia-smi while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                                       "--format=csv,noheader,nounits", "-lms", "100"],
+                                      stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.p = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.rows = []
+        if self.p is None:
+            return False
+        time.sleep(0.2)
+        self.p.terminate()
+        try:
+            out, _ = self.p.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+            out, _ = self.p.communicate()
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                self.rows.append(f)
+        return False
+
+    def summary(self):
+        if not getattr(self, "rows", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in self.rows:
+            for i, n in enumerate(names):
+                if "Active" in r[5 + i] and "Not" not in r[5 + i]:
+                    reasons.add(n)
+        # median under load: drop idle samples below half of max
+        top = max(mx) if mx else None
+        load = [s for s in sm if top is None or s > 0.3 * top] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": top,
+                "reasons": sorted(reasons), "samples": len(self.rows)}
+
+
+def dist_setup(n_gpus):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_loop(fn, steps, warmup, ws):
+    """CUDA-event time of `steps` calls of fn on the current stream, after `warmup` calls."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    barrier(ws)
+    return s.elapsed_time(e) / steps      # ms per call
+
+
+# ---------------------------------------------------------------------------------------------
+
+def cpu_oracle_sample(budget_s=12.0):
+    """Times the float64 oracle (as it stands) on a bounded sample of the prefill workload:
+    the first T' tokens of H' heads, with T' sized from a short calibration run so that the
+    whole sample takes about `budget_s` seconds on all host cores. Returns a dict in Mtok/s."""
+    from oracle import ref
+    cores = ref.online_cores()
+    w = K.WORKLOADS[WORKLOAD]
+    Hs = max(1, min(w.H, cores))
+    cal_T = 1024
+    d = K.make_prefill(w, T=cal_T, H=1)
+    args = [d[x].float().numpy() for x in ("q", "k", "v", "log_alpha", "beta")]
+    t0 = time.perf_counter()
+    ref.forward(*args, S0=d["S0"].double().numpy(), nthreads=1)
+    per_tok_head = (time.perf_counter() - t0) / cal_T
+    Ts = int(max(1024, min(w.T, budget_s / per_tok_head * min(Hs, cores) / Hs)))
+    d = K.make_prefill(w, T=Ts, H=Hs)
+    args = [d[x].float().numpy() for x in ("q", "k", "v", "log_alpha", "beta")]
+    t0 = time.perf_counter()
+    ref.forward(*args, S0=d["S0"].double().numpy(), nthreads=Hs)
+    dt = time.perf_counter() - t0
+    tok_equiv = Ts * Hs / w.H                 # tokens of the full 32-head workload
+    return {"value": tok_equiv / dt / 1e6, "unit": "Mtok/s", "cores": min(Hs, cores),
+            "kind": "oracle",
+            "sample": "float64 C recurrence on the first %d tokens of %d of the %d heads "
+                      "(%.1f s; scaled to tokens of all %d heads)" % (Ts, Hs, w.H, dt, w.H),
+            "seconds": dt, "host_cores": cores}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = K.WORKLOADS[WORKLOAD]
+    vals = []
+    budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for i in range(args.warmup + args.steps):
+        r = cpu_oracle_sample(budget_s=budget)
+        if i >= args.warmup:
+            vals.append(r)
+    v = statistics.median([r["value"] for r in vals])
+    ms = w.T / (v * 1e6) * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "Mtok/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": 1, "seq_len": w.T, "heads": w.H,
+                       "head_dim": D, "chunk": C, "parallelism": "none (host cores)"},
+            "cpu_baseline": {"kind": "oracle", "cores": vals[-1]["cores"], "sample": vals[-1]["sample"],
+                             "value": v, "unit": "Mtok/s"},
+            "e2e": {"value": v, "unit": "Mtok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------------
+
+def run_native(args):
+    ws, rank, local = dist_setup(args.gpus)
+    import kimi_delta_attention_25_b200 as kda
+    kda.load()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    pk = peaks()
+    w = K.WORKLOADS[WORKLOAD]
+    d = K.make_prefill(w, device=dev, seed=w.seed + rank)
+    B, T, H = w.B, w.T, w.H
+    out = torch.empty(B, T, H, D, dtype=torch.float32, device=dev)
+    Sf = torch.empty(B, H, D, D, dtype=torch.float32, device=dev)
+    wsz = kda.chunk_fwd_workspace_size(B, T, H, B)
+    work = torch.empty(max(256, wsz), dtype=torch.uint8, device=dev)
+
+    def step():
+        kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"],
+                      out=out, S_final=Sf, workspace=work)
+
+    step()
+    torch.cuda.synchronize()
+    assert kda.workspace_status(work) == kda.KDA_OK
+    with Clocks(local) as clk:
+        ms = time_loop(step, args.steps, args.warmup, ws)
+    ms = max_over_ranks(ms, ws)
+    tokens = B * T
+    value = ws * tokens / (ms * 1e-3) / 1e6                   # Mtok/s, whole job
+    th = B * T * H
+    alg_bytes = th * PREFILL_BYTES_PER_TOKEN_HEAD
+    flops = th * PREFILL_FLOPS_PER_TOKEN_HEAD
+    gbs = alg_bytes / (ms * 1e-3) / 1e9
+    tfs = flops / (ms * 1e-3) / 1e12
+
+    # ---- end to end through the public call with pinned host buffers
+    host = {x: d[x].cpu().pin_memory() for x in ("q", "k", "v", "log_alpha", "beta", "S0")}
+    dbuf = {x: torch.empty_like(d[x]) for x in host}
+    h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h_sf = torch.empty(Sf.shape, dtype=Sf.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = h_out.numel() * h_out.element_size() + h_sf.numel() * h_sf.element_size()
+
+    def e2e_step():
+        for x in host:
+            dbuf[x].copy_(host[x], non_blocking=True)
+        kda.chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["log_alpha"], dbuf["beta"],
+                      S0=dbuf["S0"], out=out, S_final=Sf, workspace=work)
+        h_out.copy_(out, non_blocking=True)
+        h_sf.copy_(Sf, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    ms_e2e = max_over_ranks(time_loop(e2e_step, e2e_steps, 1, ws), ws)
+    e2e_val = ws * tokens / (ms_e2e * 1e-3) / 1e6
+    del host, dbuf, h_out, h_sf
+
+    # ---- decode step
+    dec = run_decode(kda, dev, pk, ws, local, args)
+
+    del d, out
+    torch.cuda.empty_cache()
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": ws * B, "seq_len": T, "heads": H,
+                       "head_dim": D, "chunk": C, "state": "fp32", "gates": "fp32", "out": "fp32",
+                       "l2": "inputs larger than L2 (6.5 GB per step), no flush",
+                       "parallelism": "dp%d (independent heads/sequences per GPU)" % ws},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm"], "traffic": None,
+                         "peak_source": "of %s" % pk["src"],
+                         "kernel": "kda chunk prefill",
+                         "algorithmic_bytes_per_launch": alg_bytes,
+                         "tensor_tflops_useful": tfs, "tensor_frac_useful": tfs / pk["bf16"]},
+            "e2e": {"value": e2e_val, "unit": "Mtok/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+            "gpu_launches": args.steps * 1,
+            "clocks": clk.summary(),
+            "decode": dec,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+def run_decode(kda, dev, pk, ws, local, args):
+    w = K.WORKLOADS[DECODE]
+    N, H = w.B, w.H
+    S = K.make_decode_state(w, device=dev)
+    nsteps = w.decode_steps
+    xs = [K.make_decode_step(w, s, device=dev) for s in range(nsteps)]
+    out = torch.empty(N, H, D, dtype=torch.float32, device=dev)
+    it = [0]
+
+    def one():
+        x = xs[it[0] % nsteps]
+        it[0] += 1
+        kda.decode_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S, out=out)
+
+    with Clocks(local) as clk:
+        ms = time_loop(one, nsteps, 5, ws)
+    ms = max_over_ranks(ms, ws)
+    heads = N * H
+    state_b = heads * DECODE_STATE_BYTES_PER_HEAD
+    io_b = heads * DECODE_IO_BYTES_PER_HEAD
+    us = ms * 1e3
+    gbs = state_b / (ms * 1e-3) / 1e9
+    return {"workload": DECODE, "us_per_step": us, "steps": nsteps,
+            "state_gbs": gbs, "total_gbs": (state_b + io_b) / (ms * 1e-3) / 1e9,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm"], "traffic": None, "peak_source": "of %s" % pk["src"]},
+            "tokens_per_s_whole_job": ws * N / (ms * 1e-3),
+            "gpu_launches": nsteps, "clocks": clk.summary()}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,132 @@
+/*
+ * libkda.h -- C ABI of libkda, a B200 (sm_100a) implementation of the KDA
+ * (Kimi Delta Attention) layer's hot path: chunkwise prefill and the decode step.
+ *
+ * The operation (every head keeps a d_k x d_v state S):
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T ,   o_t = S_t^T q_t
+ *
+ * alpha_t = exp(log_alpha_t) in (0, 1]^{d_k} is the channel-wise forget gate,
+ * beta_t in [0, 1] the write gate. KDA is described as Gated DeltaNet with
+ * fine-grained, per-channel gates ("Kimi Linear" article (jdon.com), the
+ * passage on KDA's gating; KimiLinear KDA/MLA tutorial (icman.com.cn), sec. 2:
+ * fixed-size state, channel-level gating); the erase term (I - beta k k^T)
+ * and the need for unit-norm keys come from the same tutorial, sec. 5. The
+ * pages print no formula; the order "decay, erase and write, then read" is the
+ * plainest reading of that delta-rule update. The layer hands q/k/v over as
+ * "... h d" (lpnh.cn Kimi Linear KDA/NoPE article, sec. 4), so tensors here
+ * are laid out token-major with heads inside, the head dimension fastest.
+ *
+ * General rules for every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *    allocates no device memory; scratch comes from the caller's workspace.
+ *  - Tensors are dense, row-major, last index fastest, with no padding.
+ *  - q, k, v, out, log_alpha, S0, S_final, S_inout and workspace must be
+ *    16-byte aligned; beta and cu_seqlens 4-byte aligned. A misaligned or
+ *    NULL required pointer returns KDA_ERR_INVALID_ARG before any launch.
+ *  - Only d_k = d_v = 128 is implemented; other sizes return KDA_ERR_UNSUPPORTED.
+ *  - q and k are expected to be L2-normalised per head (a precondition of the
+ *    layer, not applied here). log_alpha must be finite and <= 0, beta in [0, 1];
+ *    neither is checked. The chunked prefill additionally needs the cumulative
+ *    log-decay inside one 64-token chunk to stay above -80 per channel
+ *    (exp of its negation must be finite in fp32); the decode step has no such limit.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream). A KDA_ERR_CUDA return means a launch failed.
+ *  - Calls are thread-safe; concurrent calls must not share output buffers
+ *    or workspaces.
+ *  - Errors are returned, never thrown.
+ */
+#ifndef LIBKDA_H
+#define LIBKDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or cu_seqlens content */
+    KDA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (d_k, d_v != 128) */
+    KDA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    KDA_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up */
+} kda_status_t;
+
+typedef enum {
+    KDA_F32 = 0,               /* float32 */
+    KDA_BF16 = 1               /* bfloat16 (round-to-nearest-even on output) */
+} kda_dtype_t;
+
+/* Bytes of device workspace kda_chunk_fwd needs for these sizes (always >= 256;
+ * the first 256 bytes hold the device status word read by kda_workspace_status).
+ * Returns 0 for sizes kda_chunk_fwd would reject. */
+size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int N, int dk, int dv,
+                                    kda_dtype_t dtype);
+
+/* Chunkwise-parallel prefill (chunk of 64 tokens): the recurrence above over
+ * every sequence and head, returning every o_t and the final state.
+ * Chunked form with a WY (UT) representation: KimiLinear KDA/MLA tutorial
+ * (icman.com.cn), sec. 3 (chunk_size 64) and sec. 6 (chunk-parallel + WY);
+ * training and long prompts use this chunk mode (lpnh.cn article, sec. 5).
+ *
+ *   q, k       [B, T, H, dk]  dtype           v    [B, T, H, dv] dtype
+ *   (dtype is the element type of q, k and v; out_dtype that of out. An fp32
+ *    out keeps the result unrounded for what follows, e.g. an output norm;
+ *    a bf16 out halves the output traffic and adds one bf16 rounding.)
+ *   log_alpha  [B, T, H, dk]  float32         beta [B, T, H]     float32
+ *   S0         [N, H, dk, dv] float32, or NULL for a zero initial state
+ *   cu_seqlens NULL: N must equal B and batch row b is one sequence of T tokens.
+ *              Otherwise int32 [N+1] device array of packed offsets (B must be 1):
+ *              cu_seqlens[0] = 0, non-decreasing, cu_seqlens[N] = T. Sequences may
+ *              be empty (then S_final = S0). Contents are checked on the device:
+ *              a violation writes KDA_ERR_INVALID_ARG to the workspace status word
+ *              (read it with kda_workspace_status) and the affected sequences are
+ *              skipped.
+ *   out        [B, T, H, dv]  out_dtype  (written: o_t for every token)
+ *   S_final    [N, H, dk, dv] float32, or NULL (not written)
+ *   workspace  device buffer of kda_chunk_fwd_workspace_size(...) bytes,
+ *              workspace_bytes its size. Its status word is cleared by this call.
+ * S0 and S_final may alias (in-place continuation); no other buffers may overlap.
+ * T = 0 or N = 0 is valid (only S_final = S0 is written). */
+kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const float *beta,
+                           const float *S0, const int32_t *cu_seqlens,
+                           void *out, float *S_final,
+                           int B, int T, int H, int N, int dk, int dv,
+                           kda_dtype_t dtype, kda_dtype_t out_dtype,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/* One decode step for N independent sequences (one token each), updating the
+ * state in place: the recurrent ("fused_recurrent") mode the layer uses for
+ * short queries and generation (lpnh.cn article, sec. 2 and 5); the per-step
+ * cost is fixed by the state size, not by the context length (KimiLinear
+ * KDA/MLA tutorial (icman.com.cn), sec. 1 and 2).
+ *
+ *   q, k       [N, H, dk] dtype     v [N, H, dv] dtype
+ *   log_alpha  [N, H, dk] float32   beta [N, H] float32
+ *   S_inout    [N, H, dk, dv] float32, read as S_{t-1} and overwritten with S_t
+ *   out        [N, H, dv] out_dtype, written with o_t = S_t^T q_t
+ * N = 0 is valid (nothing is launched). */
+kda_status_t kda_decode_step(const void *q, const void *k, const void *v,
+                             const float *log_alpha, const float *beta,
+                             float *S_inout, void *out,
+                             int N, int H, int dk, int dv, kda_dtype_t dtype,
+                             kda_dtype_t out_dtype, void *stream);
+
+/* Waits for `stream`, then copies the workspace status word to *status
+ * (KDA_OK when every device-side check passed). */
+kda_status_t kda_workspace_status(const void *workspace, void *stream, int32_t *status);
+
+/* Static, human-readable name of a status code. */
+const char *kda_status_string(kda_status_t status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBKDA_H */

@@ -1,0 +1,155 @@
+"""libkda: B200 (sm_100a) kernels for the KDA (Kimi Delta Attention) hot path.
+
+Thin Python binding over the C ABI in ``include/libkda.h``: argument
+marshalling only. PyTorch supplies device memory and streams; every step of
+the computation runs in the CUDA kernels of ``libkda.so``. There is no CPU
+fallback: if the library is missing or no CUDA device is present, calls raise.
+
+Names follow the C entry points:
+
+* ``chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None)`` -> ``(out, S_final)``
+* ``decode_step(q, k, v, log_alpha, beta, S)`` -> ``out`` (``S`` updated in place)
+* ``chunk_fwd_workspace_size``, ``workspace_status``, ``status_string``
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = ["chunk_fwd", "decode_step", "chunk_fwd_workspace_size", "workspace_status",
+           "status_string", "library_path", "load", "KDAError",
+           "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA", "KDA_ERR_TIMEOUT"]
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
+KDA_F32, KDA_BF16 = 0, 1
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_PKG, "libkda.so")
+_lib = None
+
+# Every entry point declared in include/libkda.h.
+EXPORTS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
+           "kda_workspace_status", "kda_status_string", "kda_version")
+
+
+class KDAError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__("%s: %s (status %d)" % (where, status_string(code), code))
+        self.code = code
+
+
+def load():
+    """Load ``libkda.so`` (built in-tree by ``python -m kimi_delta_attention_25_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(library_path):
+        raise RuntimeError("libkda.so not found at %s; build it with "
+                           "`python -m kimi_delta_attention_25_b200.build`" % library_path)
+    lib = ctypes.CDLL(library_path)
+    P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.kda_chunk_fwd_workspace_size.argtypes = [I, I, I, I, I, I, I]
+    lib.kda_chunk_fwd_workspace_size.restype = Z
+    lib.kda_chunk_fwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P]
+    lib.kda_chunk_fwd.restype = I
+    lib.kda_decode_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P]
+    lib.kda_decode_step.restype = I
+    lib.kda_workspace_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
+    lib.kda_workspace_status.restype = I
+    lib.kda_status_string.argtypes = [I]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_version.restype = I
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load().kda_status_string(int(code)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return KDA_F32
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    raise TypeError("q/k/v must be float32 or bfloat16, got %s" % t.dtype)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libkda takes CUDA tensors only (no CPU fallback)")
+        if t is not None and not t.is_contiguous():
+            raise ValueError("libkda takes contiguous tensors only")
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def chunk_fwd_workspace_size(B, T, H, N, dk=128, dv=128, dtype=torch.bfloat16) -> int:
+    code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    return int(load().kda_chunk_fwd_workspace_size(B, T, H, N, dk, dv, code))
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, S_final=None,
+              workspace=None, want_state=True, out_dtype=torch.float32):
+    """Chunkwise KDA prefill. Shapes: q, k, log_alpha [B,T,H,dk]; v [B,T,H,dv];
+    beta [B,T,H]; S0 [N,H,dk,dv] fp32 or None; cu_seqlens int32 [N+1] or None.
+    Returns (out [B,T,H,dv] in out_dtype (or the dtype of a given ``out``),
+    S_final [N,H,dk,dv] fp32 or None)."""
+    lib = load()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = B if cu_seqlens is None else cu_seqlens.shape[0] - 1
+    if out is None:
+        out = torch.empty(B, T, H, dv, dtype=out_dtype, device=q.device)
+    if S_final is None and want_state:
+        S_final = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
+    _need_cuda(q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final)
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    code = _dtype_code(q)
+    ws_bytes = lib.kda_chunk_fwd_workspace_size(B, T, H, N, dk, dv, code)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=q.device)
+    st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                           _ptr(cu_seqlens), _ptr(out), _ptr(S_final), B, T, H, N, dk, dv, code,
+                           _dtype_code(out), _ptr(workspace), workspace.numel(), _stream(q.device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_fwd")
+    chunk_fwd.last_workspace = workspace
+    return out, S_final
+
+
+def workspace_status(workspace: torch.Tensor) -> int:
+    """Device status word of a workspace after a kda_chunk_fwd call (syncs the stream)."""
+    v = ctypes.c_int32(0)
+    st = load().kda_workspace_status(_ptr(workspace), _stream(workspace.device), ctypes.byref(v))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_workspace_status")
+    return int(v.value)
+
+
+def decode_step(q, k, v, log_alpha, beta, S, out=None, out_dtype=torch.float32):
+    """One decode step: q, k, log_alpha [N,H,dk]; v [N,H,dv]; beta [N,H]; S [N,H,dk,dv] fp32
+    (updated in place). Returns out [N,H,dv] in out_dtype (or the dtype of a given ``out``)."""
+    lib = load()
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty(N, H, dv, dtype=out_dtype, device=q.device)
+    _need_cuda(q, k, v, log_alpha, beta, S, out)
+    st = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S),
+                             _ptr(out), N, H, dk, dv, _dtype_code(q), _dtype_code(out),
+                             _stream(q.device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_decode_step")
+    return out

@@ -1,0 +1,120 @@
+// api.cu -- the extern "C" entry points of libkda: argument checks, then kernel launches.
+//
+// Every check that can be made from the host is made here, before anything is enqueued, and
+// reported as a status code. The one check that needs device data (the contents of cu_seqlens)
+// is made by the kernels, which record it in the caller's workspace status word.
+#include <cuda_runtime.h>
+
+#include "kda_internal.cuh"
+
+using namespace kda;
+
+namespace {
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+kda_status_t map_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int kda_version(void) { return 100; }
+
+const char *kda_status_string(kda_status_t s)
+{
+    switch (s) {
+    case KDA_OK: return "ok";
+    case KDA_ERR_INVALID_ARG: return "invalid argument";
+    case KDA_ERR_UNSUPPORTED: return "unsupported size (only d_k = d_v = 128)";
+    case KDA_ERR_CUDA: return "CUDA error";
+    case KDA_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int N, int dk, int dv, kda_dtype_t dtype)
+{
+    if (B < 0 || T < 0 || H <= 0 || N < 0 || dk != kHeadDim || dv != kHeadDim) return 0;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return 0;
+    return kStatusBytes;
+}
+
+kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const float *beta,
+                           const float *S0, const int32_t *cu_seqlens,
+                           void *out, float *S_final,
+                           int B, int T, int H, int N, int dk, int dv,
+                           kda_dtype_t dtype, kda_dtype_t out_dtype,
+                           void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (out_dtype != KDA_F32 && out_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || H <= 0 || N < 0) return KDA_ERR_INVALID_ARG;
+    if (dk != kHeadDim || dv != kHeadDim) return KDA_ERR_UNSUPPORTED;
+    if (cu_seqlens) {
+        if (B != 1) return KDA_ERR_INVALID_ARG;
+        if (!aligned(cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
+    } else if (N != B) {
+        return KDA_ERR_INVALID_ARG;
+    }
+    if ((long long)B * T > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    const bool has_tokens = (long long)B * T > 0;
+    if (has_tokens) {
+        if (!q || !k || !v || !log_alpha || !beta || !out) return KDA_ERR_INVALID_ARG;
+        if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+            !aligned(log_alpha, 16) || !aligned(beta, 4))
+            return KDA_ERR_INVALID_ARG;
+    }
+    if ((S0 && !aligned(S0, 16)) || (S_final && !aligned(S_final, 16))) return KDA_ERR_INVALID_ARG;
+    const size_t need = kda_chunk_fwd_workspace_size(B, T, H, N, dk, dv, dtype);
+    if (!workspace || !aligned(workspace, 16) || workspace_bytes < need) return KDA_ERR_INVALID_ARG;
+
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, st);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    if (N == 0) return KDA_OK;
+
+    PrefillArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.S0 = S0;
+    a.cu_seqlens = cu_seqlens; a.out = out; a.S_final = S_final;
+    a.B = B; a.T = T; a.H = H; a.N = N;
+    a.status = (int32_t *)workspace;
+    a.scratch = (unsigned char *)workspace + kStatusBytes;
+    a.scratch_bytes = workspace_bytes - kStatusBytes;
+    return map_cuda(launch_chunk_fp32(a, dtype, out_dtype, st));
+}
+
+kda_status_t kda_decode_step(const void *q, const void *k, const void *v,
+                             const float *log_alpha, const float *beta,
+                             float *S_inout, void *out,
+                             int N, int H, int dk, int dv, kda_dtype_t dtype,
+                             kda_dtype_t out_dtype, void *stream)
+{
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (out_dtype != KDA_F32 && out_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (N < 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+    if (dk != kHeadDim || dv != kHeadDim) return KDA_ERR_UNSUPPORTED;
+    if (N == 0) return KDA_OK;
+    if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !log_alpha || !beta || !S_inout || !out) return KDA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(log_alpha, 16) || !aligned(S_inout, 16) || !aligned(beta, 4))
+        return KDA_ERR_INVALID_ARG;
+    return map_cuda(launch_decode(q, k, v, log_alpha, beta, S_inout, out, N, H, dtype, out_dtype,
+                                  (cudaStream_t)stream));
+}
+
+kda_status_t kda_workspace_status(const void *workspace, void *stream, int32_t *status)
+{
+    if (!workspace || !status) return KDA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    int32_t v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    *status = v;
+    return KDA_OK;
+}
+
+}  // extern "C"

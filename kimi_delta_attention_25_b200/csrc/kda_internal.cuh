@@ -1,0 +1,74 @@
+// kda_internal.cuh -- shared device helpers and launcher prototypes of libkda.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "libkda.h"
+
+namespace kda {
+
+constexpr int kHeadDim = 128;   // d_k = d_v supported by every kernel
+constexpr int kChunk = 64;      // chunk length of the prefill (tokens)
+constexpr size_t kStatusBytes = 256;  // workspace prefix holding the device status word
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Records the first device-side error in the workspace status word.
+__device__ __forceinline__ void set_status(int32_t *status, int32_t code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+// Resolves the token span [t0, t1) of sequence n (flat token index = b * T + t)
+// and checks cu_seqlens on the device. Returns false (and flags the status word)
+// when the offsets are inconsistent; the caller then skips the sequence.
+__device__ __forceinline__ bool sequence_span(const int32_t *cu_seqlens, int n, int N, int T,
+                                              int64_t *t0, int64_t *t1, int32_t *status) {
+    if (cu_seqlens == nullptr) {
+        *t0 = (int64_t)n * T;
+        *t1 = *t0 + T;
+        return true;
+    }
+    const int32_t a = cu_seqlens[n], b = cu_seqlens[n + 1];
+    bool ok = (a >= 0) && (b >= a) && (b <= T);
+    if (n == 0 && a != 0) ok = false;
+    if (n == N - 1 && b != T) ok = false;
+    if (!ok) {
+        set_status(status, KDA_ERR_INVALID_ARG);
+        return false;
+    }
+    *t0 = a;
+    *t1 = b;
+    return true;
+}
+
+struct PrefillArgs {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta, *S0;
+    const int32_t *cu_seqlens;
+    void *out;
+    float *S_final;
+    int B, T, H, N;
+    int32_t *status;      // device status word (workspace prefix)
+    void *scratch;        // workspace after the status prefix
+    size_t scratch_bytes;
+};
+
+// CUDA-core fp32 chunk path (any input dtype; fp32 arithmetic throughout).
+cudaError_t launch_chunk_fp32(const PrefillArgs &a, kda_dtype_t dtype, kda_dtype_t out_dtype,
+                              cudaStream_t stream);
+
+// Decode step (memory-bound state update in place).
+cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,
+                          const float *beta, float *S, void *out, int N, int H,
+                          kda_dtype_t dtype, kda_dtype_t out_dtype, cudaStream_t stream);
+
+}  // namespace kda

@@ -1,0 +1,109 @@
+"""The C-ABI library loads, exports every entry point of include/libkda.h, and rejects bad
+arguments on the host before anything is launched (no GPU needed: every call here returns
+before its first CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import kimi_delta_attention_25_b200 as kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "libkda.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(kda_[a-z0-9_]+)\s*\(", src, re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from kimi_delta_attention_25_b200 import build
+    build.build()
+    return kda.load()
+
+
+def test_header_declares_the_entry_points():
+    assert declared_functions() == sorted(kda.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    nm = os.popen("nm -D --defined-only %s" % kda.library_path).read()
+    for name in declared_functions():
+        assert re.search(r"\bT %s\b" % name, nm), name
+
+
+def test_status_strings_and_version(lib):
+    assert kda.status_string(kda.KDA_OK) == "ok"
+    assert "invalid" in kda.status_string(kda.KDA_ERR_INVALID_ARG)
+    assert lib.kda_version() >= 100
+
+
+def test_workspace_size(lib):
+    assert kda.chunk_fwd_workspace_size(1, 8192, 16, 1) >= 256
+    assert kda.chunk_fwd_workspace_size(1, 8192, 16, 1, dk=64) == 0
+    assert kda.chunk_fwd_workspace_size(-1, 8192, 16, 1) == 0
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: each call below fails a host check first
+
+
+def _chunk(lib, **kw):
+    P = ctypes.c_void_p
+    a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, S0=None, cu=None, out=FAKE, Sf=None,
+             B=1, T=64, H=2, N=1, dk=128, dv=128, dtype=1, odt=0, ws=FAKE, wsb=256)
+    a.update(kw)
+    return lib.kda_chunk_fwd(P(a["q"]), P(a["k"]), P(a["v"]), P(a["la"]), P(a["beta"]), P(a["S0"]),
+                             P(a["cu"]), P(a["out"]), P(a["Sf"]), a["B"], a["T"], a["H"], a["N"],
+                             a["dk"], a["dv"], a["dtype"], a["odt"], P(a["ws"]), a["wsb"], None)
+
+
+def test_chunk_fwd_host_checks(lib):
+    assert _chunk(lib, dk=64) == kda.KDA_ERR_UNSUPPORTED
+    assert _chunk(lib, dv=256) == kda.KDA_ERR_UNSUPPORTED
+    assert _chunk(lib, q=None) == kda.KDA_ERR_INVALID_ARG
+    assert _chunk(lib, q=FAKE + 2) == kda.KDA_ERR_INVALID_ARG            # misaligned
+    assert _chunk(lib, S0=FAKE + 8) == kda.KDA_ERR_INVALID_ARG
+    assert _chunk(lib, N=2) == kda.KDA_ERR_INVALID_ARG                    # N != B without cu_seqlens
+    assert _chunk(lib, B=2, cu=FAKE) == kda.KDA_ERR_INVALID_ARG           # packed needs B == 1
+    assert _chunk(lib, cu=FAKE + 2) == kda.KDA_ERR_INVALID_ARG
+    assert _chunk(lib, ws=None) == kda.KDA_ERR_INVALID_ARG
+    assert _chunk(lib, wsb=16) == kda.KDA_ERR_INVALID_ARG
+    assert _chunk(lib, dtype=7) == kda.KDA_ERR_INVALID_ARG
+    assert _chunk(lib, odt=5) == kda.KDA_ERR_INVALID_ARG
+    assert _chunk(lib, H=0) == kda.KDA_ERR_INVALID_ARG
+    assert _chunk(lib, T=-1) == kda.KDA_ERR_INVALID_ARG
+
+
+def _decode(lib, **kw):
+    P = ctypes.c_void_p
+    a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, S=FAKE, out=FAKE, N=4, H=2, dk=128,
+             dv=128, dtype=1, odt=0)
+    a.update(kw)
+    return lib.kda_decode_step(P(a["q"]), P(a["k"]), P(a["v"]), P(a["la"]), P(a["beta"]), P(a["S"]),
+                               P(a["out"]), a["N"], a["H"], a["dk"], a["dv"], a["dtype"], a["odt"],
+                               None)
+
+
+def test_decode_host_checks(lib):
+    assert _decode(lib, N=0) == kda.KDA_OK                                # nothing to do
+    assert _decode(lib, dk=96) == kda.KDA_ERR_UNSUPPORTED
+    assert _decode(lib, S=None) == kda.KDA_ERR_INVALID_ARG
+    assert _decode(lib, S=FAKE + 4) == kda.KDA_ERR_INVALID_ARG
+    assert _decode(lib, beta=FAKE + 2) == kda.KDA_ERR_INVALID_ARG
+    assert _decode(lib, H=-1) == kda.KDA_ERR_INVALID_ARG
+    assert _decode(lib, dtype=3) == kda.KDA_ERR_INVALID_ARG
+    assert _decode(lib, odt=2) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(1, 64, 2, 128)
+    with pytest.raises(ValueError):
+        kda.chunk_fwd(x, x, x, x, torch.zeros(1, 64, 2))

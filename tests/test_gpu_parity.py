@@ -1,0 +1,218 @@
+"""GPU parity: libkda (through its C ABI) against the float64 oracle on the same seeded inputs.
+
+Sizes span several 64-token chunks and a ragged tail; the full-size workloads are checked on
+sampled heads / sequences that the oracle recomputes from scratch. Tolerances: max|err| <=
+1e-4 * RMS(ref) for fp32 inputs, <= 2e-2 * RMS(ref) for bf16 inputs (fp32 state), applied to
+the outputs and to the final state separately.
+"""
+import numpy as np
+import pytest
+import torch
+
+import kda_inputs as K
+import kimi_delta_attention_25_b200 as kda
+from oracle import ref
+from tests.kda_check import TOL, assert_close, assert_close_bf16_out, np32, oracle_prefill, to_device
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from kimi_delta_attention_25_b200 import build
+    build.build()
+    kda.load()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+def _run_check(d, tol, heads=None, check_state=True, out_dtype=torch.float32):
+    g = to_device(d, DEV)
+    out, Sf = kda.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], S0=g["S0"],
+                            cu_seqlens=g["cu_seqlens"], out_dtype=out_dtype)
+    assert out.dtype == out_dtype
+    assert kda.workspace_status(kda.chunk_fwd.last_workspace) == kda.KDA_OK
+    ro, rs = oracle_prefill(d, heads=heads)
+    o = out if heads is None else out[:, :, heads]
+    s = Sf if heads is None else Sf[:, heads]
+    if out_dtype == torch.bfloat16:
+        e1 = assert_close_bf16_out(np32(o), ro, tol, "out (bf16)")
+    else:
+        e1 = assert_close(np32(o), ro, tol, "out")
+    e2 = assert_close(np32(s), rs, tol, "S_final") if check_state else 0.0
+    return e1, e2
+
+
+# ---- the small workloads, whole ------------------------------------------------------------
+
+def test_fp32_t256_h2_whole():
+    w = K.WORKLOADS["fp32_t256_h2"]
+    _run_check(K.make_prefill(w), TOL[torch.float32])
+
+
+def test_bf16_t8k_h16_whole():
+    w = K.WORKLOADS["bf16_t8k_h16"]
+    _run_check(K.make_prefill(w, device=DEV), TOL[torch.bfloat16])
+
+
+def test_bf16_t8k_h16_whole_bf16_out():
+    w = K.WORKLOADS["bf16_t8k_h16"]
+    _run_check(K.make_prefill(w, device=DEV), TOL[torch.bfloat16], out_dtype=torch.bfloat16)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 127, 200])
+def test_ragged_lengths(dtype, T):
+    w = K.Workload("ragged", B=2, T=T, H=3, dtype=dtype, alpha_lo=0.9, alpha_hi=0.999, s0_std=0.1)
+    _run_check(K.make_prefill(w, seed=T), TOL[K.to_dtype(dtype)])
+    _run_check(K.make_prefill(w, seed=T), TOL[K.to_dtype(dtype)], out_dtype=torch.bfloat16)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_varlen_with_empty_sequences(dtype):
+    torch.manual_seed(0)
+    lens = [70, 0, 1, 64, 0, 129]
+    cu = torch.tensor(np.cumsum([0] + lens), dtype=torch.int32)
+    T = int(cu[-1])
+    w = K.Workload("varlen", B=1, T=T, H=2, dtype=dtype, s0_std=0.1)
+    d = K.make_prefill(w, seed=3)
+    d["S0"] = 0.1 * torch.randn(len(lens), 2, 128, 128)
+    d["cu_seqlens"] = cu
+    _run_check(d, TOL[K.to_dtype(dtype)])
+
+
+def test_zero_initial_state_and_no_final_state():
+    w = K.Workload("nostate", B=1, T=100, H=2, dtype="bf16")
+    d = to_device(K.make_prefill(w, seed=5), DEV)
+    out, Sf = kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], want_state=False)
+    assert Sf is None
+    ro, _ = oracle_prefill(d)
+    assert_close(np32(out), ro, TOL[torch.bfloat16], "out")
+
+
+def test_invalid_cu_seqlens_flagged_on_device():
+    w = K.Workload("bad", B=1, T=128, H=2, dtype="bf16")
+    d = to_device(K.make_prefill(w, seed=6), DEV)
+    for bad in ([0, 100, 50, 128], [0, 64, 129], [1, 64, 128]):
+        cu = torch.tensor(bad, dtype=torch.int32, device=DEV)
+        kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], cu_seqlens=cu)
+        assert kda.workspace_status(kda.chunk_fwd.last_workspace) == kda.KDA_ERR_INVALID_ARG
+    cu = torch.tensor([0, 64, 128], dtype=torch.int32, device=DEV)
+    kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], cu_seqlens=cu)
+    assert kda.workspace_status(kda.chunk_fwd.last_workspace) == kda.KDA_OK
+
+
+# ---- properties ----------------------------------------------------------------------------
+
+def test_causality_bitwise():
+    w = K.Workload("causal", B=1, T=200, H=2, dtype="bf16", s0_std=0.1)
+    d = to_device(K.make_prefill(w, seed=7), DEV)
+    o1, _ = kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"])
+    t = 130
+    v2 = d["v"].clone()
+    v2[:, t + 1:] += 1.0
+    k2 = d["k"].clone()
+    k2[:, t + 1:] = k2[:, t + 1:].flip(-1)
+    o2, _ = kda.chunk_fwd(d["q"], k2, v2, d["log_alpha"], d["beta"], S0=d["S0"])
+    assert torch.equal(o1[:, :t + 1], o2[:, :t + 1])
+    assert not torch.equal(o1[:, t + 1:], o2[:, t + 1:])
+
+
+def test_split_continuation():
+    w = K.Workload("split", B=1, T=300, H=2, dtype="f32", s0_std=0.1)
+    d = to_device(K.make_prefill(w, seed=8), DEV)
+    o, s = kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"])
+    c = 100
+    part = lambda x, sl: x[:, sl].contiguous()  # noqa: E731
+    a, sa = kda.chunk_fwd(*(part(d[x], slice(0, c)) for x in ("q", "k", "v", "log_alpha", "beta")),
+                          S0=d["S0"])
+    b, sb = kda.chunk_fwd(*(part(d[x], slice(c, None)) for x in ("q", "k", "v", "log_alpha", "beta")),
+                          S0=sa)
+    assert_close(np32(torch.cat([a, b], 1)), np32(o), 1e-5, "out")
+    assert_close(np32(sb), np32(s), 1e-5, "S_final")
+
+
+def test_decode_steps_equal_chunked_prefill():
+    w = K.Workload("dec_vs_chunk", B=1, T=70, H=3, dtype="f32", s0_std=0.1)
+    d = to_device(K.make_prefill(w, seed=9), DEV)
+    o, s = kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"])
+    S = d["S0"].clone()
+    outs = []
+    for t in range(w.T):
+        x = {n: d[n][:, t].contiguous() for n in ("q", "k", "v", "log_alpha", "beta")}
+        outs.append(kda.decode_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S))
+    assert_close(np32(torch.stack(outs, 1)), np32(o), 1e-4, "out")
+    assert_close(np32(S), np32(s), 1e-4, "S")
+
+
+# ---- decode --------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decode_small(dtype, out_dtype):
+    w = K.Workload("dec", B=5, T=1, H=3, dtype=dtype, alpha_lo=0.95, alpha_hi=0.9999, s0_std=0.1)
+    S = K.make_decode_state(w, N=5, H=3)
+    Sg = S.to(DEV)
+    Sd = S.double().numpy()
+    for step in range(3):
+        x = K.make_decode_step(w, step, N=5, H=3)
+        g = to_device(x, DEV)
+        o = kda.decode_step(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], Sg, out_dtype=out_dtype)
+        cu = np.arange(6)
+        ro, Sd = ref.forward(np32(x["q"])[None], np32(x["k"])[None], np32(x["v"])[None],
+                             np32(x["log_alpha"])[None], np32(x["beta"])[None], S0=Sd, cu_seqlens=cu)
+        if out_dtype == torch.bfloat16:
+            assert_close_bf16_out(np32(o), ro[0], TOL[K.to_dtype(dtype)], "out step %d" % step)
+        else:
+            assert_close(np32(o), ro[0], TOL[K.to_dtype(dtype)], "out step %d" % step)
+    assert_close(np32(Sg), Sd, TOL[K.to_dtype(dtype)], "S")
+
+
+# ---- full-size workloads, sampled ----------------------------------------------------------
+
+@pytest.mark.slow
+def test_bf16_t128k_h32_sampled_heads():
+    w = K.WORKLOADS["bf16_t128k_h32"]
+    d = K.make_prefill(w, device=DEV)
+    _run_check(d, TOL[torch.bfloat16], heads=[0, 13, 31])
+
+
+@pytest.mark.slow
+def test_bf16_varlen8_262k_h32_sampled_sequences():
+    w = K.WORKLOADS["bf16_varlen8_262k_h32"]
+    d = K.make_prefill(w, device=DEV)
+    g = d
+    out, Sf = kda.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], S0=g["S0"],
+                            cu_seqlens=g["cu_seqlens"])
+    assert kda.workspace_status(kda.chunk_fwd.last_workspace) == kda.KDA_OK
+    cu = d["cu_seqlens"].tolist()
+    for n, h in [(1, 0), (0, 21), (7, 31)]:
+        sl = slice(cu[n], cu[n + 1])
+        sub = {x: d[x][:, sl][:, :, [h]] for x in ("q", "k", "v", "log_alpha", "beta")}
+        sub["S0"] = d["S0"][n:n + 1, [h]]
+        sub["cu_seqlens"] = None
+        ro, rs = oracle_prefill(sub)
+        assert_close(np32(out[:, sl][:, :, [h]]), ro, TOL[torch.bfloat16], "out seq %d head %d" % (n, h))
+        assert_close(np32(Sf[n:n + 1, [h]]), rs, TOL[torch.bfloat16], "S_final seq %d head %d" % (n, h))
+
+
+@pytest.mark.slow
+def test_decode_n256_h32_1000_steps_sampled():
+    w = K.WORKLOADS["decode_n256_h32"]
+    S = K.make_decode_state(w, device=DEV)
+    pairs = [(0, 0), (3, 17), (100, 5), (128, 31), (255, 0), (255, 31), (17, 9), (200, 22)]
+    ni = torch.tensor([p[0] for p in pairs])
+    hi = torch.tensor([p[1] for p in pairs])
+    Sd = S[ni, hi].double().cpu().numpy()[:, None]          # [P, 1, dk, dv]
+    cu = np.arange(len(pairs) + 1)
+    tol = TOL[torch.bfloat16]
+    for step in range(w.decode_steps):
+        x = K.make_decode_step(w, step, device=DEV)
+        o = kda.decode_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S)
+        sub = {n: np32(x[n][ni, hi]) for n in ("q", "k", "v", "log_alpha", "beta")}
+        ro, Sd = ref.forward(sub["q"][None, :, None], sub["k"][None, :, None], sub["v"][None, :, None],
+                             sub["log_alpha"][None, :, None], sub["beta"][None, :, None],
+                             S0=Sd, cu_seqlens=cu)
+        if step % 50 == 49:
+            assert_close(np32(o[ni, hi]), ro[0, :, 0], tol, "out step %d" % step)
+    assert_close(np32(S[ni, hi]), Sd[:, 0], tol, "S after 1000 steps")
