@@ -82,6 +82,7 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v,
     a.status = (int32_t *)workspace;
     a.scratch = (unsigned char *)workspace + kStatusBytes;
     a.scratch_bytes = workspace_bytes - kStatusBytes;
+    if (dtype == KDA_BF16 && chunk_tc_supported(a)) return map_cuda(launch_chunk_tc(a, out_dtype, st));
     return map_cuda(launch_chunk_fp32(a, dtype, out_dtype, st));
 }
 

@@ -66,6 +66,10 @@ struct PrefillArgs {
 cudaError_t launch_chunk_fp32(const PrefillArgs &a, kda_dtype_t dtype, kda_dtype_t out_dtype,
                               cudaStream_t stream);
 
+// Tensor-core (tcgen05) chunk path for bf16 q/k/v; fp32 state and accumulation.
+bool chunk_tc_supported(const PrefillArgs &a);
+cudaError_t launch_chunk_tc(const PrefillArgs &a, kda_dtype_t out_dtype, cudaStream_t stream);
+
 // Decode step (memory-bound state update in place).
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,
                           const float *beta, float *S, void *out, int N, int H,

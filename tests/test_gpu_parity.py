@@ -216,3 +216,19 @@ def test_decode_n256_h32_1000_steps_sampled():
         if step % 50 == 49:
             assert_close(np32(o[ni, hi]), ro[0, :, 0], tol, "out step %d" % step)
     assert_close(np32(S[ni, hi]), Sd[:, 0], tol, "S after 1000 steps")
+
+
+def test_tensor_core_path_reports_out_of_range_decay():
+    """bf16 inputs run on f16 tensor-core operands, which need the decay accumulated over one
+    64-token chunk to stay above e^-10.4 per channel; stronger decay is reported, not hidden."""
+    w = K.Workload("strong_decay", B=1, T=128, H=2, dtype="bf16", alpha_lo=0.5, alpha_hi=0.6)
+    d = to_device(K.make_prefill(w, seed=11), DEV)
+    kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"])
+    assert kda.workspace_status(kda.chunk_fwd.last_workspace) == kda.KDA_ERR_UNSUPPORTED
+    # the fp32 path covers it (cumulative log-decay down to about -80 per chunk)
+    f = {x: (d[x].float() if x in ("q", "k", "v") else d[x]) for x in ("q", "k", "v", "log_alpha", "beta")}
+    out, Sf = kda.chunk_fwd(f["q"], f["k"], f["v"], f["log_alpha"], f["beta"])
+    assert kda.workspace_status(kda.chunk_fwd.last_workspace) == kda.KDA_OK
+    ro, rs = oracle_prefill(f)
+    assert_close(np32(out), ro, TOL[torch.float32], "out")
+    assert_close(np32(Sf), rs, TOL[torch.float32], "S_final")
