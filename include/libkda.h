@@ -115,6 +115,33 @@ kda_status_t kda_decode_step(const void *q, const void *k, const void *v,
                              int N, int H, int dk, int dv, kda_dtype_t dtype,
                              kda_dtype_t out_dtype, void *stream);
 
+/* Capacity of the library-owned scratch array used by kda_chunk_fwd_noalloc (bytes). */
+#define KDA_NOALLOC_SCRATCH_BYTES 4096
+
+/* kda_chunk_fwd without a workspace argument, for callers that cannot allocate device memory:
+ * code running while a CUDA graph is being captured (allocating there is not allowed and would
+ * break the capture), plug-ins whose host runtime owns all device memory and passes in only the
+ * input and output buffers, and memory-capped servers that may not grow their footprint per call.
+ * The pages describe no such entry point; it has no counterpart there.
+ *
+ * Arguments, layouts and results are those of kda_chunk_fwd; the caller still passes (and owns)
+ * every input and output. Instead of a workspace, the library uses a static device array of
+ * KDA_NOALLOC_SCRATCH_BYTES that every GPU on which the library is loaded holds until the process
+ * exits. The first call on a device looks up that array's device address (with the device
+ * current) and caches it; make that first call before any stream capture begins. Sizes whose
+ * scratch need (kda_chunk_fwd_workspace_size) exceeds the array are refused with
+ * KDA_ERR_UNSUPPORTED. The function calls no cudaMalloc, cudaFree or other allocating routine.
+ * The array is shared by every call and keeps the last call's contents; each call clears its
+ * status header first. Calls whose work overlaps on the GPU (for example on two streams) race
+ * on that shared array: serialise them. Device-side check results (cu_seqlens contents, the
+ * tensor-core decay range) are written to that shared status header and are not returned. */
+kda_status_t kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
+                                   const float *log_alpha, const float *beta,
+                                   const float *S0, const int32_t *cu_seqlens,
+                                   void *out, float *S_final,
+                                   int B, int T, int H, int N, int dk, int dv,
+                                   kda_dtype_t dtype, kda_dtype_t out_dtype, void *stream);
+
 /* Waits for `stream`, then copies the workspace status word to *status
  * (KDA_OK when every device-side check passed). */
 kda_status_t kda_workspace_status(const void *workspace, void *stream, int32_t *status);

@@ -32,7 +32,7 @@ _lib = None
 
 # Every entry point declared in include/libkda.h.
 EXPORTS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
-           "kda_workspace_status", "kda_status_string", "kda_version")
+           "kda_workspace_status", "kda_status_string", "kda_version", "kda_chunk_fwd_noalloc")
 
 
 class KDAError(RuntimeError):
@@ -62,6 +62,8 @@ def load():
     lib.kda_status_string.argtypes = [I]
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_version.restype = I
+    lib.kda_chunk_fwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P]
+    lib.kda_chunk_fwd_noalloc.restype = I
     _lib = lib
     return lib
 
@@ -153,3 +155,20 @@ def decode_step(q, k, v, log_alpha, beta, S, out=None, out_dtype=torch.float32):
     if st != KDA_OK:
         raise KDAError(st, "kda_decode_step")
     return out
+
+
+def chunk_fwd_noalloc(q, k, v, log_alpha, beta, out, S_final=None, S0=None, cu_seqlens=None):
+    """``kda_chunk_fwd_noalloc``: the chunked prefill without a workspace, for callers that may not
+    allocate device memory (for example while a CUDA graph is being captured). ``out`` (and
+    ``S_final`` if wanted) must be given; nothing is allocated here or in the library."""
+    lib = load()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = B if cu_seqlens is None else cu_seqlens.shape[0] - 1
+    _need_cuda(q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final)
+    st = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                                   _ptr(cu_seqlens), _ptr(out), _ptr(S_final), B, T, H, N, dk, dv,
+                                   _dtype_code(q), _dtype_code(out), _stream(q.device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_fwd_noalloc")
+    return out, S_final
