@@ -331,6 +331,30 @@ def run_decode(kda, dev, pk, ws, local, args):
             "gpu_launches": nsteps, "clocks": clk.summary()}
 
 
+def run_profile_case(args):
+    """One small invocation for Nsight Compute captures: `prefill` runs kda_chunk_fwd on the
+    first `--tokens` tokens of the 32-head bf16 workload (inputs > L2, a few GB at most) twice;
+    `decode` runs 8 decode steps of the 256 x 32 decode workload."""
+    import kimi_delta_attention_25_b200 as kda
+    kda.load()
+    dev = torch.device("cuda", 0)
+    if args.profile == "prefill":
+        w = K.WORKLOADS[WORKLOAD]
+        d = K.make_prefill(w, device=dev, T=args.tokens)
+        for _ in range(2):
+            kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"])
+        torch.cuda.synchronize()
+        assert kda.workspace_status(kda.chunk_fwd.last_workspace) == kda.KDA_OK
+    else:
+        w = K.WORKLOADS[DECODE]
+        S = K.make_decode_state(w, device=dev)
+        xs = [K.make_decode_step(w, s, device=dev) for s in range(8)]
+        for x in xs:
+            kda.decode_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S)
+        torch.cuda.synchronize()
+    print("profile case %s done" % args.profile)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -338,7 +362,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["prefill", "decode"], default=None,
+                    help="run one small case for an Nsight Compute capture instead of the benchmark")
+    ap.add_argument("--tokens", type=int, default=32768, help="tokens of the --profile prefill case")
     args = ap.parse_args()
+    if args.profile:
+        run_profile_case(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
