@@ -131,11 +131,8 @@ def barrier(ws):
 
 
 def max_over_ranks(x, ws):
-    if ws == 1:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
+    from kimi_delta_attention_25_b200 import shard
+    return shard.max_over_ranks(x, device="cuda") if ws > 1 else x
 
 
 def time_loop(fn, steps, warmup, ws):
@@ -220,7 +217,8 @@ def run_native(args):
     torch.cuda.set_device(dev)
     pk = peaks()
     w = K.WORKLOADS[WORKLOAD]
-    d = K.make_prefill(w, device=dev, seed=w.seed + rank)
+    from kimi_delta_attention_25_b200 import shard
+    d = K.make_prefill(w, device=dev, seed=shard.rank_seed(w.seed, rank))
     B, T, H = w.B, w.T, w.H
     out = torch.empty(B, T, H, D, dtype=torch.float32, device=dev)
     Sf = torch.empty(B, H, D, D, dtype=torch.float32, device=dev)

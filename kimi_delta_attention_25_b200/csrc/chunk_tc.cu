@@ -1,5 +1,5 @@
-// chunk_tc.cu -- chunkwise KDA prefill on the sm_100a tensor cores (tcgen05 + TMEM + TMA) for
-// bf16 q/k/v: f16 MMA operands, fp32 accumulation and an fp32 inter-chunk state.
+// chunk_tc.cu -- chunkwise KDA prefill on the sm_100a tensor cores (tcgen05 + TMEM) for bf16
+// q/k/v: f16 MMA operands, fp32 accumulation and an fp32 inter-chunk state.
 //
 // Why f16 operands: every product below rounds its operands once; with bf16's 8-bit significand
 // the nine rounded operands together put the worst output 3-5% of RMS away from the exact result
@@ -14,26 +14,27 @@
 //   Kt = K f,  Qt = Q f,  Kend = K b,  Kh = K b / gamma (= K e^{-g})
 //   A  = StrictLower(diag(beta) Kt Kh^T),  M = tril(Qt Kh^T),  Tb = (I + A)^{-1} diag(beta)
 //   W  = Tb Kt;   U = Tb V - W S;   O = Qt S + M U;   S <- Diag(gamma) S + Kend^T U
-// f and b are running products of alpha = exp(log_alpha) (forward and backward within the chunk),
-// so every factor is <= 1 except 1/gamma.
+// f and b are running products of alpha = exp(log_alpha) (forward and backward within the chunk).
 //
-// Work split: one CTA (128 threads, one warpgroup) per (sequence, head, 32-column block of d_v).
-// The value columns of S evolve independently, so the four blocks of a head never communicate;
-// each recomputes the d_v-independent part of the chunk. The chunk loop is sequential per CTA:
-//   TMA (q, k, v block into a 2-stage ring; log_alpha single-buffered) ->
-//   elementwise decay scaling (CUDA cores, fp32) ->
-//   P1: [Qt; Kt] Kh^T                   (UMMA M=128 N=64  K=128) -> A (fp32 smem), M (f16 smem)
-//   T = (I + A)^{-1} by 16x16 blocks    (CUDA cores, fp32)       -> Tb (f16 smem)
-//   P3: [Tb; 0] Kt                      (UMMA M=128 N=128 K=64)  -> W (f16 smem)
-//   S1: [W; Qt] S - [Tb; 0] V           (UMMA M=128 N=32, K=128 then 64) -> -U | Qt S
-//   S2: Kend^T U -> D7 ;  MU: [0; M] U accumulated onto Qt S  (UMMA M=128 N=32 K=64)
-//   epilogue: S <- gamma S + D7 (fp32 registers, thread = key channel), O -> out
-// Operand tiles use the 128-byte (64-byte for 32-wide tiles) swizzled canonical layouts; stacked
-// operands ([Qt; Kt], [W; Qt], [Tb; 0], [0; M]) are contiguous row ranges of one region so that a
-// single M=128 instruction covers both halves.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
+// Work split: one CTA per (sequence, head, 32-column block of d_v). The value columns of S evolve
+// independently, so the four blocks of a head never communicate; each recomputes the
+// d_v-independent part of a chunk. Inside a CTA two warp groups run a two-stage pipeline:
+//
+//   prep group (8 warps) for chunk c+1            scan group (4 warps) for chunk c
+//   --------------------------------------        ------------------------------------------
+//   coalesced loads (next chunk prefetched         S1: D5 += [W; Qt] S          (M=128,N=32,K=128)
+//     to L2 one chunk ahead)                       U  = -(D5 rows 0-63) -> f16
+//   decay scaling (fp32) -> Kt Qt Kh Kend (f16)    S2: D7 = Kend^T U            (M=128,N=32,K=64)
+//   P1: Qt Kh^T, Kt Kh^T  (two M=64, N=64, K=128)  MU: D5 += [0; M] U           (M=128,N=32,K=64)
+//   M (f16), A (fp32); T = (I + A)^{-1} (fp32,     S <- gamma S + D7 (fp32 registers), S -> f16
+//     16x16 diagonal blocks + register-tiled       O = D5 rows 64-127 -> out
+//     block products); Tb = T diag(beta) (f16)
+//   P3: [Tb; 0] Kt -> W;  seed D5 = -[Tb; 0] V
+//
+// Operands produced for the scan (W, Qt, Tb, M, Kend, V and the seeded accumulator) are double
+// buffered by chunk parity; `ready` hands a parity to the scan group and `free` returns it.
+// Stacked operands ([W; Qt], [Tb; 0], [0; M]) are contiguous row ranges of one swizzled region so
+// that one M=128 instruction covers both halves.
 #include "kda_internal.cuh"
 #include "sm100.cuh"
 
@@ -42,54 +43,60 @@ namespace {
 
 using namespace sm100;
 
-constexpr int NT = 128;
 constexpr int C = kChunk;          // 64
 constexpr int DK = kHeadDim;       // 128
 constexpr int DVB = 32;            // value columns per CTA
+constexpr int SG_THREADS = 128;    // scan group: warps 0-3
+constexpr int PG_THREADS = 256;    // prep group: warps 4-11
+constexpr int NT = SG_THREADS + PG_THREADS;
 
-// ---- shared memory plan (byte offsets from a 1024-byte aligned base)
-constexpr uint32_t X_REGION = 192 * 128;              // rows 0-63 W, 64-127 Qt, 128-191 Kt
-constexpr uint32_t X_BYTES = 2 * X_REGION;            // two 64-channel halves
-constexpr uint32_t V_BYTES = C * DVB * 2;             // 4 KiB, 64-byte rows
-constexpr uint32_t OFF_X0 = 0;
-constexpr uint32_t OFF_X1 = OFF_X0 + X_BYTES;         // 49152
-constexpr uint32_t OFF_V0 = OFF_X1 + X_BYTES;         // 98304
-constexpr uint32_t OFF_V1 = OFF_V0 + V_BYTES;
-constexpr uint32_t OFF_LA = OFF_V1 + V_BYTES;         // 106496, 32 KiB log_alpha / later A, T
-constexpr uint32_t LA_BYTES = 34 * 1024;
-constexpr uint32_t OFF_KH = OFF_LA + LA_BYTES;        // Kh: two halves of 64 x 128 B
-constexpr uint32_t OFF_KE = OFF_KH + 16384;           // Kend
-constexpr uint32_t OFF_Y = OFF_KE + 16384;            // rows 0-63 Tb, 64-127 zero, 128-191 M
-constexpr uint32_t OFF_SB = OFF_Y + 192 * 128;        // S f16, 128 rows x 64 B
-constexpr uint32_t OFF_UB = OFF_SB + DK * DVB * 2;    // U f16, 64 rows x 64 B
-constexpr uint32_t OFF_TOT = OFF_UB + C * DVB * 2;    // 8 x 128 fp32 row-block products
-constexpr uint32_t OFF_GAM = OFF_TOT + 8 * 128 * 4;   // 128 fp32
-constexpr uint32_t OFF_BET = OFF_GAM + 128 * 4;       // 64 fp32
-constexpr uint32_t OFF_TMP = OFF_BET + 64 * 4;        // 3 x 16 x 16 fp32 scratch for the inverse
-constexpr uint32_t OFF_BAR = OFF_TMP + 3 * 256 * 4;   // mbarriers
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 64;
-constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;    // alignment slack
-static_assert(SMEM_ALLOC <= 232448, "shared memory plan exceeds 227 KiB");
-
-constexpr int LDA = 65;            // fp32 row stride of A and T (in the log_alpha region)
-constexpr uint32_t OFF_AF = 0;                     // within OFF_LA
-constexpr uint32_t OFF_TF = 64 * LDA * 4;          // 16640
-
-constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t TM_D1 = 0;      // 64 cols: [Qt;Kt] Kh^T
-constexpr uint32_t TM_D3 = 64;     // 128 cols: [Tb;0] Kt
-constexpr uint32_t TM_D5 = 192;    // 32 cols: -U | O
-constexpr uint32_t TM_D7 = 224;    // 32 cols: Kend^T U
-
-constexpr uint32_t TX_STAGE = 4 * 8192 + V_BYTES;  // q, k halves + v block
 // Operands are rounded to f16 (11-bit significand) for the tensor cores: the largest one, Kh =
 // K e^{-g}, must stay finite, so the decay accumulated over one chunk must keep e^{g} above
 // 2^-15 per channel (cumulative log-decay >= -10.4). Chunks beyond that report UNSUPPORTED.
 constexpr float kMinChunkDecay = 3.0517578125e-05f;
-constexpr uint32_t TX_LA = C * DK * 4;
+
+// ---- shared memory plan (byte offsets from a 1024-byte aligned base)
+constexpr uint32_t X_HALF = 128 * 128;                 // per 64-channel half: rows 0-63 W, 64-127 Qt
+constexpr uint32_t X_BYTES = 2 * X_HALF;
+constexpr uint32_t Y_BYTES = 192 * 128;                // rows 0-63 Tb, 64-127 zero, 128-191 M
+constexpr uint32_t KE_BYTES = 2 * 64 * 128;            // Kend, two halves
+constexpr uint32_t V_BYTES = C * DVB * 2;              // v block (f16), 64-byte rows
+constexpr uint32_t OFF_X0 = 0;
+constexpr uint32_t OFF_X1 = OFF_X0 + X_BYTES;
+constexpr uint32_t OFF_Y0 = OFF_X1 + X_BYTES;
+constexpr uint32_t OFF_Y1 = OFF_Y0 + Y_BYTES;
+constexpr uint32_t OFF_KE0 = OFF_Y1 + Y_BYTES;
+constexpr uint32_t OFF_KE1 = OFF_KE0 + KE_BYTES;
+constexpr uint32_t OFF_V0 = OFF_KE1 + KE_BYTES;
+constexpr uint32_t OFF_V1 = OFF_V0 + V_BYTES;
+constexpr uint32_t OFF_KT = OFF_V1 + V_BYTES;          // Kt (f16), two halves
+constexpr uint32_t OFF_KH = OFF_KT + 16384;            // Kh (f16); after P1: A^T (fp32, column-major)
+constexpr uint32_t OFF_TF = OFF_KH + 16384;            // T (fp32, row-major)
+constexpr uint32_t OFF_SB = OFF_TF + 16384;            // S (f16), 128 rows x 64 B
+constexpr uint32_t OFF_UB = OFF_SB + DK * DVB * 2;     // U (f16), 64 rows x 64 B
+constexpr uint32_t OFF_PS = OFF_UB + C * DVB * 2;      // block-product scratch of the inverse (fp32)
+constexpr uint32_t OFF_GAM = OFF_PS + 32 * 32 * 4;     // gamma, 2 x 128 fp32
+constexpr uint32_t OFF_BET = OFF_GAM + 2 * 128 * 4;    // beta, 64 fp32
+constexpr uint32_t OFF_BAR = OFF_BET + 64 * 4;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 128;
+constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
+static_assert(SMEM_ALLOC <= 232448, "shared memory plan exceeds 227 KiB");
+static_assert((OFF_Y0 | OFF_Y1 | OFF_KE0 | OFF_KE1 | OFF_KT | OFF_KH | OFF_SB | OFF_UB) % 1024 == 0,
+              "swizzled operand regions must be 1024-byte aligned");
+
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_D1A = 0;     // 64 cols, M=64 layout: Qt Kh^T
+constexpr uint32_t TM_D1B = 64;    // 64 cols, M=64 layout: Kt Kh^T
+constexpr uint32_t TM_D3 = 128;    // 128 cols: [Tb; 0] Kt (rows 0-63 = W)
+constexpr uint32_t TM_D5 = 256;    // 2 x 32 cols: -U | O per chunk parity
+constexpr uint32_t TM_D7 = 320;    // 32 cols: Kend^T U
+
+// mbarrier slots
+enum { B_READY = 0, B_FREE = 2, B_P1 = 4, B_P3 = 5, B_S1 = 6, B_S2 = 7, B_MU = 8, N_BARS = 9 };
 
 struct TcParams {
-    const float *beta, *S0;
+    const __nv_bfloat16 *q, *k, *v;
+    const float *log_alpha, *beta, *S0;
     const int32_t *cu_seqlens;
     void *out;
     float *S_final;
@@ -97,482 +104,541 @@ struct TcParams {
     int32_t *status;
 };
 
-__device__ __forceinline__ float bf2f(uint16_t x) { return __uint_as_float((uint32_t)x << 16); }
-
-// unit lower-triangular inverse T = (I + A)^{-1}, A strictly lower (fp32, row stride LDA),
-// by 16 x 16 blocks: diagonal blocks by forward substitution, then block diagonals 1..3 with
-// T_ij = -T_ii * sum_{k=j}^{i-1} L_ik T_kj. All 128 threads participate; ends synchronised.
-__device__ void unit_lower_inverse(const float *Af, float *Tf, float *tmp, int tid)
-{
-    // diagonal blocks: thread -> (block b, column j)
-    if (tid < 64) {
-        const int b = tid >> 4, j = tid & 15, o = 16 * b;
-        float x[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float v = (r == j) ? 1.f : 0.f;
-#pragma unroll
-            for (int i = 0; i < r; ++i) v -= Af[(o + r) * LDA + o + i] * x[i];
-            x[r] = (r < j) ? 0.f : v;
-        }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) Tf[(o + r) * LDA + o + j] = x[r];
-    }
-    // zero the strictly upper blocks so later full 16-term products stay exact
-    for (int idx = tid; idx < 64 * 64; idx += NT) {
-        const int r = idx >> 6, cidx = idx & 63;
-        if ((cidx >> 4) > (r >> 4)) Tf[r * LDA + cidx] = 0.f;
-    }
-    __syncthreads();
-    for (int d = 1; d <= 3; ++d) {
-        const int nb = 4 - d;                  // blocks (i, i-d), i = d..3
-        // P_i = sum_{k=i-d}^{i-1} L_ik T_k,(i-d)
-        for (int e = tid; e < nb * 256; e += NT) {
-            const int q = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-            const int i = d + q, j = i - d;
-            float acc = 0.f;
-            for (int kb = j; kb < i; ++kb) {
-#pragma unroll
-                for (int x = 0; x < 16; ++x)
-                    acc += Af[(16 * i + rr) * LDA + 16 * kb + x] * Tf[(16 * kb + x) * LDA + 16 * j + cc];
-            }
-            tmp[q * 256 + rr * 16 + cc] = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < nb * 256; e += NT) {
-            const int q = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-            const int i = d + q, j = i - d;
-            float acc = 0.f;
-#pragma unroll
-            for (int x = 0; x < 16; ++x)
-                acc += Tf[(16 * i + rr) * LDA + 16 * i + x] * tmp[q * 256 + x * 16 + cc];
-            Tf[(16 * i + rr) * LDA + 16 * j + cc] = -acc;
-        }
-        __syncthreads();
-    }
+__device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+__device__ __forceinline__ uint4 ldg_nc(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+__device__ __forceinline__ float4 ldg_nc_f4(const float *p) {
+    const uint4 r = ldg_nc(p);
+    return make_float4(__uint_as_float(r.x), __uint_as_float(r.y), __uint_as_float(r.z), __uint_as_float(r.w));
 }
 
-template <typename T, typename TO>
+// Unit lower-triangular inverse T = (I + A)^{-1} for a 64 x 64 strictly lower A held column-major
+// (AT[c * 64 + r] = A[r][c]); T is written row-major (T[r * 64 + c]). Diagonal 16 x 16 blocks by
+// forward substitution in registers; then T_{b+1,b} = -T_{b+1,b+1} A_{b+1,b} T_{b,b} inside each
+// 32 x 32 half, then T_{hi,lo} = -T_hi A_{hi,lo} T_lo for the off-diagonal 32 x 32 block.
+// Called by the 256 prep threads (pt = 0..255); ends synchronised.
+__device__ __forceinline__ void prep_inverse(int pt, const float *AT, float *Tf, float *Ps)
+{
+    const int pw = pt >> 5, lane = pt & 31;
+    if (pw < 4) {
+        if (lane < 16) {
+            const int o = 16 * pw, j = lane;
+            float xv[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) xv[r] = (r == j) ? 1.f : 0.f;
+#pragma unroll
+            for (int i = 0; i < 15; ++i) {
+                float col[16];
+                const float4 *cp = reinterpret_cast<const float4 *>(AT + (o + i) * 64 + o);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 t = cp[u];
+                    col[4 * u] = t.x; col[4 * u + 1] = t.y; col[4 * u + 2] = t.z; col[4 * u + 3] = t.w;
+                }
+                const float xi = xv[i];
+#pragma unroll
+                for (int r = i + 1; r < 16; ++r) xv[r] -= col[r] * xi;
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) Tf[(o + r) * 64 + o + j] = xv[r];
+        }
+    } else {
+        // zero the strictly upper 16 x 16 blocks of T
+        for (int e = pt - 128; e < 64 * 64; e += 128) {
+            const int r = e >> 6, c = e & 63;
+            if ((c >> 4) > (r >> 4)) Tf[e] = 0.f;
+        }
+    }
+    named_bar_sync(1, PG_THREADS);
+    // level 1a: P_b = A_{b+1,b} T_{b,b} for b = 0, 2 (two outputs per thread)
+    {
+        const int blk = pt >> 7, idx = pt & 127, r = idx >> 3, c0 = (idx & 7) * 2;
+        const int b = 2 * blk;
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float a = AT[(16 * b + k) * 64 + 16 * (b + 1) + r];
+            const float2 t = *reinterpret_cast<const float2 *>(Tf + (16 * b + k) * 64 + 16 * b + c0);
+            a0 += a * t.x;
+            a1 += a * t.y;
+        }
+        *reinterpret_cast<float2 *>(Ps + blk * 256 + r * 16 + c0) = make_float2(a0, a1);
+    }
+    named_bar_sync(1, PG_THREADS);
+    // level 1b: T_{b+1,b} = -T_{b+1,b+1} P_b
+    {
+        const int blk = pt >> 7, idx = pt & 127, r = idx >> 3, c0 = (idx & 7) * 2;
+        const int b = 2 * blk, o = 16 * (b + 1);
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float t = Tf[(o + r) * 64 + o + k];
+            const float2 pv = *reinterpret_cast<const float2 *>(Ps + blk * 256 + k * 16 + c0);
+            a0 += t * pv.x;
+            a1 += t * pv.y;
+        }
+        *reinterpret_cast<float2 *>(Tf + (o + r) * 64 + 16 * b + c0) = make_float2(-a0, -a1);
+    }
+    named_bar_sync(1, PG_THREADS);
+    // level 2a: P = A[32:64, 0:32] T[0:32, 0:32] (four outputs per thread)
+    {
+        const int r = pt >> 3, c0 = (pt & 7) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+            const float a = AT[k * 64 + 32 + r];
+            const float4 t = *reinterpret_cast<const float4 *>(Tf + k * 64 + c0);
+            acc.x += a * t.x; acc.y += a * t.y; acc.z += a * t.z; acc.w += a * t.w;
+        }
+        *reinterpret_cast<float4 *>(Ps + r * 32 + c0) = acc;
+    }
+    named_bar_sync(1, PG_THREADS);
+    // level 2b: T[32:64, 0:32] = -T[32:64, 32:64] P
+    {
+        const int r = pt >> 3, c0 = (pt & 7) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+            const float t = Tf[(32 + r) * 64 + 32 + k];
+            const float4 pv = *reinterpret_cast<const float4 *>(Ps + k * 32 + c0);
+            acc.x += t * pv.x; acc.y += t * pv.y; acc.z += t * pv.z; acc.w += t * pv.w;
+        }
+        *reinterpret_cast<float4 *>(Tf + (32 + r) * 64 + c0) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+    }
+    named_bar_sync(1, PG_THREADS);
+}
+
+// =================================================================================== kernel
+template <typename TO>
 __global__ void __launch_bounds__(NT, 1)
-chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
-                TcParams p)
+chunk_tc_kernel(TcParams p)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int jb = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
     const int j0 = jb * DVB;
     const int H = p.H;
 
-    uint64_t *bar_full = reinterpret_cast<uint64_t *>(sm + OFF_BAR);       // [2]
-    uint64_t *bar_la = bar_full + 2;
-    uint64_t *bar_mma = bar_full + 3;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_full + 4);
-    int *abort_flag = reinterpret_cast<int *>(bar_full + 5);
-    float *tot = reinterpret_cast<float *>(sm + OFF_TOT);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + N_BARS);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + N_BARS) + 1;
     float *gam = reinterpret_cast<float *>(sm + OFF_GAM);
     float *bet = reinterpret_cast<float *>(sm + OFF_BET);
-    float *Af = reinterpret_cast<float *>(sm + OFF_LA + OFF_AF);
-    float *Tf = reinterpret_cast<float *>(sm + OFF_LA + OFF_TF);
-    float *tmpf = reinterpret_cast<float *>(sm + OFF_TMP);
-    const uint32_t sbase = smem_u32(sm);
 
     int64_t t0, t1;
-    const bool ok_span = sequence_span(p.cu_seqlens, n, p.N, p.T, &t0, &t1, p.status);
-    if (!ok_span) return;                                  // uniform across the CTA
+    if (!sequence_span(p.cu_seqlens, n, p.N, p.T, &t0, &t1, p.status)) return;   // uniform
     const int nchunks = (int)((t1 - t0 + C - 1) / C);
 
     if (warp == 0) { tmem_alloc(tmem_slot, TMEM_COLS); tmem_relinquish(); }
     if (tid == 0) {
-        mbar_init(&bar_full[0], 1);
-        mbar_init(&bar_full[1], 1);
-        mbar_init(bar_la, 1);
-        mbar_init(bar_mma, 1);
+        for (int i = 0; i < N_BARS; ++i) mbar_init(&bars[i], 1);
         *abort_flag = 0;
         fence_mbar_init();
-        tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v); tma_prefetch_desc(&tm_la);
     }
-    // zero block of Y (rows 64-127) -- stays zero for the whole kernel
-    for (int i = tid; i < 64 * 128 / 16; i += NT)
-        reinterpret_cast<uint4 *>(sm + OFF_Y + 64 * 128)[i] = make_uint4(0, 0, 0, 0);
-    // initial state: thread = key channel c, 32 fp32 columns in registers
-    float S[DVB];
-    {
-        const size_t sidx = (((size_t)n * H + h) * DK + tid) * DK + j0;
-#pragma unroll
-        for (int j = 0; j < DVB; j += 4) {
-            float4 v = p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + sidx + j) : make_float4(0, 0, 0, 0);
-            S[j] = v.x; S[j + 1] = v.y; S[j + 2] = v.z; S[j + 3] = v.w;
-        }
+    // zero blocks of both Y regions (rows 64-127), never written again
+    for (int i = tid; i < 2 * 64 * 128 / 16; i += NT) {
+        const int y = i / (64 * 128 / 16), o = i % (64 * 128 / 16);
+        reinterpret_cast<uint4 *>(sm + (y ? OFF_Y1 : OFF_Y0) + 64 * 128)[o] = make_uint4(0, 0, 0, 0);
     }
-    auto store_state_f16 = [&]() {
-        // S (f16) as the MN-major B operand of S1: row = key channel (64-byte rows, 64B swizzle)
-        unsigned char *row = sm + OFF_SB;
-#pragma unroll
-        for (int j = 0; j < DVB; j += 8) {
-            uint4 v;
-            v.x = pack_f16x2(S[j], S[j + 1]); v.y = pack_f16x2(S[j + 2], S[j + 3]);
-            v.z = pack_f16x2(S[j + 4], S[j + 5]); v.w = pack_f16x2(S[j + 6], S[j + 7]);
-            *reinterpret_cast<uint4 *>(row + sw64_offset(tid, j)) = v;
-        }
-    };
-    store_state_f16();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    uint32_t mma_phase = 0;
-    uint32_t n_full_issued[2] = {0u, 0u}, n_la_issued = 0u;      // meaningful in thread 0 only
+    auto fail = [&]() { set_status(p.status, KDA_ERR_TIMEOUT); *abort_flag = 1; };
 
-    auto issue_loads = [&](int c) {        // q, k, v of chunk c into stage c & 1
-        const int s = c & 1;
-        const int tok = (int)(t0 + (int64_t)c * C);
-        unsigned char *X = sm + (s ? OFF_X1 : OFF_X0);
-        ++n_full_issued[s];
-        mbar_arrive_expect_tx(&bar_full[s], TX_STAGE);
-        for (int kh = 0; kh < 2; ++kh) {
-            tma_load_3d(X + kh * X_REGION + 64 * 128, &tm_q, &bar_full[s], 64 * kh, h, tok);
-            tma_load_3d(X + kh * X_REGION + 128 * 128, &tm_k, &bar_full[s], 64 * kh, h, tok);
-        }
-        tma_load_3d(sm + (s ? OFF_V1 : OFF_V0), &tm_v, &bar_full[s], j0, h, tok);
-    };
-    auto issue_la = [&](int c) {
-        const int tok = (int)(t0 + (int64_t)c * C);
-        ++n_la_issued;
-        mbar_arrive_expect_tx(bar_la, TX_LA);
-        tma_load_3d(sm + OFF_LA, &tm_la, bar_la, 0, h, tok);
-    };
-    auto fail = [&]() {
-        set_status(p.status, KDA_ERR_TIMEOUT);
-        *abort_flag = 1;
-    };
-    auto wait_mma = [&]() {
-        if (!mbar_wait(bar_mma, mma_phase & 1)) fail();
-        ++mma_phase;
-        tc_fence_after();
-    };
+    if (warp >= 4) {
+        // =========================================================================== prep group
+        const int pt = tid - SG_THREADS, pw = warp - 4, q4 = warp & 3, half = pw >> 2;
+        const float LOG2E = 1.4426950408889634f;
+        float *AT = reinterpret_cast<float *>(sm + OFF_KH);
+        float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
+        float *Ps = reinterpret_cast<float *>(sm + OFF_PS);
+        uint32_t n_p1 = 0, n_p3 = 0;               // commits issued (thread 0)
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c & 1;
+            const int64_t tok0 = t0 + (int64_t)c * C;
+            const int L = (t1 - tok0 < C) ? (int)(t1 - tok0) : C;
+            unsigned char *X = sm + (s ? OFF_X1 : OFF_X0);
+            unsigned char *Y = sm + (s ? OFF_Y1 : OFF_Y0);
+            unsigned char *KE = sm + (s ? OFF_KE1 : OFF_KE0);
+            unsigned char *Vs = sm + (s ? OFF_V1 : OFF_V0);
+            if (c >= 2 && !mbar_wait(&bars[B_FREE + s], ((c >> 1) - 1) & 1)) fail();
+            tc_fence_after();
 
-    if (tid == 0 && nchunks > 0) {
-        issue_loads(0);
-        issue_la(0);
-        if (nchunks > 1) issue_loads(1);
-    }
-
-    const float LOG2E = 1.4426950408889634f;
-    int c = 0;
-    for (; c < nchunks; ++c) {
-        const int s = c & 1;
-        const int64_t tok0 = t0 + (int64_t)c * C;
-        const int L = (t1 - tok0 < C) ? (int)(t1 - tok0) : C;
-        unsigned char *X = sm + (s ? OFF_X1 : OFF_X0);
-        unsigned char *Vs = sm + (s ? OFF_V1 : OFF_V0);
-        const uint32_t aX = smem_u32(X), aV = smem_u32(Vs), aY = sbase + OFF_Y;
-
-        if (tid < C) bet[tid] = (tid < L) ? p.beta[(size_t)(tok0 + tid) * H + h] : 0.f;
-        if (!mbar_wait(&bar_full[s], (c >> 1) & 1)) fail();
-        if (!mbar_wait(bar_la, c & 1)) fail();
-
-        // ---------------- elementwise decay scaling: thread -> 8 rows x 8 channels
-        {
-            const int rb = tid >> 4, cc = tid & 15, kh = cc >> 3, lc = cc & 7;
-            const float *LA = reinterpret_cast<const float *>(sm + OFF_LA);
-            float a[8][8];
-#pragma unroll
-            for (int x = 0; x < 8; ++x) {
-                const int r = 8 * rb + x;
-                const float4 l0 = *reinterpret_cast<const float4 *>(LA + r * DK + 8 * cc);
-                const float4 l1 = *reinterpret_cast<const float4 *>(LA + r * DK + 8 * cc + 4);
-                const bool valid = r < L;
-                a[x][0] = valid ? exp2f(l0.x * LOG2E) : 1.f; a[x][1] = valid ? exp2f(l0.y * LOG2E) : 1.f;
-                a[x][2] = valid ? exp2f(l0.z * LOG2E) : 1.f; a[x][3] = valid ? exp2f(l0.w * LOG2E) : 1.f;
-                a[x][4] = valid ? exp2f(l1.x * LOG2E) : 1.f; a[x][5] = valid ? exp2f(l1.y * LOG2E) : 1.f;
-                a[x][6] = valid ? exp2f(l1.z * LOG2E) : 1.f; a[x][7] = valid ? exp2f(l1.w * LOG2E) : 1.f;
-            }
-            // local inclusive prefix and exclusive suffix products over the 8 rows
-            float pre[8][8], suf[8][8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                float run = 1.f;
-#pragma unroll
-                for (int x = 0; x < 8; ++x) { run *= a[x][e]; pre[x][e] = run; }
-                float rs = 1.f;
-#pragma unroll
-                for (int x = 7; x >= 0; --x) { suf[x][e] = rs; rs *= a[x][e]; }
-                tot[rb * 128 + 8 * cc + e] = run;
-            }
-            __syncthreads();
-            float before[8], after[8], rg[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                float bfr = 1.f, aft = 1.f;
-                for (int y = 0; y < 8; ++y) {
-                    const float tv = tot[y * 128 + 8 * cc + e];
-                    if (y < rb) bfr *= tv;
-                    if (y > rb) aft *= tv;
-                }
-                before[e] = bfr;
-                after[e] = aft;
-                const float g = bfr * pre[7][e] * aft;           // gamma = product over the chunk
-                rg[e] = 1.f / g;
-                if (rb == 0) gam[8 * cc + e] = g;
-                if (g < kMinChunkDecay) set_status(p.status, KDA_ERR_UNSUPPORTED);
-            }
-            {   // v block: bf16 -> f16 in place (16 elements per thread; layout unchanged)
-                uint4 *vv = reinterpret_cast<uint4 *>(Vs) + 2 * tid;
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    uint4 x = vv[u];
-                    x.x = bf16x2_to_f16x2(x.x); x.y = bf16x2_to_f16x2(x.y);
-                    x.z = bf16x2_to_f16x2(x.z); x.w = bf16x2_to_f16x2(x.w);
-                    vv[u] = x;
+            // ---- prefetch the next chunk's rows into L2
+            if (c + 1 < nchunks) {
+                const int64_t nt0 = tok0 + C;
+                const int nL = (t1 - nt0 < C) ? (int)(t1 - nt0) : C;
+                const int r = pt >> 2, part = pt & 3;
+                if (r < nL) {
+                    const size_t row = ((size_t)(nt0 + r) * H + h) * DK;
+                    prefetch_l2(p.log_alpha + row + 32 * part);
+                    if (part < 2) {
+                        prefetch_l2(p.q + row + 64 * part);
+                        prefetch_l2(p.k + row + 64 * part);
+                    } else if (part == 2) {
+                        prefetch_l2(p.v + row + j0);
+                    } else {
+                        prefetch_l2(p.beta + (size_t)(nt0 + r) * H + h);
+                    }
                 }
             }
-            unsigned char *Xk = X + kh * X_REGION + 128 * 128;   // k -> Kt in place
-            unsigned char *Xq = X + kh * X_REGION + 64 * 128;    // q -> Qt in place
-            unsigned char *Kh = sm + OFF_KH + kh * 8192;
-            unsigned char *Ke = sm + OFF_KE + kh * 8192;
+            // ---- beta and the v block (bf16 -> f16, 64-byte swizzled rows)
+            if (pt < C) bet[pt] = (pt < L) ? p.beta[(size_t)(tok0 + pt) * H + h] : 0.f;
+            {
+                const int r = pt >> 2, cq = (pt & 3) * 8;
+                uint4 o = make_uint4(0, 0, 0, 0);
+                if (r < L) {
+                    const uint4 raw = ldg_nc(p.v + ((size_t)(tok0 + r) * H + h) * DK + j0 + cq);
+                    o.x = bf16x2_to_f16x2(raw.x); o.y = bf16x2_to_f16x2(raw.y);
+                    o.z = bf16x2_to_f16x2(raw.z); o.w = bf16x2_to_f16x2(raw.w);
+                }
+                *reinterpret_cast<uint4 *>(Vs + sw64_offset(r, cq)) = o;
+            }
+            // ---- decay scaling: thread -> rows 4rb..4rb+3, channels 8cc..8cc+7; the 16 row blocks
+            //      of one channel chunk sit on 16 consecutive lanes
+            {
+                const int cc = pt >> 4, rb = pt & 15, kh = cc >> 3, lc = cc & 7;
+                float a[4][8];
+                uint4 kr[4], qr[4];
 #pragma unroll
-            for (int x = 0; x < 8; ++x) {
-                const int r = 8 * rb + x;
-                const uint32_t off = sw128_offset(r, 8 * lc);
-                const uint4 kraw = *reinterpret_cast<const uint4 *>(Xk + off);
-                const uint4 qraw = *reinterpret_cast<const uint4 *>(Xq + off);
-                const uint16_t *kv = reinterpret_cast<const uint16_t *>(&kraw);
-                const uint16_t *qv = reinterpret_cast<const uint16_t *>(&qraw);
-                const bool valid = r < L;
-                float kt[8], qt[8], ke[8], kc[8];
+                for (int x = 0; x < 4; ++x) {
+                    const int r = 4 * rb + x;
+                    if (r < L) {
+                        const size_t row = ((size_t)(tok0 + r) * H + h) * DK + 8 * cc;
+                        const float4 l0 = ldg_nc_f4(p.log_alpha + row);
+                        const float4 l1 = ldg_nc_f4(p.log_alpha + row + 4);
+                        kr[x] = ldg_nc(p.k + row);
+                        qr[x] = ldg_nc(p.q + row);
+                        a[x][0] = l0.x; a[x][1] = l0.y; a[x][2] = l0.z; a[x][3] = l0.w;
+                        a[x][4] = l1.x; a[x][5] = l1.y; a[x][6] = l1.z; a[x][7] = l1.w;
+                    } else {
+                        kr[x] = make_uint4(0, 0, 0, 0);
+                        qr[x] = kr[x];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) a[x][e] = 0.f;
+                    }
+                }
+                // alpha; local inclusive prefix (pre) and exclusive suffix (suf) over the 4 rows;
+                // products over the other row blocks from the neighbouring lanes
+                float pre[4][8], suf[4][8], before[8], after[8], g[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const float kk = valid ? bf2f(kv[e]) : 0.f;
-                    const float qq = valid ? bf2f(qv[e]) : 0.f;
-                    const float f = before[e] * pre[x][e];
-                    const float b = suf[x][e] * after[e];
-                    kt[e] = kk * f;
-                    qt[e] = qq * f;
-                    ke[e] = kk * b;
-                    kc[e] = ke[e] * rg[e];
+                    float run = 1.f;
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) { a[x][e] = exp2f(a[x][e] * LOG2E); run *= a[x][e]; pre[x][e] = run; }
+                    float rs = 1.f;
+#pragma unroll
+                    for (int x = 3; x >= 0; --x) { suf[x][e] = rs; rs *= a[x][e]; }
+                    float inc = run, sfx = run;
+#pragma unroll
+                    for (int o = 1; o < 16; o <<= 1) {
+                        const float u = __shfl_up_sync(0xffffffffu, inc, o, 16);
+                        const float d = __shfl_down_sync(0xffffffffu, sfx, o, 16);
+                        if (rb >= o) inc *= u;
+                        if (rb + o < 16) sfx *= d;
+                    }
+                    const float bu = __shfl_up_sync(0xffffffffu, inc, 1, 16);
+                    const float ad = __shfl_down_sync(0xffffffffu, sfx, 1, 16);
+                    before[e] = (rb == 0) ? 1.f : bu;
+                    after[e] = (rb == 15) ? 1.f : ad;
+                    g[e] = __shfl_sync(0xffffffffu, inc, 15, 16);
                 }
-                uint4 o;
-                o.x = pack_f16x2(kt[0], kt[1]); o.y = pack_f16x2(kt[2], kt[3]);
-                o.z = pack_f16x2(kt[4], kt[5]); o.w = pack_f16x2(kt[6], kt[7]);
-                *reinterpret_cast<uint4 *>(Xk + off) = o;
-                o.x = pack_f16x2(qt[0], qt[1]); o.y = pack_f16x2(qt[2], qt[3]);
-                o.z = pack_f16x2(qt[4], qt[5]); o.w = pack_f16x2(qt[6], qt[7]);
-                *reinterpret_cast<uint4 *>(Xq + off) = o;
-                o.x = pack_f16x2(ke[0], ke[1]); o.y = pack_f16x2(ke[2], ke[3]);
-                o.z = pack_f16x2(ke[4], ke[5]); o.w = pack_f16x2(ke[6], ke[7]);
-                *reinterpret_cast<uint4 *>(Ke + off) = o;
-                o.x = pack_f16x2(kc[0], kc[1]); o.y = pack_f16x2(kc[2], kc[3]);
-                o.z = pack_f16x2(kc[4], kc[5]); o.w = pack_f16x2(kc[6], kc[7]);
-                *reinterpret_cast<uint4 *>(Kh + off) = o;
-            }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (*abort_flag) break;
-        tc_fence_after();
-
-        // ---------------- P1: D1 = [Qt; Kt] Kh^T  (M=128, N=64, K=128)
-        if (tid == 0) {
-            const uint32_t id = idesc_f16(128, 64, 0, 0);
+                if (rb == 0) {
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t kh = ks >> 2, ko = (ks & 3) * 32;
-                const uint64_t ad = smem_desc(aX + kh * X_REGION + 64 * 128 + ko, 16, 1024, SW_128B);
-                const uint64_t bd = smem_desc(sbase + OFF_KH + kh * 8192 + ko, 16, 1024, SW_128B);
-                umma_ss(tmem + TM_D1, ad, bd, id, ks > 0);
-            }
-            umma_commit(bar_mma);
-        }
-        wait_mma();
-        // rows 0-63: M = tril(Qt Kh^T) -> f16 Y rows 128-191; rows 64-127: A -> fp32
-        {
-            float v[64];
-            const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16) + TM_D1;
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                float r16[16];
-                tmem_ld16(ta + 16 * q4, r16);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) v[16 * q4 + e] = r16[e];
-            }
-            if (tid < 64) {
-                const int r = tid;
-                unsigned char *row = sm + OFF_Y;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    float m8[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) m8[e] = (8 * ch + e <= r) ? v[8 * ch + e] : 0.f;
-                    uint4 o;
-                    o.x = pack_f16x2(m8[0], m8[1]); o.y = pack_f16x2(m8[2], m8[3]);
-                    o.z = pack_f16x2(m8[4], m8[5]); o.w = pack_f16x2(m8[6], m8[7]);
-                    *reinterpret_cast<uint4 *>(row + sw128_offset(128 + r, 8 * ch)) = o;
+                    for (int e = 0; e < 8; ++e) {
+                        gam[s * 128 + 8 * cc + e] = g[e];
+                        if (g[e] < kMinChunkDecay) set_status(p.status, KDA_ERR_UNSUPPORTED);
+                    }
                 }
-            } else {
-                const int r = tid - 64;
-                const float br = bet[r];
+                float rg[8];
 #pragma unroll
-                for (int i = 0; i < 64; ++i) Af[r * LDA + i] = (i < r) ? br * v[i] : 0.f;
+                for (int e = 0; e < 8; ++e) rg[e] = 1.f / g[e];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int r = 4 * rb + x;
+                    const uint32_t off = sw128_offset(r, 8 * lc);
+                    const uint32_t kw[4] = {kr[x].x, kr[x].y, kr[x].z, kr[x].w};
+                    const uint32_t qw[4] = {qr[x].x, qr[x].y, qr[x].z, qr[x].w};
+                    uint32_t okt[4], oqt[4], oke[4], okh[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int e = 2 * u;
+                        const float f0 = before[e] * pre[x][e], f1 = before[e + 1] * pre[x][e + 1];
+                        const float b0 = suf[x][e] * after[e], b1 = suf[x][e + 1] * after[e + 1];
+                        const float k0 = bf_lo(kw[u]), k1 = bf_hi(kw[u]);
+                        const float q0 = bf_lo(qw[u]), q1 = bf_hi(qw[u]);
+                        const float e0 = k0 * b0, e1 = k1 * b1;
+                        okt[u] = pack_f16x2(k0 * f0, k1 * f1);
+                        oqt[u] = pack_f16x2(q0 * f0, q1 * f1);
+                        oke[u] = pack_f16x2(e0, e1);
+                        okh[u] = pack_f16x2(e0 * rg[e], e1 * rg[e + 1]);
+                    }
+                    *reinterpret_cast<uint4 *>(sm + OFF_KT + kh * 8192 + off) = make_uint4(okt[0], okt[1], okt[2], okt[3]);
+                    *reinterpret_cast<uint4 *>(X + kh * X_HALF + 64 * 128 + off) = make_uint4(oqt[0], oqt[1], oqt[2], oqt[3]);
+                    *reinterpret_cast<uint4 *>(KE + kh * 8192 + off) = make_uint4(oke[0], oke[1], oke[2], oke[3]);
+                    *reinterpret_cast<uint4 *>(sm + OFF_KH + kh * 8192 + off) = make_uint4(okh[0], okh[1], okh[2], okh[3]);
+                }
             }
-        }
-        tc_fence_before();
-        __syncthreads();
-
-        // ---------------- T = (I + A)^{-1};  Tb = T diag(beta) -> f16 Y rows 0-63
-        unit_lower_inverse(Af, Tf, tmpf, tid);
-        {
-            const int r = tid >> 1, half = tid & 1;
-            unsigned char *row = sm + OFF_Y;
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(1, PG_THREADS);
+            if (*abort_flag) break;                // uniform: read after a group barrier
+            tc_fence_after();
+            // ---- P1: D1A = Qt Kh^T, D1B = Kt Kh^T   (M=64, N=64, K=128)
+            if (pt == 0) {
+                ++n_p1;
+                const uint32_t id = idesc_f16(64, 64, 0, 0);
+                const uint32_t aX = smem_u32(X);
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                const int c0 = 32 * half + 8 * ch;
-                float t8[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) t8[e] = (c0 + e <= r) ? Tf[r * LDA + c0 + e] * bet[c0 + e] : 0.f;
-                uint4 o;
-                o.x = pack_f16x2(t8[0], t8[1]); o.y = pack_f16x2(t8[2], t8[3]);
-                o.z = pack_f16x2(t8[4], t8[5]); o.w = pack_f16x2(t8[6], t8[7]);
-                *reinterpret_cast<uint4 *>(row + sw128_offset(r, c0)) = o;
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t kh = ks >> 2, ko = (ks & 3) * 32;
+                    const uint64_t bd = smem_desc(sbase + OFF_KH + kh * 8192 + ko, 16, 1024, SW_128B);
+                    umma_ss(tmem + TM_D1A, smem_desc(aX + kh * X_HALF + 64 * 128 + ko, 16, 1024, SW_128B), bd, id, ks > 0);
+                    umma_ss(tmem + TM_D1B, smem_desc(sbase + OFF_KT + kh * 8192 + ko, 16, 1024, SW_128B), bd, id, ks > 0);
+                }
+                umma_commit(&bars[B_P1]);
             }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        // log_alpha region (A, T) is free: prefetch the next chunk's log_alpha
-        if (tid == 0 && c + 1 < nchunks) issue_la(c + 1);
-        tc_fence_after();
-
-        // ---------------- P3: D3 = [Tb; 0] Kt  (M=128, N=128, K=64; B = Kt MN-major)
-        if (tid == 0) {
-            const uint32_t id = idesc_f16(128, 128, 0, 1);
+            if (!mbar_wait(&bars[B_P1], c & 1)) fail();
+            tc_fence_after();
+            // ---- P1 epilogue: half 0 -> M (f16, Y rows 128-191); half 1 -> A^T (fp32, column-major)
+            {
+                const uint32_t ta = tmem + ((uint32_t)(32 * q4) << 16) + (half ? TM_D1B : TM_D1A);
+                float v[64];
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t ad = smem_desc(aY + ks * 32, 16, 1024, SW_128B);
-                const uint64_t bd = smem_desc(aX + 128 * 128 + ks * 2048, X_REGION, 1024, SW_128B);
-                umma_ss(tmem + TM_D3, ad, bd, id, ks > 0);
+                for (int q = 0; q < 4; ++q) {
+                    float r16[16];
+                    tmem_ld16(ta + 16 * q, r16);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[16 * q + e] = r16[e];
+                }
+                if (lane < 16) {
+                    const int r = 16 * q4 + lane;
+                    if (half == 0) {
+#pragma unroll
+                        for (int ch = 0; ch < 8; ++ch) {
+                            uint32_t w4[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const int i = 8 * ch + 2 * u;
+                                w4[u] = pack_f16x2(i <= r ? v[i] : 0.f, i + 1 <= r ? v[i + 1] : 0.f);
+                            }
+                            *reinterpret_cast<uint4 *>(Y + sw128_offset(128 + r, 8 * ch)) =
+                                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                        }
+                    } else {
+                        const float br = bet[r];
+#pragma unroll
+                        for (int i = 0; i < 64; ++i) AT[i * 64 + r] = (i < r) ? br * v[i] : 0.f;
+                    }
+                }
             }
-            umma_commit(bar_mma);
-        }
-        wait_mma();
-        if (tid < 64) {                      // W rows -> f16 X rows 0-63 (both halves)
-            const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16) + TM_D3;
-#pragma unroll
-            for (int q8 = 0; q8 < 8; ++q8) {
-                float r16[16];
-                tmem_ld16(ta + 16 * q8, r16);
-                tmem_ld_wait();
-                const int col = 16 * q8, kh = col >> 6, cl = col & 63;
-                unsigned char *base = X + kh * X_REGION;
+            tc_fence_before();
+            named_bar_sync(1, PG_THREADS);
+            if (*abort_flag) break;
+            // ---- T = (I + A)^{-1};  Tb = T diag(beta) -> f16 Y rows 0-63
+            prep_inverse(pt, AT, Tf, Ps);
+            {
+                const int r = pt >> 2, c0 = (pt & 3) * 16;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    uint4 o;
-                    o.x = pack_f16x2(r16[8 * hh + 0], r16[8 * hh + 1]);
-                    o.y = pack_f16x2(r16[8 * hh + 2], r16[8 * hh + 3]);
-                    o.z = pack_f16x2(r16[8 * hh + 4], r16[8 * hh + 5]);
-                    o.w = pack_f16x2(r16[8 * hh + 6], r16[8 * hh + 7]);
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(tid, cl + 8 * hh)) = o;
+                    const int cb = c0 + 8 * hh;
+                    const float4 t0v = *reinterpret_cast<const float4 *>(Tf + r * 64 + cb);
+                    const float4 t1v = *reinterpret_cast<const float4 *>(Tf + r * 64 + cb + 4);
+                    const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = cb + 2 * u;
+                        w4[u] = pack_f16x2(i <= r ? tv[2 * u] * bet[i] : 0.f,
+                                           i + 1 <= r ? tv[2 * u + 1] * bet[i + 1] : 0.f);
+                    }
+                    *reinterpret_cast<uint4 *>(Y + sw128_offset(r, cb)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }
             }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(1, PG_THREADS);
+            tc_fence_after();
+            // ---- P3: D3 = [Tb; 0] Kt (M=128, N=128, K=64); seed D5[s] = -[Tb; 0] V (M=128, N=32)
+            if (pt == 0) {
+                ++n_p3;
+                const uint32_t aY = smem_u32(Y);
+                const uint32_t id3 = idesc_f16(128, 128, 0, 1);
+                const uint32_t ids = idesc_f16(128, 32, 0, 1) | (1u << 13);   // negate A
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t ad = smem_desc(aY + ks * 32, 16, 1024, SW_128B);
+                    umma_ss(tmem + TM_D3, ad, smem_desc(sbase + OFF_KT + ks * 2048, 8192, 1024, SW_128B), id3, ks > 0);
+                    umma_ss(tmem + TM_D5 + 32 * s, ad, smem_desc(smem_u32(Vs) + ks * 1024, 16, 512, SW_64B), ids, ks > 0);
+                }
+                umma_commit(&bars[B_P3]);
+            }
+            if (!mbar_wait(&bars[B_P3], c & 1)) fail();
+            tc_fence_after();
+            // ---- W epilogue: rows 0-63 of D3 (TMEM lanes 0-63) -> f16 X rows 0-63
+            if (q4 < 2) {
+                const int r = 32 * q4 + lane;
+                const uint32_t ta = tmem + ((uint32_t)(32 * q4) << 16) + TM_D3 + 64 * half;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float r16[16];
+                    tmem_ld16(ta + 16 * q, r16);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint4 o;
+                        o.x = pack_f16x2(r16[8 * hh + 0], r16[8 * hh + 1]);
+                        o.y = pack_f16x2(r16[8 * hh + 2], r16[8 * hh + 3]);
+                        o.z = pack_f16x2(r16[8 * hh + 4], r16[8 * hh + 5]);
+                        o.w = pack_f16x2(r16[8 * hh + 6], r16[8 * hh + 7]);
+                        *reinterpret_cast<uint4 *>(X + half * X_HALF + sw128_offset(r, 16 * q + 8 * hh)) = o;
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(1, PG_THREADS);
+            if (*abort_flag) break;
+            if (pt == 0) mbar_arrive(&bars[B_READY + s]);
         }
+        if (*abort_flag && pt == 0) {      // drain this thread's MMAs still in flight (bounded)
+            if (n_p1) mbar_wait(&bars[B_P1], (n_p1 - 1) & 1, 100000000LL);
+            if (n_p3) mbar_wait(&bars[B_P3], (n_p3 - 1) & 1, 100000000LL);
+        }
+    } else {
+        // =========================================================================== scan group
+        const int st = tid;                      // key channel / TMEM lane
+        float S[DVB];
+        {
+            const size_t sidx = (((size_t)n * H + h) * DK + st) * DK + j0;
+#pragma unroll
+            for (int j = 0; j < DVB; j += 4) {
+                const float4 v = p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + sidx + j) : make_float4(0, 0, 0, 0);
+                S[j] = v.x; S[j + 1] = v.y; S[j + 2] = v.z; S[j + 3] = v.w;
+            }
+        }
+        auto store_state = [&]() {
+#pragma unroll
+            for (int j = 0; j < DVB; j += 8) {
+                uint4 v;
+                v.x = pack_f16x2(S[j], S[j + 1]); v.y = pack_f16x2(S[j + 2], S[j + 3]);
+                v.z = pack_f16x2(S[j + 4], S[j + 5]); v.w = pack_f16x2(S[j + 6], S[j + 7]);
+                *reinterpret_cast<uint4 *>(sm + OFF_SB + sw64_offset(st, j)) = v;
+            }
+        };
+        store_state();
         fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-
-        // ---------------- S1: D5 = [W; Qt] S  -  [Tb; 0] V   (M=128, N=32)
-        if (tid == 0) {
+        named_bar_sync(2, SG_THREADS);
+        uint32_t n_s1 = 0, n_s2 = 0;               // commits issued (thread 0)
+        auto issue_s1 = [&](int c) -> bool {   // scan thread 0 only
+            const int s = c & 1;
+            if (!mbar_wait(&bars[B_READY + s], (c >> 1) & 1)) return false;
+            ++n_s1;
+            tc_fence_after();
+            const uint32_t aX = sbase + (s ? OFF_X1 : OFF_X0);
             const uint32_t id = idesc_f16(128, 32, 0, 1);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t kh = ks >> 2, ko = (ks & 3) * 32;
-                const uint64_t ad = smem_desc(aX + kh * X_REGION + ko, 16, 1024, SW_128B);
-                const uint64_t bd = smem_desc(sbase + OFF_SB + ks * 1024, 16, 512, SW_64B);
-                umma_ss(tmem + TM_D5, ad, bd, id, ks > 0);
+                umma_ss(tmem + TM_D5 + 32 * s, smem_desc(aX + kh * X_HALF + ko, 16, 1024, SW_128B),
+                        smem_desc(sbase + OFF_SB + ks * 1024, 16, 512, SW_64B), id, 1);
             }
-            const uint32_t idn = id | (1u << 13);            // negate A
+            umma_commit(&bars[B_S1]);
+            return true;
+        };
+        if (st == 0 && nchunks > 0 && !issue_s1(0)) fail();
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c & 1;
+            const int64_t tok0 = t0 + (int64_t)c * C;
+            const int L = (t1 - tok0 < C) ? (int)(t1 - tok0) : C;
+            const uint32_t d5 = tmem + TM_D5 + 32 * s;
+            if (!mbar_wait(&bars[B_S1], c & 1)) fail();
+            tc_fence_after();
+            // U = -(D5 rows 0-63) -> f16 MN-major [token][32]
+            if (warp < 2) {
+                const uint32_t ta = d5 + ((uint32_t)(32 * warp) << 16);
+                float u[32];
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t ad = smem_desc(aY + ks * 32, 16, 1024, SW_128B);
-                const uint64_t bd = smem_desc(aV + ks * 1024, 16, 512, SW_64B);
-                umma_ss(tmem + TM_D5, ad, bd, idn, 1);
-            }
-            umma_commit(bar_mma);
-        }
-        wait_mma();
-        if (tid < 64) {                      // U = -(rows 0-63) -> f16 MN-major [token][32]
-            const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16) + TM_D5;
-            float u[32];
-#pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-                float r16[16];
-                tmem_ld16(ta + 16 * q2, r16);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) u[16 * q2 + e] = -r16[e];
-            }
-            unsigned char *row = sm + OFF_UB;
-#pragma unroll
-            for (int j = 0; j < DVB; j += 8) {
-                uint4 o;
-                o.x = pack_f16x2(u[j], u[j + 1]); o.y = pack_f16x2(u[j + 2], u[j + 3]);
-                o.z = pack_f16x2(u[j + 4], u[j + 5]); o.w = pack_f16x2(u[j + 6], u[j + 7]);
-                *reinterpret_cast<uint4 *>(row + sw64_offset(tid, j)) = o;
-            }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-
-        // ---------------- S2: D7 = Kend^T U ;  MU: D5 += [0; M] U
-        if (tid == 0) {
-            const uint32_t id2 = idesc_f16(128, 32, 1, 1);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t ad = smem_desc(sbase + OFF_KE + ks * 2048, 8192, 1024, SW_128B);
-                const uint64_t bd = smem_desc(sbase + OFF_UB + ks * 1024, 16, 512, SW_64B);
-                umma_ss(tmem + TM_D7, ad, bd, id2, ks > 0);
-            }
-            const uint32_t idm = idesc_f16(128, 32, 0, 1);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t ad = smem_desc(aY + 64 * 128 + ks * 32, 16, 1024, SW_128B);
-                const uint64_t bd = smem_desc(sbase + OFF_UB + ks * 1024, 16, 512, SW_64B);
-                umma_ss(tmem + TM_D5, ad, bd, idm, 1);
-            }
-            umma_commit(bar_mma);
-        }
-        wait_mma();
-        {
-            // state update: thread = key channel
-            const uint32_t ta7 = tmem + ((uint32_t)(32 * warp) << 16) + TM_D7;
-            const float g = gam[tid];
-#pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-                float r16[16];
-                tmem_ld16(ta7 + 16 * q2, r16);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) S[16 * q2 + e] = g * S[16 * q2 + e] + r16[e];
-            }
-            // outputs: rows 64-127 of D5 are O for tokens 0-63
-            if (tid >= 64) {
-                const int r = tid - 64;
-                const uint32_t ta5 = tmem + ((uint32_t)(32 * warp) << 16) + TM_D5;
-                float o32[32];
-#pragma unroll
-                for (int q2 = 0; q2 < 2; ++q2) {
+                for (int q = 0; q < 2; ++q) {
                     float r16[16];
-                    tmem_ld16(ta5 + 16 * q2, r16);
+                    tmem_ld16(ta + 16 * q, r16);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) o32[16 * q2 + e] = r16[e];
+                    for (int e = 0; e < 16; ++e) u[16 * q + e] = -r16[e];
+                }
+#pragma unroll
+                for (int j = 0; j < DVB; j += 8) {
+                    uint4 o;
+                    o.x = pack_f16x2(u[j], u[j + 1]); o.y = pack_f16x2(u[j + 2], u[j + 3]);
+                    o.z = pack_f16x2(u[j + 4], u[j + 5]); o.w = pack_f16x2(u[j + 6], u[j + 7]);
+                    *reinterpret_cast<uint4 *>(sm + OFF_UB + sw64_offset(st, j)) = o;
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(2, SG_THREADS);
+            if (*abort_flag) break;                // uniform: read after a group barrier
+            tc_fence_after();
+            if (st == 0) {
+                ++n_s2;
+                const uint32_t aKE = sbase + (s ? OFF_KE1 : OFF_KE0);
+                const uint32_t aY = sbase + (s ? OFF_Y1 : OFF_Y0);
+                const uint32_t id2 = idesc_f16(128, 32, 1, 1);
+                const uint32_t idm = idesc_f16(128, 32, 0, 1);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_ss(tmem + TM_D7, smem_desc(aKE + ks * 2048, 8192, 1024, SW_128B),
+                            smem_desc(sbase + OFF_UB + ks * 1024, 16, 512, SW_64B), id2, ks > 0);
+                umma_commit(&bars[B_S2]);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_ss(d5, smem_desc(aY + 64 * 128 + ks * 32, 16, 1024, SW_128B),
+                            smem_desc(sbase + OFF_UB + ks * 1024, 16, 512, SW_64B), idm, 1);
+                umma_commit(&bars[B_MU]);
+            }
+            if (!mbar_wait(&bars[B_S2], c & 1)) fail();
+            tc_fence_after();
+            {   // S <- gamma S + Kend^T U
+                const uint32_t ta = tmem + TM_D7 + ((uint32_t)(32 * warp) << 16);
+                const float g = gam[s * 128 + st];
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    float r16[16];
+                    tmem_ld16(ta + 16 * q, r16);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) S[16 * q + e] = g * S[16 * q + e] + r16[e];
+                }
+                store_state();
+            }
+            fence_proxy_async_smem();
+            // every scan thread observes the MU commit: it also guards UB and D5[s]
+            if (!mbar_wait(&bars[B_MU], c & 1)) fail();
+            tc_fence_after();
+            if (warp >= 2) {                 // O = D5 rows 64-127 -> out
+                const int r = st - 64;
+                const uint32_t ta = d5 + ((uint32_t)(32 * warp) << 16);
+                float o32[32];
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    float r16[16];
+                    tmem_ld16(ta + 16 * q, r16);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o32[16 * q + e] = r16[e];
                 }
                 if (r < L) {
                     TO *dst = reinterpret_cast<TO *>(p.out) + ((size_t)(tok0 + r) * H + h) * DK + j0;
@@ -592,77 +658,45 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
             }
-            store_state_f16();
+            tc_fence_before();
+            named_bar_sync(2, SG_THREADS);
+            if (*abort_flag) break;
+            if (st == 0) {
+                mbar_arrive(&bars[B_FREE + s]);
+                if (c + 1 < nchunks && !issue_s1(c + 1)) fail();
+            }
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        // stage s is free again: load chunk c + 2 into it
-        if (tid == 0 && c + 2 < nchunks) issue_loads(c + 2);
-        if (*abort_flag) break;
-    }
-
-    if (p.S_final && !*abort_flag) {
-        const size_t sidx = (((size_t)n * H + h) * DK + tid) * DK + j0;
+        if (*abort_flag && st == 0) {      // drain this thread's MMAs still in flight (bounded)
+            if (n_s1) mbar_wait(&bars[B_S1], (n_s1 - 1) & 1, 100000000LL);
+            if (n_s2) {
+                mbar_wait(&bars[B_S2], (n_s2 - 1) & 1, 100000000LL);
+                mbar_wait(&bars[B_MU], (n_s2 - 1) & 1, 100000000LL);
+            }
+        }
+        if (p.S_final && !*abort_flag) {
+            const size_t sidx = (((size_t)n * H + h) * DK + st) * DK + j0;
 #pragma unroll
-        for (int j = 0; j < DVB; j += 4)
-            *reinterpret_cast<float4 *>(p.S_final + sidx + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
-    }
-    if (*abort_flag && tid == 0) {
-        // drain TMA copies that may still be in flight (bounded) before the CTA exits: wait for
-        // the last issued phase of every load barrier
-        for (int s = 0; s < 2; ++s)
-            if (n_full_issued[s]) mbar_wait(&bar_full[s], (n_full_issued[s] - 1) & 1, 100000000LL);
-        if (n_la_issued) mbar_wait(bar_la, (n_la_issued - 1) & 1, 100000000LL);
+            for (int j = 0; j < DVB; j += 4)
+                *reinterpret_cast<float4 *>(p.S_final + sidx + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-// ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 get_encode()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
-// 3-D map over a [tokens, H, 128] tensor: dims (channel, head, token), box (bx, 1, 64).
-bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize, int H, int ntok,
-              int bx, CUtensorMapSwizzle sw)
-{
-    auto enc = get_encode();
-    if (!enc) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)DK, (cuuint64_t)H, (cuuint64_t)ntok};
-    cuuint64_t strides[2] = {(cuuint64_t)DK * esize, (cuuint64_t)DK * esize * H};
-    cuuint32_t box[3] = {(cuuint32_t)bx, 1u, (cuuint32_t)C};
-    cuuint32_t estr[3] = {1u, 1u, 1u};
-    CUresult r = enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 template <typename TO>
-cudaError_t launch_typed(const PrefillArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
-                         const CUtensorMap &mv, const CUtensorMap &ml, cudaStream_t stream)
+cudaError_t launch_typed(const PrefillArgs &a, cudaStream_t stream)
 {
     TcParams p;
-    p.beta = a.beta; p.S0 = a.S0; p.cu_seqlens = a.cu_seqlens; p.out = a.out; p.S_final = a.S_final;
-    p.T = a.T; p.H = a.H; p.N = a.N; p.status = a.status;
-    auto kern = chunk_tc_kernel<__nv_bfloat16, TO>;
+    p.q = (const __nv_bfloat16 *)a.q; p.k = (const __nv_bfloat16 *)a.k; p.v = (const __nv_bfloat16 *)a.v;
+    p.log_alpha = a.log_alpha; p.beta = a.beta; p.S0 = a.S0; p.cu_seqlens = a.cu_seqlens;
+    p.out = a.out; p.S_final = a.S_final; p.T = a.T; p.H = a.H; p.N = a.N; p.status = a.status;
+    auto kern = chunk_tc_kernel<TO>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     const dim3 grid(DK / DVB, a.H, a.N);
-    kern<<<grid, NT, SMEM_ALLOC, stream>>>(mq, mk, mv, ml, p);
+    kern<<<grid, NT, SMEM_ALLOC, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -670,26 +704,15 @@ cudaError_t launch_typed(const PrefillArgs &a, const CUtensorMap &mq, const CUte
 
 bool chunk_tc_supported(const PrefillArgs &a)
 {
-    // TMA coordinates are 32-bit; the packed token axis must fit
-    return (long long)a.B * a.T < (1LL << 31) && get_encode() != nullptr;
+    (void)a;
+    return true;
 }
 
 cudaError_t launch_chunk_tc(const PrefillArgs &a, kda_dtype_t out_dtype, cudaStream_t stream)
 {
     if (a.N == 0) return cudaSuccess;
-    const int ntok = a.B * a.T;
-    if (ntok == 0) {
-        // no tokens: every sequence is empty, S_final = S0 -- handled by the fp32 path
-        return launch_chunk_fp32(a, KDA_BF16, out_dtype, stream);
-    }
-    CUtensorMap mq, mk, mv, ml;
-    if (!make_map(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, ntok, DVB, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !make_map(&ml, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.H, ntok, DK, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
-    if (out_dtype == KDA_BF16) return launch_typed<__nv_bfloat16>(a, mq, mk, mv, ml, stream);
-    return launch_typed<float>(a, mq, mk, mv, ml, stream);
+    if (out_dtype == KDA_BF16) return launch_typed<__nv_bfloat16>(a, stream);
+    return launch_typed<float>(a, stream);
 }
 
 }  // namespace kda
