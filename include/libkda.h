@@ -61,6 +61,9 @@ typedef enum {
 
 /* Bytes of device workspace kda_chunk_fwd needs for these sizes (always >= 256;
  * the first 256 bytes hold the device status word read by kda_workspace_status).
+ * For bf16 inputs the workspace also holds the per-chunk operands that the first of the
+ * two prefill passes prepares for the second: 66048 bytes per (chunk slot, head), with
+ * floor(B*T/64) + N + 1 chunk slots per head (about 1 KiB per token and head).
  * Returns 0 for sizes kda_chunk_fwd would reject. */
 size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int N, int dk, int dv,
                                     kda_dtype_t dtype);
@@ -128,9 +131,11 @@ kda_status_t kda_decode_step(const void *q, const void *k, const void *v,
  * every input and output. Instead of a workspace, the library uses a static device array of
  * KDA_NOALLOC_SCRATCH_BYTES that every GPU on which the library is loaded holds until the process
  * exits. The first call on a device looks up that array's device address (with the device
- * current) and caches it; make that first call before any stream capture begins. Sizes whose
- * scratch need (kda_chunk_fwd_workspace_size) exceeds the array are refused with
- * KDA_ERR_UNSUPPORTED. The function calls no cudaMalloc, cudaFree or other allocating routine.
+ * current) and caches it; make that first call before any stream capture begins. bf16 inputs run
+ * the single-kernel prefill, whose only scratch is the 256-byte status header (a scratch need
+ * beyond the array would be refused with KDA_ERR_UNSUPPORTED); it is slower than the two-pass
+ * prefill kda_chunk_fwd runs with its workspace. The function calls no cudaMalloc, cudaFree or
+ * other allocating routine.
  * The array is shared by every call and keeps the last call's contents; each call clears its
  * status header first. Calls whose work overlaps on the GPU (for example on two streams) race
  * on that shared array: serialise them. Device-side check results (cu_seqlens contents, the

@@ -37,7 +37,9 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int N, int dk, int dv, 
 {
     if (B < 0 || T < 0 || H <= 0 || N < 0 || dk != kHeadDim || dv != kHeadDim) return 0;
     if (dtype != KDA_F32 && dtype != KDA_BF16) return 0;
-    return kStatusBytes;
+    if (dtype == KDA_F32) return kStatusBytes;
+    // bf16: prepared operands of every (chunk slot, head)
+    return kStatusBytes + (size_t)H * (size_t)prep_slots((long long)B * T, N) * kPrepBlockBytes;
 }
 
 kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v,
@@ -82,7 +84,13 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v,
     a.status = (int32_t *)workspace;
     a.scratch = (unsigned char *)workspace + kStatusBytes;
     a.scratch_bytes = workspace_bytes - kStatusBytes;
-    if (dtype == KDA_BF16 && chunk_tc_supported(a)) return map_cuda(launch_chunk_tc(a, out_dtype, st));
+    if (dtype == KDA_BF16) {
+        const int n_slots = (int)prep_slots((long long)B * T, N);
+        unsigned char *ws = (unsigned char *)workspace + kStatusBytes;
+        cudaError_t e2 = launch_chunk_prep(a, ws, n_slots, st);
+        if (e2 == cudaSuccess) e2 = launch_chunk_scan(a, ws, n_slots, out_dtype, st);
+        return map_cuda(e2);
+    }
     return map_cuda(launch_chunk_fp32(a, dtype, out_dtype, st));
 }
 

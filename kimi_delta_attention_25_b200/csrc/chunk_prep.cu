@@ -1,0 +1,433 @@
+// chunk_prep.cu -- first pass of the two-pass bf16 prefill: everything about a 64-token chunk
+// that does not depend on the running state S, for every (chunk, head) at once.
+//
+// Chunk form (chunk C = 64; chunk-parallel prefill with a WY/UT representation: KimiLinear
+// KDA/MLA tutorial (icman.com.cn), sec. 3 and 6; algebra derived from the recurrence). With
+// g_r = sum_{j<=r} log_alpha_j per key channel, f_r = e^{g_r}, b_r = e^{g_{L-1} - g_r}, gamma =
+// e^{g_{L-1}}:
+//   Kt = K f, Qt = Q f, Kend = K b, Kh = K b / gamma;  A = StrictLower(diag(beta) Kt Kh^T);
+//   M = tril(Qt Kh^T);  Tb = (I + A)^{-1} diag(beta);  W = Tb Kt.
+// The second pass (chunk_scan.cu) then runs the state recurrence over chunks with these operands.
+//
+// The chunks are independent, so this pass is a plain data-parallel grid: one CTA (8 warps) per
+// (chunk slot, head), two CTAs per SM. Results go to the workspace in exactly the byte layout the
+// scan wants in shared memory (f16, 128-byte swizzled canonical UMMA tiles), so the scan moves each
+// block with a few bulk copies:
+//   [0, 32K)    W (rows 0-63) and Qt (rows 64-127), two 64-channel halves, K-major
+//   [32K, 40K)  Tb, 64 x 64, K-major        [40K, 48K)  M, 64 x 64, K-major
+//   [48K, 64K)  Kend, two halves of 64 tokens x 64 channels (the MN-major A of Kend^T U)
+//   [64K, +512) gamma (fp32)
+// A chunk slot is floor(first_token / 64) + sequence, which is unique per (sequence, chunk) and
+// below floor(total_tokens / 64) + N + 1.
+#include "kda_internal.cuh"
+#include "sm100.cuh"
+
+namespace kda {
+namespace {
+
+using namespace sm100;
+
+constexpr int C = kChunk;
+constexpr int DK = kHeadDim;
+constexpr int NT = 256;
+
+// Operands are rounded to f16 for the tensor cores: Kh = K e^{-g} must stay finite, so the decay
+// accumulated over one chunk must keep e^{g} above 2^-15 per channel; beyond that UNSUPPORTED.
+constexpr float kMinChunkDecay = 3.0517578125e-05f;
+
+// shared memory (1024-aligned base)
+constexpr uint32_t OFF_QT = 0;               // Qt (f16), two halves of 64 x 128 B
+constexpr uint32_t OFF_KT = 16384;           // Kt
+constexpr uint32_t OFF_KH = 32768;           // Kh; after P1: A^T (fp32, column-major)
+constexpr uint32_t OFF_TB = 49152;           // Tb (f16), 64 x 128 B
+constexpr int LDT = 68;
+constexpr uint32_t OFF_TF = 57344;           // T (fp32, stride LDT) = 17408 B
+constexpr uint32_t OFF_PS = OFF_TF + 17408;  // 4 KB: row-block products, then inverse scratch
+constexpr uint32_t OFF_BET = OFF_PS + 4096;  // 64 fp32
+constexpr uint32_t OFF_BAR = OFF_BET + 256;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 64;
+constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
+
+constexpr uint32_t TMEM_COLS = 128;
+constexpr uint32_t TM_D1A = 0;               // Qt Kh^T  (M=64 layout), later W (cols 0-127)
+constexpr uint32_t TM_D1B = 64;              // Kt Kh^T
+
+__device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
+__device__ __forceinline__ uint2 ldg_nc_u2(const void *p) {
+    uint2 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+    return r;
+}
+__device__ __forceinline__ float4 ldg_nc_f4(const float *p) {
+    float4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w) : "l"(p));
+    return r;
+}
+
+struct PrepParams {
+    const __nv_bfloat16 *q, *k;
+    const float *log_alpha, *beta;
+    const int32_t *cu_seqlens;
+    unsigned char *ws;              // chunk blocks, [H][n_slots][kPrepBlockBytes]
+    int T, H, N, n_slots;
+    int32_t *status;
+};
+
+// Unit lower-triangular inverse (see chunk_tc.cu): A column-major in AT, T row-major stride LDT.
+__device__ __forceinline__ void inverse64(int pt, const float *AT, float *Tf, float *Ps)
+{
+    const int pw = pt >> 5, lane = pt & 31;
+    if (pw < 2) {
+        const int o = 16 * (2 * pw + (lane >> 4)), j = lane & 15;
+        float xv[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) xv[r] = (r == j) ? 1.f : 0.f;
+#pragma unroll
+        for (int i = 0; i < 15; ++i) {
+            float col[16];
+            const float4 *cp = reinterpret_cast<const float4 *>(AT + (o + i) * 64 + o);
+#pragma unroll
+            for (int u = (i + 1) >> 2; u < 4; ++u) {
+                const float4 t = cp[u];
+                col[4 * u] = t.x; col[4 * u + 1] = t.y; col[4 * u + 2] = t.z; col[4 * u + 3] = t.w;
+            }
+            const float xi = xv[i];
+#pragma unroll
+            for (int r = i + 1; r < 16; ++r) xv[r] -= col[r] * xi;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Tf[(o + r) * LDT + o + j] = xv[r];
+    } else {
+        for (int e = pt - 64; e < 64 * 64; e += NT - 64) {
+            const int r = e >> 6, c = e & 63;
+            if ((c >> 4) > (r >> 4)) Tf[r * LDT + c] = 0.f;
+        }
+    }
+    __syncthreads();
+    {   // T_{b+1,b} partial products, b = 0, 2
+        const int blk = pt >> 7, idx = pt & 127, r = idx >> 3, c0 = (idx & 7) * 2, b = 2 * blk;
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float a = AT[(16 * b + k) * 64 + 16 * (b + 1) + r];
+            const float2 t = *reinterpret_cast<const float2 *>(Tf + (16 * b + k) * LDT + 16 * b + c0);
+            a0 += a * t.x;
+            a1 += a * t.y;
+        }
+        *reinterpret_cast<float2 *>(Ps + blk * 256 + r * 16 + c0) = make_float2(a0, a1);
+    }
+    __syncthreads();
+    {
+        const int blk = pt >> 7, idx = pt & 127, r = idx >> 3, c0 = (idx & 7) * 2, b = 2 * blk, o = 16 * (b + 1);
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float t = Tf[(o + r) * LDT + o + k];
+            const float2 pv = *reinterpret_cast<const float2 *>(Ps + blk * 256 + k * 16 + c0);
+            a0 += t * pv.x;
+            a1 += t * pv.y;
+        }
+        *reinterpret_cast<float2 *>(Tf + (o + r) * LDT + 16 * b + c0) = make_float2(-a0, -a1);
+    }
+    __syncthreads();
+    {   // T[32:64, 0:32] = -T_hi (A_hi,lo T_lo)
+        const int r = pt >> 3, c0 = (pt & 7) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+            const float a = AT[k * 64 + 32 + r];
+            const float4 t = *reinterpret_cast<const float4 *>(Tf + k * LDT + c0);
+            acc.x += a * t.x; acc.y += a * t.y; acc.z += a * t.z; acc.w += a * t.w;
+        }
+        *reinterpret_cast<float4 *>(Ps + r * 32 + c0) = acc;
+    }
+    __syncthreads();
+    {
+        const int r = pt >> 3, c0 = (pt & 7) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+            const float t = Tf[(32 + r) * LDT + 32 + k];
+            const float4 pv = *reinterpret_cast<const float4 *>(Ps + k * 32 + c0);
+            acc.x += t * pv.x; acc.y += t * pv.y; acc.z += t * pv.z; acc.w += t * pv.w;
+        }
+        *reinterpret_cast<float4 *>(Tf + (32 + r) * LDT + c0) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(NT, 2)
+chunk_prep_kernel(PrepParams p)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int slot = blockIdx.x, h = blockIdx.y;
+    const int H = p.H;
+
+    // ---- which (sequence, chunk) this slot is: slot = floor(first_token / 64) + sequence
+    int n = 0;
+    int64_t s0, s1;
+    if (p.cu_seqlens) {
+        int lo = 0, hi = p.N - 1;                 // largest n with floor(cu[n]/64) + n <= slot
+        if (hi < 0) return;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.cu_seqlens[mid] / C + mid <= slot) lo = mid; else hi = mid - 1;
+        }
+        n = lo;
+        s0 = p.cu_seqlens[n];
+        s1 = p.cu_seqlens[n + 1];
+        if (s1 < s0 || s0 < 0 || s1 > p.T) return;    // reported by the scan pass
+    } else {
+        // sequence n = batch row; its first slot is (n * T) / 64 + n
+        int lo = 0, hi = p.N - 1;
+        if (hi < 0) return;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if ((int)(((int64_t)mid * p.T) / C) + mid <= slot) lo = mid; else hi = mid - 1;
+        }
+        n = lo;
+        s0 = (int64_t)n * p.T;
+        s1 = s0 + p.T;
+    }
+    const int64_t first_slot = s0 / C + n;
+    const int64_t c = slot - first_slot;
+    const int64_t tok0 = s0 + c * C;
+    if (c < 0 || tok0 >= s1) return;              // unused slot
+    const int L = (s1 - tok0 < C) ? (int)(s1 - tok0) : C;
+    unsigned char *blk = p.ws + ((size_t)h * p.n_slots + slot) * kPrepBlockBytes;
+
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 1);
+    float *AT = reinterpret_cast<float *>(sm + OFF_KH);
+    float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
+    float *Ps = reinterpret_cast<float *>(sm + OFF_PS);
+    float *bet = reinterpret_cast<float *>(sm + OFF_BET);
+
+    if (warp == 0) { tmem_alloc(tmem_slot, TMEM_COLS); tmem_relinquish(); }
+    if (tid == 0) { mbar_init(bar, 1); fence_mbar_init(); }
+
+    // ---- loads: warp w -> rows 8w..8w+7, lane -> channels 4 lane..4 lane+3 (a warp reads whole rows)
+    const int cq = lane, kh = cq >> 4, lc4 = cq & 15;
+    float4 la[8];
+    uint2 kr[8], qr[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+        const int r = 8 * warp + x;
+        if (r < L) {
+            const size_t row = ((size_t)(tok0 + r) * H + h) * DK + 4 * cq;
+            la[x] = ldg_nc_f4(p.log_alpha + row);
+            kr[x] = ldg_nc_u2(p.k + row);
+            qr[x] = ldg_nc_u2(p.q + row);
+        } else {
+            la[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+            kr[x] = make_uint2(0u, 0u);
+            qr[x] = kr[x];
+        }
+    }
+    if (tid < C) bet[tid] = (tid < L) ? p.beta[(size_t)(tok0 + tid) * H + h] : 0.f;
+
+    // ---- decay scaling: per-thread products over its 8 rows, then over the 8 warps via smem
+    float a[8][4], pre[8][4];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+        a[x][0] = __expf(la[x].x); a[x][1] = __expf(la[x].y);
+        a[x][2] = __expf(la[x].z); a[x][3] = __expf(la[x].w);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        float run = 1.f;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) { run *= a[x][e]; pre[x][e] = run; }
+    }
+    *reinterpret_cast<float4 *>(Ps + warp * 128 + 4 * cq) = make_float4(pre[7][0], pre[7][1], pre[7][2], pre[7][3]);
+    __syncthreads();
+    float before[4] = {1.f, 1.f, 1.f, 1.f}, after[4] = {1.f, 1.f, 1.f, 1.f}, g[4], rg[4];
+#pragma unroll
+    for (int y = 0; y < 8; ++y) {
+        const float4 t = *reinterpret_cast<const float4 *>(Ps + y * 128 + 4 * cq);
+        const float tv[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (y < warp) before[e] *= tv[e];
+            if (y > warp) after[e] *= tv[e];
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        g[e] = before[e] * pre[7][e] * after[e];
+        rg[e] = __frcp_rn(g[e]);
+    }
+    if (warp == 0) {
+        float *gw = reinterpret_cast<float *>(blk + kPrepGammaOff);
+        *reinterpret_cast<float4 *>(gw + 4 * cq) = make_float4(g[0], g[1], g[2], g[3]);
+        if (g[0] < kMinChunkDecay || g[1] < kMinChunkDecay || g[2] < kMinChunkDecay || g[3] < kMinChunkDecay)
+            set_status(p.status, KDA_ERR_UNSUPPORTED);
+    }
+    {
+        float suf[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll
+        for (int x = 7; x >= 0; --x) {
+            const int r = 8 * warp + x;
+            const uint32_t off = r * 128 + ((((lc4 >> 1) ^ (r & 7)) & 7) << 4) + ((lc4 & 1) << 3);
+            const uint32_t kw[2] = {kr[x].x, kr[x].y};
+            const uint32_t qw[2] = {qr[x].x, qr[x].y};
+            uint32_t okt[2], oqt[2], oke[2], okh[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int e = 2 * u;
+                const float f0 = before[e] * pre[x][e], f1 = before[e + 1] * pre[x][e + 1];
+                const float b0 = suf[e] * after[e], b1 = suf[e + 1] * after[e + 1];
+                const float k0 = bf_lo(kw[u]), k1 = bf_hi(kw[u]);
+                const float q0 = bf_lo(qw[u]), q1 = bf_hi(qw[u]);
+                const float e0 = k0 * b0, e1 = k1 * b1;
+                okt[u] = pack_f16x2(k0 * f0, k1 * f1);
+                oqt[u] = pack_f16x2(q0 * f0, q1 * f1);
+                oke[u] = pack_f16x2(e0, e1);
+                okh[u] = pack_f16x2(e0 * rg[e], e1 * rg[e + 1]);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) suf[e] *= a[x][e];
+            const uint2 vqt = make_uint2(oqt[0], oqt[1]);
+            *reinterpret_cast<uint2 *>(sm + OFF_KT + kh * 8192 + off) = make_uint2(okt[0], okt[1]);
+            *reinterpret_cast<uint2 *>(sm + OFF_QT + kh * 8192 + off) = vqt;
+            *reinterpret_cast<uint2 *>(sm + OFF_KH + kh * 8192 + off) = make_uint2(okh[0], okh[1]);
+            *reinterpret_cast<uint2 *>(blk + kPrepWQOff + kh * 16384 + 64 * 128 + off) = vqt;
+            *reinterpret_cast<uint2 *>(blk + kPrepKEOff + kh * 8192 + off) = make_uint2(oke[0], oke[1]);
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // ---- P1: D1A = Qt Kh^T, D1B = Kt Kh^T (M=64, N=64, K=128)
+    if (tid == 0) {
+        const uint32_t id = idesc_f16(64, 64, 0, 0);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t k2 = ks >> 2, ko = (ks & 3) * 32;
+            const uint64_t bd = smem_desc(sbase + OFF_KH + k2 * 8192 + ko, 16, 1024, SW_128B);
+            umma_ss(tmem + TM_D1A, smem_desc(sbase + OFF_QT + k2 * 8192 + ko, 16, 1024, SW_128B), bd, id, ks > 0);
+            umma_ss(tmem + TM_D1B, smem_desc(sbase + OFF_KT + k2 * 8192 + ko, 16, 1024, SW_128B), bd, id, ks > 0);
+        }
+        umma_commit(bar);
+    }
+    int32_t failed = 0;
+    if (tid == 0 && !mbar_wait(bar, 0)) failed = 1;
+    __syncthreads();
+    tc_fence_after();
+    // ---- P1 epilogue: warps 0-3 -> M (f16 -> workspace); warps 4-7 -> A^T (fp32, smem)
+    {
+        const int q4 = warp & 3, half = warp >> 2;
+        float v[64];
+        tmem_ld64_sync(tmem + ((uint32_t)(32 * q4) << 16) + (half ? TM_D1B : TM_D1A), v);
+        if (lane < 16) {
+            const int r = 16 * q4 + lane;
+            if (half == 0) {
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = 8 * ch + 2 * u;
+                        w4[u] = pack_f16x2(i <= r ? v[i] : 0.f, i + 1 <= r ? v[i + 1] : 0.f);
+                    }
+                    *reinterpret_cast<uint4 *>(blk + kPrepMOff + sw128_offset(r, 8 * ch)) =
+                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+            } else {
+                const float br = bet[r];
+#pragma unroll
+                for (int i = 0; i < 64; ++i) AT[i * 64 + r] = (i < r) ? br * v[i] : 0.f;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    // ---- T = (I + A)^{-1};  Tb = T diag(beta) -> f16 (smem for P3, and workspace)
+    inverse64(tid, AT, Tf, Ps);
+    {
+        const int r = tid >> 2, c0 = (tid & 3) * 16;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int cb = c0 + 8 * hh;
+            const float4 t0v = *reinterpret_cast<const float4 *>(Tf + r * LDT + cb);
+            const float4 t1v = *reinterpret_cast<const float4 *>(Tf + r * LDT + cb + 4);
+            const float4 b0v = *reinterpret_cast<const float4 *>(bet + cb);
+            const float4 b1v = *reinterpret_cast<const float4 *>(bet + cb + 4);
+            const float tv[8] = {t0v.x * b0v.x, t0v.y * b0v.y, t0v.z * b0v.z, t0v.w * b0v.w,
+                                 t1v.x * b1v.x, t1v.y * b1v.y, t1v.z * b1v.z, t1v.w * b1v.w};
+            uint32_t w4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = cb + 2 * u;
+                w4[u] = pack_f16x2(i <= r ? tv[2 * u] : 0.f, i + 1 <= r ? tv[2 * u + 1] : 0.f);
+            }
+            const uint4 o = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            *reinterpret_cast<uint4 *>(sm + OFF_TB + sw128_offset(r, cb)) = o;
+            *reinterpret_cast<uint4 *>(blk + kPrepTbOff + sw128_offset(r, cb)) = o;
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // ---- P3: W = Tb Kt (M=64, N=128, K=64; B = Kt MN-major) into columns 0-127
+    if (tid == 0) {
+        const uint32_t id = idesc_f16(64, 128, 0, 1);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            umma_ss(tmem + TM_D1A, smem_desc(sbase + OFF_TB + ks * 32, 16, 1024, SW_128B),
+                    smem_desc(sbase + OFF_KT + ks * 2048, 8192, 1024, SW_128B), id, ks > 0);
+        umma_commit(bar);
+    }
+    if (tid == 0 && !failed && !mbar_wait(bar, 1)) failed = 1;
+    __syncthreads();
+    tc_fence_after();
+    // ---- W epilogue (M=64 layout: lanes 0-15 of each quadrant), warps 0-3 cols 0-63, 4-7 cols 64-127
+    {
+        const int q4 = warp & 3, half = warp >> 2;
+        float w[64];
+        tmem_ld64_sync(tmem + ((uint32_t)(32 * q4) << 16) + TM_D1A + 64 * half, w);
+        if (lane < 16) {
+            const int r = 16 * q4 + lane;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                uint4 o;
+                o.x = pack_f16x2(w[8 * ch + 0], w[8 * ch + 1]);
+                o.y = pack_f16x2(w[8 * ch + 2], w[8 * ch + 3]);
+                o.z = pack_f16x2(w[8 * ch + 4], w[8 * ch + 5]);
+                o.w = pack_f16x2(w[8 * ch + 6], w[8 * ch + 7]);
+                *reinterpret_cast<uint4 *>(blk + kPrepWQOff + half * 16384 + sw128_offset(r, 8 * ch)) = o;
+            }
+        }
+    }
+    if (failed) set_status(p.status, KDA_ERR_TIMEOUT);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slots, cudaStream_t stream)
+{
+    PrepParams p;
+    p.q = (const __nv_bfloat16 *)a.q; p.k = (const __nv_bfloat16 *)a.k;
+    p.log_alpha = a.log_alpha; p.beta = a.beta; p.cu_seqlens = a.cu_seqlens;
+    p.ws = ws; p.T = a.T; p.H = a.H; p.N = a.N; p.n_slots = n_slots; p.status = a.status;
+    cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(n_slots, a.H);
+    chunk_prep_kernel<<<grid, NT, SMEM_ALLOC, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

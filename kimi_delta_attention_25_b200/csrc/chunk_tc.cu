@@ -71,8 +71,9 @@ constexpr uint32_t OFF_V0 = OFF_KE1 + KE_BYTES;
 constexpr uint32_t OFF_V1 = OFF_V0 + V_BYTES;
 constexpr uint32_t OFF_KT = OFF_V1 + V_BYTES;          // Kt (f16), two halves
 constexpr uint32_t OFF_KH = OFF_KT + 16384;            // Kh (f16); after P1: A^T (fp32, column-major)
-constexpr uint32_t OFF_TF = OFF_KH + 16384;            // T (fp32, row-major)
-constexpr uint32_t OFF_SB = OFF_TF + 16384;            // S (f16), 128 rows x 64 B
+constexpr int LDT = 68;                                // row stride of T (floats): conflict-free columns
+constexpr uint32_t OFF_TF = OFF_KH + 16384;            // T (fp32, row-major, stride LDT)
+constexpr uint32_t OFF_SB = OFF_TF + 18432;            // S (f16), 128 rows x 64 B
 constexpr uint32_t OFF_UB = OFF_SB + DK * DVB * 2;     // U (f16), 64 rows x 64 B
 constexpr uint32_t OFF_PS = OFF_UB + C * DVB * 2;      // block-product scratch of the inverse (fp32)
 constexpr uint32_t OFF_GAM = OFF_PS + 32 * 32 * 4;     // gamma, 2 x 128 fp32
@@ -115,46 +116,50 @@ __device__ __forceinline__ uint4 ldg_nc(const void *p) {
                  : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
     return r;
 }
+__device__ __forceinline__ uint2 ldg_nc_u2(const void *p) {
+    uint2 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+    return r;
+}
 __device__ __forceinline__ float4 ldg_nc_f4(const float *p) {
     const uint4 r = ldg_nc(p);
     return make_float4(__uint_as_float(r.x), __uint_as_float(r.y), __uint_as_float(r.z), __uint_as_float(r.w));
 }
 
 // Unit lower-triangular inverse T = (I + A)^{-1} for a 64 x 64 strictly lower A held column-major
-// (AT[c * 64 + r] = A[r][c]); T is written row-major (T[r * 64 + c]). Diagonal 16 x 16 blocks by
+// (AT[c * 64 + r] = A[r][c]); T is written row-major with stride LDT. Diagonal 16 x 16 blocks by
 // forward substitution in registers; then T_{b+1,b} = -T_{b+1,b+1} A_{b+1,b} T_{b,b} inside each
 // 32 x 32 half, then T_{hi,lo} = -T_hi A_{hi,lo} T_lo for the off-diagonal 32 x 32 block.
 // Called by the 256 prep threads (pt = 0..255); ends synchronised.
 __device__ __forceinline__ void prep_inverse(int pt, const float *AT, float *Tf, float *Ps)
 {
     const int pw = pt >> 5, lane = pt & 31;
-    if (pw < 4) {
-        if (lane < 16) {
-            const int o = 16 * pw, j = lane;
-            float xv[16];
+    if (pw < 2) {
+        // warp 0: blocks 0 and 1 (lanes 0-15 / 16-31); warp 1: blocks 2 and 3
+        const int o = 16 * (2 * pw + (lane >> 4)), j = lane & 15;
+        float xv[16];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) xv[r] = (r == j) ? 1.f : 0.f;
+        for (int r = 0; r < 16; ++r) xv[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
-            for (int i = 0; i < 15; ++i) {
-                float col[16];
-                const float4 *cp = reinterpret_cast<const float4 *>(AT + (o + i) * 64 + o);
+        for (int i = 0; i < 15; ++i) {
+            float col[16];
+            const float4 *cp = reinterpret_cast<const float4 *>(AT + (o + i) * 64 + o);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float4 t = cp[u];
-                    col[4 * u] = t.x; col[4 * u + 1] = t.y; col[4 * u + 2] = t.z; col[4 * u + 3] = t.w;
-                }
-                const float xi = xv[i];
-#pragma unroll
-                for (int r = i + 1; r < 16; ++r) xv[r] -= col[r] * xi;
+            for (int u = (i + 1) >> 2; u < 4; ++u) {
+                const float4 t = cp[u];
+                col[4 * u] = t.x; col[4 * u + 1] = t.y; col[4 * u + 2] = t.z; col[4 * u + 3] = t.w;
             }
+            const float xi = xv[i];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) Tf[(o + r) * 64 + o + j] = xv[r];
+            for (int r = i + 1; r < 16; ++r) xv[r] -= col[r] * xi;
         }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Tf[(o + r) * LDT + o + j] = xv[r];
     } else {
         // zero the strictly upper 16 x 16 blocks of T
-        for (int e = pt - 128; e < 64 * 64; e += 128) {
+        for (int e = pt - 64; e < 64 * 64; e += 192) {
             const int r = e >> 6, c = e & 63;
-            if ((c >> 4) > (r >> 4)) Tf[e] = 0.f;
+            if ((c >> 4) > (r >> 4)) Tf[r * LDT + c] = 0.f;
         }
     }
     named_bar_sync(1, PG_THREADS);
@@ -166,7 +171,7 @@ __device__ __forceinline__ void prep_inverse(int pt, const float *AT, float *Tf,
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
             const float a = AT[(16 * b + k) * 64 + 16 * (b + 1) + r];
-            const float2 t = *reinterpret_cast<const float2 *>(Tf + (16 * b + k) * 64 + 16 * b + c0);
+            const float2 t = *reinterpret_cast<const float2 *>(Tf + (16 * b + k) * LDT + 16 * b + c0);
             a0 += a * t.x;
             a1 += a * t.y;
         }
@@ -180,12 +185,12 @@ __device__ __forceinline__ void prep_inverse(int pt, const float *AT, float *Tf,
         float a0 = 0.f, a1 = 0.f;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-            const float t = Tf[(o + r) * 64 + o + k];
+            const float t = Tf[(o + r) * LDT + o + k];
             const float2 pv = *reinterpret_cast<const float2 *>(Ps + blk * 256 + k * 16 + c0);
             a0 += t * pv.x;
             a1 += t * pv.y;
         }
-        *reinterpret_cast<float2 *>(Tf + (o + r) * 64 + 16 * b + c0) = make_float2(-a0, -a1);
+        *reinterpret_cast<float2 *>(Tf + (o + r) * LDT + 16 * b + c0) = make_float2(-a0, -a1);
     }
     named_bar_sync(1, PG_THREADS);
     // level 2a: P = A[32:64, 0:32] T[0:32, 0:32] (four outputs per thread)
@@ -195,7 +200,7 @@ __device__ __forceinline__ void prep_inverse(int pt, const float *AT, float *Tf,
 #pragma unroll 8
         for (int k = 0; k < 32; ++k) {
             const float a = AT[k * 64 + 32 + r];
-            const float4 t = *reinterpret_cast<const float4 *>(Tf + k * 64 + c0);
+            const float4 t = *reinterpret_cast<const float4 *>(Tf + k * LDT + c0);
             acc.x += a * t.x; acc.y += a * t.y; acc.z += a * t.z; acc.w += a * t.w;
         }
         *reinterpret_cast<float4 *>(Ps + r * 32 + c0) = acc;
@@ -207,13 +212,47 @@ __device__ __forceinline__ void prep_inverse(int pt, const float *AT, float *Tf,
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
         for (int k = 0; k < 32; ++k) {
-            const float t = Tf[(32 + r) * 64 + 32 + k];
+            const float t = Tf[(32 + r) * LDT + 32 + k];
             const float4 pv = *reinterpret_cast<const float4 *>(Ps + k * 32 + c0);
             acc.x += t * pv.x; acc.y += t * pv.y; acc.z += t * pv.z; acc.w += t * pv.w;
         }
-        *reinterpret_cast<float4 *>(Tf + (32 + r) * 64 + c0) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+        *reinterpret_cast<float4 *>(Tf + (32 + r) * LDT + c0) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
     }
     named_bar_sync(1, PG_THREADS);
+}
+
+// One prep thread's share of a chunk's inputs, loaded from global memory into registers one chunk
+// ahead so that the load latency overlaps the previous chunk's work: rows 8rb..8rb+7 and channels
+// 4cq..4cq+3 of q, k and log_alpha (rb = pt & 7, cq = pt >> 3), eight v values (row pt >> 2,
+// columns 8 (pt & 3)..+7 of the d_v block) and, for pt < 64, beta of row pt.
+struct RawChunk {
+    float4 la[8];
+    uint2 kr[8], qr[8];
+    uint4 v;
+    float beta;
+};
+
+__device__ __forceinline__ void prep_load(RawChunk &R, const TcParams &p, int64_t tok0, int L, int h,
+                                          int j0, int pt)
+{
+    const int H = p.H, cq = pt >> 3, rb = pt & 7;
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+        const int r = 8 * rb + x;
+        if (r < L) {
+            const size_t row = ((size_t)(tok0 + r) * H + h) * DK + 4 * cq;
+            R.la[x] = ldg_nc_f4(p.log_alpha + row);
+            R.kr[x] = ldg_nc_u2(p.k + row);
+            R.qr[x] = ldg_nc_u2(p.q + row);
+        } else {
+            R.la[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+            R.kr[x] = make_uint2(0u, 0u);
+            R.qr[x] = R.kr[x];
+        }
+    }
+    const int rv = pt >> 2;
+    R.v = (rv < L) ? ldg_nc(p.v + ((size_t)(tok0 + rv) * H + h) * DK + j0 + 8 * (pt & 3)) : make_uint4(0, 0, 0, 0);
+    R.beta = (pt < L && pt < C) ? p.beta[(size_t)(tok0 + pt) * H + h] : 0.f;
 }
 
 // =================================================================================== kernel
@@ -260,123 +299,83 @@ chunk_tc_kernel(TcParams p)
     if (warp >= 4) {
         // =========================================================================== prep group
         const int pt = tid - SG_THREADS, pw = warp - 4, q4 = warp & 3, half = pw >> 2;
-        const float LOG2E = 1.4426950408889634f;
         float *AT = reinterpret_cast<float *>(sm + OFF_KH);
         float *Tf = reinterpret_cast<float *>(sm + OFF_TF);
         float *Ps = reinterpret_cast<float *>(sm + OFF_PS);
         uint32_t n_p1 = 0, n_p3 = 0;               // commits issued (thread 0)
+        RawChunk R;
+        if (nchunks > 0) prep_load(R, p, t0, (t1 - t0 < C) ? (int)(t1 - t0) : C, h, j0, pt);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c & 1;
             const int64_t tok0 = t0 + (int64_t)c * C;
-            const int L = (t1 - tok0 < C) ? (int)(t1 - tok0) : C;
             unsigned char *X = sm + (s ? OFF_X1 : OFF_X0);
             unsigned char *Y = sm + (s ? OFF_Y1 : OFF_Y0);
             unsigned char *KE = sm + (s ? OFF_KE1 : OFF_KE0);
             unsigned char *Vs = sm + (s ? OFF_V1 : OFF_V0);
-            if (c >= 2 && !mbar_wait(&bars[B_FREE + s], ((c >> 1) - 1) & 1)) fail();
+            if (c >= 2) {               // one thread polls; the group barrier releases the others
+                if (pt == 0 && !mbar_wait(&bars[B_FREE + s], ((c >> 1) - 1) & 1)) fail();
+                named_bar_sync(1, PG_THREADS);
+            }
             tc_fence_after();
 
-            // ---- prefetch the next chunk's rows into L2
-            if (c + 1 < nchunks) {
-                const int64_t nt0 = tok0 + C;
-                const int nL = (t1 - nt0 < C) ? (int)(t1 - nt0) : C;
-                const int r = pt >> 2, part = pt & 3;
-                if (r < nL) {
-                    const size_t row = ((size_t)(nt0 + r) * H + h) * DK;
-                    prefetch_l2(p.log_alpha + row + 32 * part);
-                    if (part < 2) {
-                        prefetch_l2(p.q + row + 64 * part);
-                        prefetch_l2(p.k + row + 64 * part);
-                    } else if (part == 2) {
-                        prefetch_l2(p.v + row + j0);
-                    } else {
-                        prefetch_l2(p.beta + (size_t)(nt0 + r) * H + h);
-                    }
-                }
-            }
             // ---- beta and the v block (bf16 -> f16, 64-byte swizzled rows)
-            if (pt < C) bet[pt] = (pt < L) ? p.beta[(size_t)(tok0 + pt) * H + h] : 0.f;
+            if (pt < C) bet[pt] = R.beta;
             {
-                const int r = pt >> 2, cq = (pt & 3) * 8;
-                uint4 o = make_uint4(0, 0, 0, 0);
-                if (r < L) {
-                    const uint4 raw = ldg_nc(p.v + ((size_t)(tok0 + r) * H + h) * DK + j0 + cq);
-                    o.x = bf16x2_to_f16x2(raw.x); o.y = bf16x2_to_f16x2(raw.y);
-                    o.z = bf16x2_to_f16x2(raw.z); o.w = bf16x2_to_f16x2(raw.w);
-                }
-                *reinterpret_cast<uint4 *>(Vs + sw64_offset(r, cq)) = o;
+                uint4 o;
+                o.x = bf16x2_to_f16x2(R.v.x); o.y = bf16x2_to_f16x2(R.v.y);
+                o.z = bf16x2_to_f16x2(R.v.z); o.w = bf16x2_to_f16x2(R.v.w);
+                *reinterpret_cast<uint4 *>(Vs + sw64_offset(pt >> 2, 8 * (pt & 3))) = o;
             }
-            // ---- decay scaling: thread -> rows 4rb..4rb+3, channels 8cc..8cc+7; the 16 row blocks
-            //      of one channel chunk sit on 16 consecutive lanes
+            // ---- decay scaling: thread -> rows 8rb..8rb+7, channels 4cq..4cq+3; the 8 row blocks of
+            //      one channel quad sit on 8 consecutive lanes
             {
-                const int cc = pt >> 4, rb = pt & 15, kh = cc >> 3, lc = cc & 7;
-                float a[4][8];
-                uint4 kr[4], qr[4];
+                const int cq = pt >> 3, rb = pt & 7, kh = cq >> 4, lc4 = cq & 15;
+                float a[8][4], pre[8][4], before[4], after[4], g[4], rg[4];
 #pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    const int r = 4 * rb + x;
-                    if (r < L) {
-                        const size_t row = ((size_t)(tok0 + r) * H + h) * DK + 8 * cc;
-                        const float4 l0 = ldg_nc_f4(p.log_alpha + row);
-                        const float4 l1 = ldg_nc_f4(p.log_alpha + row + 4);
-                        kr[x] = ldg_nc(p.k + row);
-                        qr[x] = ldg_nc(p.q + row);
-                        a[x][0] = l0.x; a[x][1] = l0.y; a[x][2] = l0.z; a[x][3] = l0.w;
-                        a[x][4] = l1.x; a[x][5] = l1.y; a[x][6] = l1.z; a[x][7] = l1.w;
-                    } else {
-                        kr[x] = make_uint4(0, 0, 0, 0);
-                        qr[x] = kr[x];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) a[x][e] = 0.f;
-                    }
+                for (int x = 0; x < 8; ++x) {
+                    a[x][0] = __expf(R.la[x].x); a[x][1] = __expf(R.la[x].y);
+                    a[x][2] = __expf(R.la[x].z); a[x][3] = __expf(R.la[x].w);
                 }
-                // alpha; local inclusive prefix (pre) and exclusive suffix (suf) over the 4 rows;
-                // products over the other row blocks from the neighbouring lanes
-                float pre[4][8], suf[4][8], before[8], after[8], g[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
+                for (int e = 0; e < 4; ++e) {
                     float run = 1.f;
 #pragma unroll
-                    for (int x = 0; x < 4; ++x) { a[x][e] = exp2f(a[x][e] * LOG2E); run *= a[x][e]; pre[x][e] = run; }
-                    float rs = 1.f;
-#pragma unroll
-                    for (int x = 3; x >= 0; --x) { suf[x][e] = rs; rs *= a[x][e]; }
+                    for (int x = 0; x < 8; ++x) { run *= a[x][e]; pre[x][e] = run; }
                     float inc = run, sfx = run;
 #pragma unroll
-                    for (int o = 1; o < 16; o <<= 1) {
-                        const float u = __shfl_up_sync(0xffffffffu, inc, o, 16);
-                        const float d = __shfl_down_sync(0xffffffffu, sfx, o, 16);
+                    for (int o = 1; o < 8; o <<= 1) {
+                        const float u = __shfl_up_sync(0xffffffffu, inc, o, 8);
+                        const float d = __shfl_down_sync(0xffffffffu, sfx, o, 8);
                         if (rb >= o) inc *= u;
-                        if (rb + o < 16) sfx *= d;
+                        if (rb + o < 8) sfx *= d;
                     }
-                    const float bu = __shfl_up_sync(0xffffffffu, inc, 1, 16);
-                    const float ad = __shfl_down_sync(0xffffffffu, sfx, 1, 16);
+                    const float bu = __shfl_up_sync(0xffffffffu, inc, 1, 8);
+                    const float ad = __shfl_down_sync(0xffffffffu, sfx, 1, 8);
                     before[e] = (rb == 0) ? 1.f : bu;
-                    after[e] = (rb == 15) ? 1.f : ad;
-                    g[e] = __shfl_sync(0xffffffffu, inc, 15, 16);
+                    after[e] = (rb == 7) ? 1.f : ad;
+                    g[e] = __shfl_sync(0xffffffffu, inc, 7, 8);
+                    rg[e] = __frcp_rn(g[e]);
                 }
                 if (rb == 0) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        gam[s * 128 + 8 * cc + e] = g[e];
+                    for (int e = 0; e < 4; ++e) {
+                        gam[s * 128 + 4 * cq + e] = g[e];
                         if (g[e] < kMinChunkDecay) set_status(p.status, KDA_ERR_UNSUPPORTED);
                     }
                 }
-                float rg[8];
+                float suf[4] = {1.f, 1.f, 1.f, 1.f};
 #pragma unroll
-                for (int e = 0; e < 8; ++e) rg[e] = 1.f / g[e];
+                for (int x = 7; x >= 0; --x) {
+                    const int r = 8 * rb + x;
+                    const uint32_t off = r * 128 + ((((lc4 >> 1) ^ (r & 7)) & 7) << 4) + ((lc4 & 1) << 3);
+                    const uint32_t kw[2] = {R.kr[x].x, R.kr[x].y};
+                    const uint32_t qw[2] = {R.qr[x].x, R.qr[x].y};
+                    uint32_t okt[2], oqt[2], oke[2], okh[2];
 #pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    const int r = 4 * rb + x;
-                    const uint32_t off = sw128_offset(r, 8 * lc);
-                    const uint32_t kw[4] = {kr[x].x, kr[x].y, kr[x].z, kr[x].w};
-                    const uint32_t qw[4] = {qr[x].x, qr[x].y, qr[x].z, qr[x].w};
-                    uint32_t okt[4], oqt[4], oke[4], okh[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < 2; ++u) {
                         const int e = 2 * u;
                         const float f0 = before[e] * pre[x][e], f1 = before[e + 1] * pre[x][e + 1];
-                        const float b0 = suf[x][e] * after[e], b1 = suf[x][e + 1] * after[e + 1];
+                        const float b0 = suf[e] * after[e], b1 = suf[e + 1] * after[e + 1];
                         const float k0 = bf_lo(kw[u]), k1 = bf_hi(kw[u]);
                         const float q0 = bf_lo(qw[u]), q1 = bf_hi(qw[u]);
                         const float e0 = k0 * b0, e1 = k1 * b1;
@@ -385,10 +384,12 @@ chunk_tc_kernel(TcParams p)
                         oke[u] = pack_f16x2(e0, e1);
                         okh[u] = pack_f16x2(e0 * rg[e], e1 * rg[e + 1]);
                     }
-                    *reinterpret_cast<uint4 *>(sm + OFF_KT + kh * 8192 + off) = make_uint4(okt[0], okt[1], okt[2], okt[3]);
-                    *reinterpret_cast<uint4 *>(X + kh * X_HALF + 64 * 128 + off) = make_uint4(oqt[0], oqt[1], oqt[2], oqt[3]);
-                    *reinterpret_cast<uint4 *>(KE + kh * 8192 + off) = make_uint4(oke[0], oke[1], oke[2], oke[3]);
-                    *reinterpret_cast<uint4 *>(sm + OFF_KH + kh * 8192 + off) = make_uint4(okh[0], okh[1], okh[2], okh[3]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) suf[e] *= a[x][e];
+                    *reinterpret_cast<uint2 *>(sm + OFF_KT + kh * 8192 + off) = make_uint2(okt[0], okt[1]);
+                    *reinterpret_cast<uint2 *>(X + kh * X_HALF + 64 * 128 + off) = make_uint2(oqt[0], oqt[1]);
+                    *reinterpret_cast<uint2 *>(KE + kh * 8192 + off) = make_uint2(oke[0], oke[1]);
+                    *reinterpret_cast<uint2 *>(sm + OFF_KH + kh * 8192 + off) = make_uint2(okh[0], okh[1]);
                 }
             }
             fence_proxy_async_smem();
@@ -410,20 +411,18 @@ chunk_tc_kernel(TcParams p)
                 }
                 umma_commit(&bars[B_P1]);
             }
-            if (!mbar_wait(&bars[B_P1], c & 1)) fail();
+            // ---- the next chunk's inputs go out now; their latency overlaps P1, T and P3
+            if (c + 1 < nchunks) {
+                const int64_t nt0 = tok0 + C;
+                prep_load(R, p, nt0, (t1 - nt0 < C) ? (int)(t1 - nt0) : C, h, j0, pt);
+            }
+            if (pt == 0 && !mbar_wait(&bars[B_P1], c & 1)) fail();
+            named_bar_sync(1, PG_THREADS);
             tc_fence_after();
             // ---- P1 epilogue: half 0 -> M (f16, Y rows 128-191); half 1 -> A^T (fp32, column-major)
             {
-                const uint32_t ta = tmem + ((uint32_t)(32 * q4) << 16) + (half ? TM_D1B : TM_D1A);
                 float v[64];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float r16[16];
-                    tmem_ld16(ta + 16 * q, r16);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) v[16 * q + e] = r16[e];
-                }
+                tmem_ld64_sync(tmem + ((uint32_t)(32 * q4) << 16) + (half ? TM_D1B : TM_D1A), v);
                 if (lane < 16) {
                     const int r = 16 * q4 + lane;
                     if (half == 0) {
@@ -455,15 +454,17 @@ chunk_tc_kernel(TcParams p)
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     const int cb = c0 + 8 * hh;
-                    const float4 t0v = *reinterpret_cast<const float4 *>(Tf + r * 64 + cb);
-                    const float4 t1v = *reinterpret_cast<const float4 *>(Tf + r * 64 + cb + 4);
-                    const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
+                    const float4 t0v = *reinterpret_cast<const float4 *>(Tf + r * LDT + cb);
+                    const float4 t1v = *reinterpret_cast<const float4 *>(Tf + r * LDT + cb + 4);
+                    const float4 b0v = *reinterpret_cast<const float4 *>(bet + cb);
+                    const float4 b1v = *reinterpret_cast<const float4 *>(bet + cb + 4);
+                    const float tv[8] = {t0v.x * b0v.x, t0v.y * b0v.y, t0v.z * b0v.z, t0v.w * b0v.w,
+                                         t1v.x * b1v.x, t1v.y * b1v.y, t1v.z * b1v.z, t1v.w * b1v.w};
                     uint32_t w4[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const int i = cb + 2 * u;
-                        w4[u] = pack_f16x2(i <= r ? tv[2 * u] * bet[i] : 0.f,
-                                           i + 1 <= r ? tv[2 * u + 1] * bet[i + 1] : 0.f);
+                        w4[u] = pack_f16x2(i <= r ? tv[2 * u] : 0.f, i + 1 <= r ? tv[2 * u + 1] : 0.f);
                     }
                     *reinterpret_cast<uint4 *>(Y + sw128_offset(r, cb)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }
@@ -486,26 +487,22 @@ chunk_tc_kernel(TcParams p)
                 }
                 umma_commit(&bars[B_P3]);
             }
-            if (!mbar_wait(&bars[B_P3], c & 1)) fail();
+            if (pt == 0 && !mbar_wait(&bars[B_P3], c & 1)) fail();
+            named_bar_sync(1, PG_THREADS);
             tc_fence_after();
             // ---- W epilogue: rows 0-63 of D3 (TMEM lanes 0-63) -> f16 X rows 0-63
             if (q4 < 2) {
                 const int r = 32 * q4 + lane;
-                const uint32_t ta = tmem + ((uint32_t)(32 * q4) << 16) + TM_D3 + 64 * half;
+                float w[64];
+                tmem_ld64_sync(tmem + ((uint32_t)(32 * q4) << 16) + TM_D3 + 64 * half, w);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float r16[16];
-                    tmem_ld16(ta + 16 * q, r16);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        uint4 o;
-                        o.x = pack_f16x2(r16[8 * hh + 0], r16[8 * hh + 1]);
-                        o.y = pack_f16x2(r16[8 * hh + 2], r16[8 * hh + 3]);
-                        o.z = pack_f16x2(r16[8 * hh + 4], r16[8 * hh + 5]);
-                        o.w = pack_f16x2(r16[8 * hh + 6], r16[8 * hh + 7]);
-                        *reinterpret_cast<uint4 *>(X + half * X_HALF + sw128_offset(r, 16 * q + 8 * hh)) = o;
-                    }
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint4 o;
+                    o.x = pack_f16x2(w[8 * ch + 0], w[8 * ch + 1]);
+                    o.y = pack_f16x2(w[8 * ch + 2], w[8 * ch + 3]);
+                    o.z = pack_f16x2(w[8 * ch + 4], w[8 * ch + 5]);
+                    o.w = pack_f16x2(w[8 * ch + 6], w[8 * ch + 7]);
+                    *reinterpret_cast<uint4 *>(X + half * X_HALF + sw128_offset(r, 8 * ch)) = o;
                 }
             }
             fence_proxy_async_smem();
@@ -565,20 +562,16 @@ chunk_tc_kernel(TcParams p)
             const int64_t tok0 = t0 + (int64_t)c * C;
             const int L = (t1 - tok0 < C) ? (int)(t1 - tok0) : C;
             const uint32_t d5 = tmem + TM_D5 + 32 * s;
-            if (!mbar_wait(&bars[B_S1], c & 1)) fail();
+            if (st == 0 && !mbar_wait(&bars[B_S1], c & 1)) fail();
+            named_bar_sync(2, SG_THREADS);
             tc_fence_after();
             // U = -(D5 rows 0-63) -> f16 MN-major [token][32]
             if (warp < 2) {
                 const uint32_t ta = d5 + ((uint32_t)(32 * warp) << 16);
                 float u[32];
+                tmem_ld32_sync(ta, u);
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    float r16[16];
-                    tmem_ld16(ta + 16 * q, r16);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) u[16 * q + e] = -r16[e];
-                }
+                for (int e = 0; e < 32; ++e) u[e] = -u[e];
 #pragma unroll
                 for (int j = 0; j < DVB; j += 8) {
                     uint4 o;
@@ -609,37 +602,28 @@ chunk_tc_kernel(TcParams p)
                             smem_desc(sbase + OFF_UB + ks * 1024, 16, 512, SW_64B), idm, 1);
                 umma_commit(&bars[B_MU]);
             }
-            if (!mbar_wait(&bars[B_S2], c & 1)) fail();
+            if (st == 0 && !mbar_wait(&bars[B_S2], c & 1)) fail();
+            named_bar_sync(2, SG_THREADS);
             tc_fence_after();
             {   // S <- gamma S + Kend^T U
                 const uint32_t ta = tmem + TM_D7 + ((uint32_t)(32 * warp) << 16);
                 const float g = gam[s * 128 + st];
+                float d7[32];
+                tmem_ld32_sync(ta, d7);
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    float r16[16];
-                    tmem_ld16(ta + 16 * q, r16);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) S[16 * q + e] = g * S[16 * q + e] + r16[e];
-                }
+                for (int e = 0; e < 32; ++e) S[e] = g * S[e] + d7[e];
                 store_state();
             }
             fence_proxy_async_smem();
-            // every scan thread observes the MU commit: it also guards UB and D5[s]
-            if (!mbar_wait(&bars[B_MU], c & 1)) fail();
+            // the MU commit also guards UB and D5[s]
+            if (st == 0 && !mbar_wait(&bars[B_MU], c & 1)) fail();
+            named_bar_sync(2, SG_THREADS);
             tc_fence_after();
             if (warp >= 2) {                 // O = D5 rows 64-127 -> out
                 const int r = st - 64;
                 const uint32_t ta = d5 + ((uint32_t)(32 * warp) << 16);
                 float o32[32];
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    float r16[16];
-                    tmem_ld16(ta + 16 * q, r16);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) o32[16 * q + e] = r16[e];
-                }
+                tmem_ld32_sync(ta, o32);
                 if (r < L) {
                     TO *dst = reinterpret_cast<TO *>(p.out) + ((size_t)(tok0 + r) * H + h) * DK + j0;
                     if constexpr (sizeof(TO) == 4) {

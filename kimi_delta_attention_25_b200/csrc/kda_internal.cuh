@@ -13,6 +13,20 @@ constexpr int kHeadDim = 128;   // d_k = d_v supported by every kernel
 constexpr int kChunk = 64;      // chunk length of the prefill (tokens)
 constexpr size_t kStatusBytes = 256;  // workspace prefix holding the device status word
 
+// Two-pass bf16 prefill: per (chunk slot, head) block of prepared operands in the workspace,
+// laid out as the scan pass wants them in shared memory (see chunk_prep.cu).
+constexpr uint32_t kPrepWQOff = 0;          // W / Qt, 32 KiB
+constexpr uint32_t kPrepTbOff = 32768;      // Tb, 8 KiB
+constexpr uint32_t kPrepMOff = 40960;       // M, 8 KiB
+constexpr uint32_t kPrepKEOff = 49152;      // Kend, 16 KiB
+constexpr uint32_t kPrepGammaOff = 65536;   // gamma, 512 B
+constexpr size_t kPrepBlockBytes = 66048;
+
+// Chunk slots per head: slot(sequence n, chunk c) = floor(first token / 64) + n.
+__host__ __device__ inline long long prep_slots(long long total_tokens, int n_seqs) {
+    return total_tokens / kChunk + n_seqs + 1;
+}
+
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 
@@ -66,9 +80,14 @@ struct PrefillArgs {
 cudaError_t launch_chunk_fp32(const PrefillArgs &a, kda_dtype_t dtype, kda_dtype_t out_dtype,
                               cudaStream_t stream);
 
-// Tensor-core (tcgen05) chunk path for bf16 q/k/v; fp32 state and accumulation.
+// Tensor-core (tcgen05) chunk path for bf16 q/k/v in one kernel (no workspace beyond the status).
 bool chunk_tc_supported(const PrefillArgs &a);
 cudaError_t launch_chunk_tc(const PrefillArgs &a, kda_dtype_t out_dtype, cudaStream_t stream);
+
+// Two-pass tensor-core chunk path for bf16 q/k/v: prepared operands go through the workspace.
+cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slots, cudaStream_t stream);
+cudaError_t launch_chunk_scan(const PrefillArgs &a, const unsigned char *ws, int n_slots,
+                              kda_dtype_t out_dtype, cudaStream_t stream);
 
 // Decode step (memory-bound state update in place).
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,

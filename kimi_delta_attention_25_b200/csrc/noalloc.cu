@@ -77,9 +77,10 @@ extern "C" kda_status_t kda_chunk_fwd_noalloc(const void *q, const void *k, cons
             return KDA_ERR_INVALID_ARG;
     }
     if ((S0 && !aligned_to(S0, 16)) || (S_final && !aligned_to(S_final, 16))) return KDA_ERR_INVALID_ARG;
-    // sizes whose scratch need exceeds the static array are refused
-    const size_t need = kda_chunk_fwd_workspace_size(B, T, H, N, dk, dv, dtype);
-    if (need == 0 || need > kNoAllocScratchBytes) return KDA_ERR_UNSUPPORTED;
+    // This entry point runs the single-kernel prefill, whose only scratch is the status header;
+    // a need beyond the static array is refused.
+    const size_t need = kStatusBytes;
+    if (need > kNoAllocScratchBytes) return KDA_ERR_UNSUPPORTED;
 
     void *scratch = nullptr;
     kda_status_t st = scratch_address(&scratch);
