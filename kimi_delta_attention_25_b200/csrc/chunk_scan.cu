@@ -9,11 +9,14 @@
 // representation, KimiLinear KDA/MLA tutorial (icman.com.cn), sec. 3 and 6.)
 //
 // One CTA per (sequence, head, 32-wide block of d_v): the value columns of S evolve independently.
-// Warp 4 is the producer: it bulk-copies each chunk's prepared block (W/Qt, Tb, M, Kend, gamma;
-// already in the swizzled shared-memory layout) into a two-stage ring with cp.async.bulk, tracked
-// by mbarriers with transaction counts. Warps 0-3 run the chain; the v block of the next chunk is
-// loaded into registers while the current chunk is in flight. Only the tensor-core instructions of
-// the chain sit between consecutive chunks.
+// Three roles, coupled only by mbarriers (no group-wide barrier inside the chunk loop):
+//   warp 5 (lane 0)   issues every tcgen05.mma and commit;
+//   warp 4            loader: bulk-copies each chunk's prepared block (W/Qt, Tb, M, Kend, gamma,
+//                     already in the swizzled layout) into a two-stage ring and converts the v
+//                     block to f16 beside it;
+//   warps 0-3         epilogues: U (TMEM -> f16 smem), the fp32 state update, the outputs.
+// Only S1 -> U -> S2 -> S sits on the serial chain; the next chunk's seed and the output product
+// are queued behind S2, and the output epilogue uses the other half of the double-buffered D5.
 #include "kda_internal.cuh"
 #include "sm100.cuh"
 
@@ -25,8 +28,7 @@ using namespace sm100;
 constexpr int C = kChunk;
 constexpr int DK = kHeadDim;
 constexpr int DVB = 32;
-constexpr int SG = 128;                       // scan threads (warps 0-3)
-constexpr int NT = SG + 32;                   // + producer warp
+constexpr int NT = 192;                       // warps 0-3 epilogue, 4 loader, 5 MMA issuer
 
 // one ring stage (offsets inside a stage; stages are 1024-aligned)
 constexpr uint32_t ST_WQ = 0;                 // 32 KB: W rows 0-63, Qt rows 64-127 (two halves)
@@ -38,18 +40,31 @@ constexpr uint32_t STAGE = 78848;             // 77 KB
 constexpr uint32_t OFF_SB = 2 * STAGE;        // S (f16), 128 rows x 64 B
 constexpr uint32_t OFF_UB = OFF_SB + 8192;    // U (f16), 64 rows x 64 B
 constexpr uint32_t OFF_BAR = OFF_UB + 4096;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 128;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
 static_assert(SMEM_ALLOC <= 232448, "shared memory plan exceeds 227 KiB");
 static_assert(ST_G + 512 <= STAGE && STAGE % 1024 == 0, "stage layout");
 
 constexpr uint32_t BLOCK_TX = 32768 + 8192 + 8192 + 16384 + 512;   // bytes copied per chunk
 
-constexpr uint32_t TMEM_COLS = 64;
-constexpr uint32_t TM_D5 = 0;
-constexpr uint32_t TM_D7 = 32;
+constexpr uint32_t TMEM_COLS = 128;
+constexpr uint32_t TM_D5 = 0;                 // 2 x 32 columns: -U | O, by chunk parity
+constexpr uint32_t TM_D7 = 64;                // 32 columns: Kend^T U
 
-enum { B_FULL = 0, B_EMPTY = 2, B_S1 = 4, B_S2 = 5, B_MU = 6, N_BARS = 7 };
+// mbarriers: [2] = by stage / chunk parity. A barrier that one role waits on never runs two phases
+// ahead of that role: every arrival on it depends, through another barrier, on the waiter having
+// consumed the previous phase (per-parity barriers where that would not hold otherwise).
+enum {
+    B_FULL = 0,      // 2: stage loaded (bulk-copy bytes + loader's v arrival)           count 2
+    B_EMPTY = 2,     // 2: stage consumed (MU commit + 128 epilogue threads)              count 129
+    B_D5FREE = 4,    // 2: outputs of D5[s] read (64 epilogue threads)                    count 64
+    B_MU = 6,        // 2: output product of D5[s] complete (commit)                      count 1
+    B_SREADY = 8,    // state of the next chunk in smem (128 epilogue threads)            count 128
+    B_UREADY = 9,    // U in smem (64 epilogue threads)                                   count 64
+    B_S1 = 10, B_S2 = 11,   // MMA completions (commit)                                   count 1
+    B_DRAIN = 12,    // every MMA of the CTA complete (final commit)                      count 1
+    N_BARS = 13
+};
 
 struct ScanParams {
     const __nv_bfloat16 *v;
@@ -95,13 +110,23 @@ chunk_scan_kernel(ScanParams p)
 
     if (warp == 0) { tmem_alloc(tmem_slot, TMEM_COLS); tmem_relinquish(); }
     if (tid == 0) {
-        for (int i = 0; i < N_BARS; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars[B_FULL + i], 2);
+            mbar_init(&bars[B_EMPTY + i], 129);
+            mbar_init(&bars[B_D5FREE + i], 64);
+            mbar_init(&bars[B_MU + i], 1);
+        }
+        mbar_init(&bars[B_SREADY], 128);
+        mbar_init(&bars[B_UREADY], 64);
+        mbar_init(&bars[B_S1], 1);
+        mbar_init(&bars[B_S2], 1);
+        mbar_init(&bars[B_DRAIN], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     for (int i = tid; i < 2 * 8192 / 16; i += NT) {      // zero rows 64-127 of both Y regions
-        const int st = i / (8192 / 16), o = i % (8192 / 16);
-        reinterpret_cast<uint4 *>(sm + st * STAGE + ST_Y + 8192)[o] = make_uint4(0, 0, 0, 0);
+        const int stg = i / (8192 / 16), o = i % (8192 / 16);
+        reinterpret_cast<uint4 *>(sm + stg * STAGE + ST_Y + 8192)[o] = make_uint4(0, 0, 0, 0);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -109,32 +134,110 @@ chunk_scan_kernel(ScanParams p)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     auto fail = [&]() { set_status(p.status, KDA_ERR_TIMEOUT); *abort_flag = 1; };
+    // a wait whose outcome is the same for the whole (converged) warp, so that warp-collective
+    // tcgen05.ld never runs with some lanes gone
+    auto warp_wait = [&](uint64_t *bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity)) != 0;
+    };
+    auto warp_abort = [&]() { return __any_sync(0xffffffffu, *abort_flag != 0) != 0; };
 
-    if (warp == 4) {
-        // ================================================================ producer (one lane)
+    if (warp == 5) {
+        // ======================================================================== MMA issuer
         if (lane == 0) {
-            uint32_t issued[2] = {0u, 0u};
-            for (int c = 0; c < nchunks; ++c) {
+            uint32_t n_issued = 0;
+            const uint32_t id_seed = idesc_f16(128, 32, 0, 1) | (1u << 13);   // -[Tb; 0] V
+            const uint32_t id_s1 = idesc_f16(128, 32, 0, 1);                  // [W; Qt] S
+            const uint32_t id_s2 = idesc_f16(128, 32, 1, 1);                  // Kend^T U
+            const uint32_t id_mu = idesc_f16(128, 32, 0, 1);                  // [0; M] U
+            for (int c = 0; c < nchunks && !*abort_flag; ++c) {
                 const int s = c & 1;
-                if (*abort_flag) break;
-                if (c >= 2 && !mbar_wait(&bars[B_EMPTY + s], ((c >> 1) - 1) & 1)) { fail(); break; }
+                const uint32_t astg = sbase + s * STAGE;
+                const uint32_t d5 = tmem + TM_D5 + 32 * s;
+                if (!mbar_wait(&bars[B_FULL + s], (c >> 1) & 1)) { fail(); break; }
+                ++n_issued;
+                if (c >= 2 && !mbar_wait(&bars[B_D5FREE + s], ((c >> 1) - 1) & 1)) { fail(); break; }
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_ss(d5, smem_desc(astg + ST_Y + ks * 32, 16, 1024, SW_128B),
+                            smem_desc(astg + ST_V + ks * 1024, 16, 512, SW_64B), id_seed, ks > 0);
+                if (!mbar_wait(&bars[B_SREADY], c & 1)) { fail(); break; }
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t kh = ks >> 2, ko = (ks & 3) * 32;
+                    umma_ss(d5, smem_desc(astg + ST_WQ + kh * 16384 + ko, 16, 1024, SW_128B),
+                            smem_desc(sbase + OFF_SB + ks * 1024, 16, 512, SW_64B), id_s1, 1);
+                }
+                umma_commit(&bars[B_S1]);
+                if (!mbar_wait(&bars[B_UREADY], c & 1)) { fail(); break; }
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_ss(tmem + TM_D7, smem_desc(astg + ST_KE + ks * 2048, 8192, 1024, SW_128B),
+                            smem_desc(sbase + OFF_UB + ks * 1024, 16, 512, SW_64B), id_s2, ks > 0);
+                umma_commit(&bars[B_S2]);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_ss(d5, smem_desc(astg + ST_Y + 8192 + ks * 32, 16, 1024, SW_128B),
+                            smem_desc(sbase + OFF_UB + ks * 1024, 16, 512, SW_64B), id_mu, 1);
+                umma_commit(&bars[B_MU + s]);
+                umma_commit(&bars[B_EMPTY + s]);      // its MMA share of releasing stage s
+            }
+            if (n_issued) {                           // every MMA complete before TMEM is freed
+                umma_commit(&bars[B_DRAIN]);
+                if (!mbar_wait(&bars[B_DRAIN], 0, 100000000LL)) set_status(p.status, KDA_ERR_TIMEOUT);
+            }
+        }
+    } else if (warp == 4) {
+        // ============================================================================ loader
+        uint32_t issued[2] = {0u, 0u};
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c & 1;
+            unsigned char *stg = sm + s * STAGE;
+            if (warp_abort()) break;
+            int ok = 1;
+            if (c >= 2 && lane == 0) ok = mbar_wait(&bars[B_EMPTY + s], ((c >> 1) - 1) & 1);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) { if (lane == 0) fail(); break; }
+            if (lane == 0) {
                 const unsigned char *blk = p.ws + ((size_t)h * p.n_slots + (first_slot + c)) * kPrepBlockBytes;
-                unsigned char *stg = sm + s * STAGE;
                 mbar_arrive_expect_tx(&bars[B_FULL + s], BLOCK_TX);
                 bulk_g2s(stg + ST_WQ, blk + kPrepWQOff, 32768, &bars[B_FULL + s]);
                 bulk_g2s(stg + ST_Y, blk + kPrepTbOff, 8192, &bars[B_FULL + s]);
                 bulk_g2s(stg + ST_Y + 16384, blk + kPrepMOff, 8192, &bars[B_FULL + s]);
                 bulk_g2s(stg + ST_KE, blk + kPrepKEOff, 16384, &bars[B_FULL + s]);
                 bulk_g2s(stg + ST_G, blk + kPrepGammaOff, 512, &bars[B_FULL + s]);
-                ++issued[s];
             }
-            // no copy may still be landing when the CTA exits
+            ++issued[s];
+            // v block (bf16 -> f16): lane -> rows 2 lane, 2 lane + 1
+            const int64_t tok0 = t0 + (int64_t)c * C;
+            const int L = (t1 - tok0 < C) ? (int)(t1 - tok0) : C;
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const int r = 2 * lane + rr;
+                uint4 raw[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    raw[u] = (r < L) ? ldg_nc(p.v + ((size_t)(tok0 + r) * H + h) * DK + j0 + 8 * u)
+                                     : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    uint4 o;
+                    o.x = bf16x2_to_f16x2(raw[u].x); o.y = bf16x2_to_f16x2(raw[u].y);
+                    o.z = bf16x2_to_f16x2(raw[u].z); o.w = bf16x2_to_f16x2(raw[u].w);
+                    *reinterpret_cast<uint4 *>(stg + ST_V + sw64_offset(r, 8 * u)) = o;
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[B_FULL + s]);
+        }
+        if (lane == 0)       // no copy may still be landing when the CTA exits
             for (int s = 0; s < 2; ++s)
                 if (issued[s]) mbar_wait(&bars[B_FULL + s], (issued[s] - 1) & 1, 100000000LL);
-        }
     } else {
-        // ================================================================ scan chain
-        const int st = tid;
+        // ========================================================================= epilogues
+        const int st = tid;                   // key channel / TMEM lane
         float S[DVB];
         {
             const size_t sidx = (((size_t)n * H + h) * DK + st) * DK + j0;
@@ -153,70 +256,23 @@ chunk_scan_kernel(ScanParams p)
                 *reinterpret_cast<uint4 *>(sm + OFF_SB + sw64_offset(st, j)) = v;
             }
         };
-        // v block of a chunk: thread -> row st >> 1, columns 16 (st & 1)..+15
-        auto load_v = [&](int c, uint4 (&vr)[2]) {
-            const int64_t tok0 = t0 + (int64_t)c * C;
-            const int L = (t1 - tok0 < C) ? (int)(t1 - tok0) : C;
-            const int r = st >> 1;
-            if (r < L) {
-                const __nv_bfloat16 *src = p.v + ((size_t)(tok0 + r) * H + h) * DK + j0 + 16 * (st & 1);
-                vr[0] = ldg_nc(src);
-                vr[1] = ldg_nc(src + 8);
-            } else {
-                vr[0] = make_uint4(0, 0, 0, 0);
-                vr[1] = vr[0];
-            }
-        };
         store_state();
-        uint4 vr[2];
-        if (nchunks > 0) load_v(0, vr);
-        uint32_t n_commits = 0;
+        fence_proxy_async_smem();
+        mbar_arrive(&bars[B_SREADY]);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c & 1;
             const int64_t tok0 = t0 + (int64_t)c * C;
             const int L = (t1 - tok0 < C) ? (int)(t1 - tok0) : C;
-            unsigned char *stg = sm + s * STAGE;
-            const uint32_t astg = sbase + s * STAGE;
-            {   // v (bf16 -> f16) into the stage
-                const int r = st >> 1;
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    uint4 o;
-                    o.x = bf16x2_to_f16x2(vr[u].x); o.y = bf16x2_to_f16x2(vr[u].y);
-                    o.z = bf16x2_to_f16x2(vr[u].z); o.w = bf16x2_to_f16x2(vr[u].w);
-                    *reinterpret_cast<uint4 *>(stg + ST_V + sw64_offset(r, 16 * (st & 1) + 8 * u)) = o;
-                }
-            }
-            fence_proxy_async_smem();
-            // every scan thread observes the stage's arrival (it reads gamma from it directly)
-            if (!mbar_wait(&bars[B_FULL + s], (c >> 1) & 1)) fail();
-            tc_fence_before();
-            named_bar_sync(1, SG);
-            if (*abort_flag) break;
-            tc_fence_after();
-            if (st == 0) {
-                ++n_commits;
-                const uint32_t ids = idesc_f16(128, 32, 0, 1) | (1u << 13);   // -[Tb; 0] V
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    umma_ss(tmem + TM_D5, smem_desc(astg + ST_Y + ks * 32, 16, 1024, SW_128B),
-                            smem_desc(astg + ST_V + ks * 1024, 16, 512, SW_64B), ids, ks > 0);
-                const uint32_t id = idesc_f16(128, 32, 0, 1);                  // += [W; Qt] S
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t kh = ks >> 2, ko = (ks & 3) * 32;
-                    umma_ss(tmem + TM_D5, smem_desc(astg + ST_WQ + kh * 16384 + ko, 16, 1024, SW_128B),
-                            smem_desc(sbase + OFF_SB + ks * 1024, 16, 512, SW_64B), id, 1);
-                }
-                umma_commit(&bars[B_S1]);
-            }
-            if (c + 1 < nchunks) load_v(c + 1, vr);
-            if (st == 0 && !mbar_wait(&bars[B_S1], c & 1)) fail();
-            named_bar_sync(1, SG);
-            tc_fence_after();
-            if (warp < 2) {                  // U = -(rows 0-63) -> f16, MN-major [token][32]
+            const uint32_t d5 = tmem + TM_D5 + 32 * s;
+            if (warp_abort()) break;
+            // gamma of this chunk (read from the stage after observing its arrival directly)
+            if (!warp_wait(&bars[B_FULL + s], (c >> 1) & 1)) { fail(); break; }
+            const float g = reinterpret_cast<const float *>(sm + s * STAGE + ST_G)[st];
+            if (warp < 2) {                   // U = -(D5 rows 0-63) -> f16, MN-major [token][32]
+                if (!warp_wait(&bars[B_S1], c & 1)) { fail(); break; }
+                tc_fence_after();
                 float u[32];
-                tmem_ld32_sync(tmem + TM_D5 + ((uint32_t)(32 * warp) << 16), u);
+                tmem_ld32_sync(d5 + ((uint32_t)(32 * warp) << 16), u);
 #pragma unroll
                 for (int j = 0; j < DVB; j += 8) {
                     uint4 o;
@@ -224,45 +280,32 @@ chunk_scan_kernel(ScanParams p)
                     o.z = pack_f16x2(-u[j + 4], -u[j + 5]); o.w = pack_f16x2(-u[j + 6], -u[j + 7]);
                     *reinterpret_cast<uint4 *>(sm + OFF_UB + sw64_offset(st, j)) = o;
                 }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&bars[B_UREADY]);
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar_sync(1, SG);
+            // S <- gamma S + Kend^T U, then hand the new state to the next chunk's S1
+            if (!warp_wait(&bars[B_S2], c & 1)) { fail(); break; }
             tc_fence_after();
-            if (st == 0) {
-                const uint32_t id2 = idesc_f16(128, 32, 1, 1);                 // Kend^T U
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    umma_ss(tmem + TM_D7, smem_desc(astg + ST_KE + ks * 2048, 8192, 1024, SW_128B),
-                            smem_desc(sbase + OFF_UB + ks * 1024, 16, 512, SW_64B), id2, ks > 0);
-                umma_commit(&bars[B_S2]);
-                const uint32_t idm = idesc_f16(128, 32, 0, 1);                 // += [0; M] U
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    umma_ss(tmem + TM_D5, smem_desc(astg + ST_Y + 8192 + ks * 32, 16, 1024, SW_128B),
-                            smem_desc(sbase + OFF_UB + ks * 1024, 16, 512, SW_64B), idm, 1);
-                umma_commit(&bars[B_MU]);
-            }
-            if (st == 0 && !mbar_wait(&bars[B_S2], c & 1)) fail();
-            named_bar_sync(1, SG);
-            tc_fence_after();
-            {   // S <- gamma S + Kend^T U
-                const float g = reinterpret_cast<const float *>(stg + ST_G)[st];
+            {
                 float d7[32];
                 tmem_ld32_sync(tmem + TM_D7 + ((uint32_t)(32 * warp) << 16), d7);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) S[e] = g * S[e] + d7[e];
                 store_state();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&bars[B_SREADY]);
+                mbar_arrive(&bars[B_EMPTY + s]);      // gamma of stage s has been read
             }
-            fence_proxy_async_smem();
-            if (st == 0 && !mbar_wait(&bars[B_MU], c & 1)) fail();
-            tc_fence_before();
-            named_bar_sync(1, SG);
-            tc_fence_after();
-            if (warp >= 2) {                 // O = rows 64-127 -> out
+            if (warp >= 2) {                  // O = D5 rows 64-127 -> out
+                if (!warp_wait(&bars[B_MU + s], (c >> 1) & 1)) { fail(); break; }
+                tc_fence_after();
                 const int r = st - 64;
                 float o32[32];
-                tmem_ld32_sync(tmem + TM_D5 + ((uint32_t)(32 * warp) << 16), o32);
+                tmem_ld32_sync(d5 + ((uint32_t)(32 * warp) << 16), o32);
+                tc_fence_before();
+                mbar_arrive(&bars[B_D5FREE + s]);
                 if (r < L) {
                     TO *dst = reinterpret_cast<TO *>(p.out) + ((size_t)(tok0 + r) * H + h) * DK + j0;
                     if constexpr (sizeof(TO) == 4) {
@@ -281,15 +324,6 @@ chunk_scan_kernel(ScanParams p)
                     }
                 }
             }
-            tc_fence_before();
-            named_bar_sync(1, SG);
-            if (*abort_flag) break;
-            if (st == 0) mbar_arrive(&bars[B_EMPTY + s]);      // stage s may be refilled
-        }
-        if (*abort_flag && st == 0 && n_commits) {             // drain in-flight MMAs (bounded)
-            mbar_wait(&bars[B_S1], (n_commits - 1) & 1, 100000000LL);
-            mbar_wait(&bars[B_S2], (n_commits - 1) & 1, 100000000LL);
-            mbar_wait(&bars[B_MU], (n_commits - 1) & 1, 100000000LL);
         }
         if (p.S_final && !*abort_flag) {
             const size_t sidx = (((size_t)n * H + h) * DK + st) * DK + j0;
