@@ -7,18 +7,23 @@
 // e^{g_{L-1}}:
 //   Kt = K f, Qt = Q f, Kend = K b, Kh = K b / gamma;  A = StrictLower(diag(beta) Kt Kh^T);
 //   M = tril(Qt Kh^T);  Tb = (I + A)^{-1} diag(beta);  W = Tb Kt.
-// The second pass (chunk_scan.cu) then runs the state recurrence over chunks with these operands.
+// With U = Tb V - W S the chunk's writes, the output O = Qt S + M U regroups as
+//   O = (Qt - M W) S + (M Tb) V,
+// so the scan pass never needs M itself: this pass also forms M Tb and Qt - M W. The second pass
+// (chunk_scan.cu) then runs the state recurrence over chunks with these operands.
 //
 // The chunks are independent, so this pass is a plain data-parallel grid: one CTA (8 warps) per
 // (chunk slot, head), two CTAs per SM. Results go to the workspace in exactly the byte layout the
 // scan wants in shared memory (f16, 128-byte swizzled canonical UMMA tiles), so the scan moves each
-// block with a few bulk copies:
-//   [0, 32K)    W (rows 0-63) and Qt (rows 64-127), two 64-channel halves, K-major
-//   [32K, 40K)  Tb, 64 x 64, K-major        [40K, 48K)  M, 64 x 64, K-major
+// block with one bulk copy:
+//   [0, 32K)    X: W (rows 0-63) and Qt - M W (rows 64-127), two 64-channel halves, K-major
+//   [32K, 48K)  Y: -Tb (rows 0-63) and M Tb (rows 64-127), 64 token columns, K-major
 //   [48K, 64K)  Kend, two halves of 64 tokens x 64 channels (the MN-major A of Kend^T U)
 //   [64K, +512) gamma (fp32)
 // A chunk slot is floor(first_token / 64) + sequence, which is unique per (sequence, chunk) and
 // below floor(total_tokens / 64) + N + 1.
+#include <cuda_fp16.h>
+
 #include "kda_internal.cuh"
 #include "sm100.cuh"
 
@@ -38,18 +43,21 @@ constexpr float kMinChunkDecay = 3.0517578125e-05f;
 // shared memory (1024-aligned base)
 constexpr uint32_t OFF_QT = 0;               // Qt (f16), two halves of 64 x 128 B
 constexpr uint32_t OFF_KT = 16384;           // Kt
-constexpr uint32_t OFF_KH = 32768;           // Kh; after P1: A^T (fp32, column-major)
-constexpr uint32_t OFF_TB = 49152;           // Tb (f16), 64 x 128 B
+constexpr uint32_t OFF_TB = 32768;           // Tb (f16), 64 x 128 B; N-block 0 of [Tb | W]
+constexpr uint32_t OFF_KH = 40960;           // Kh; after P1: A^T (fp32, column-major);
+                                             // after P3: W (f16), N-blocks 1-2 of [Tb | W]
+constexpr uint32_t OFF_M = 57344;            // M (f16), 64 x 128 B
 constexpr int LDT = 68;
-constexpr uint32_t OFF_TF = 57344;           // T (fp32, stride LDT) = 17408 B
+constexpr uint32_t OFF_TF = 65536;           // T (fp32, stride LDT) = 17408 B
 constexpr uint32_t OFF_PS = OFF_TF + 17408;  // 4 KB: row-block products, then inverse scratch
 constexpr uint32_t OFF_BET = OFF_PS + 4096;  // 64 fp32
 constexpr uint32_t OFF_BAR = OFF_BET + 256;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
 
-constexpr uint32_t TMEM_COLS = 128;
-constexpr uint32_t TM_D1A = 0;               // Qt Kh^T  (M=64 layout), later W (cols 0-127)
+constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t TM_D1A = 0;               // Qt Kh^T  (M=64 layout), later W (cols 0-127),
+                                             // then M [Tb | W] (cols 0-191)
 constexpr uint32_t TM_D1B = 64;              // Kt Kh^T
 
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
@@ -292,11 +300,9 @@ chunk_prep_kernel(PrepParams p)
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) suf[e] *= a[x][e];
-            const uint2 vqt = make_uint2(oqt[0], oqt[1]);
             *reinterpret_cast<uint2 *>(sm + OFF_KT + kh * 8192 + off) = make_uint2(okt[0], okt[1]);
-            *reinterpret_cast<uint2 *>(sm + OFF_QT + kh * 8192 + off) = vqt;
+            *reinterpret_cast<uint2 *>(sm + OFF_QT + kh * 8192 + off) = make_uint2(oqt[0], oqt[1]);
             *reinterpret_cast<uint2 *>(sm + OFF_KH + kh * 8192 + off) = make_uint2(okh[0], okh[1]);
-            *reinterpret_cast<uint2 *>(blk + kPrepWQOff + kh * 16384 + 64 * 128 + off) = vqt;
             *reinterpret_cast<uint2 *>(blk + kPrepKEOff + kh * 8192 + off) = make_uint2(oke[0], oke[1]);
         }
     }
@@ -322,7 +328,7 @@ chunk_prep_kernel(PrepParams p)
     if (tid == 0 && !mbar_wait(bar, 0)) failed = 1;
     __syncthreads();
     tc_fence_after();
-    // ---- P1 epilogue: warps 0-3 -> M (f16 -> workspace); warps 4-7 -> A^T (fp32, smem)
+    // ---- P1 epilogue: warps 0-3 -> M (f16, smem); warps 4-7 -> A^T (fp32, smem)
     {
         const int q4 = warp & 3, half = warp >> 2;
         float v[64];
@@ -338,7 +344,7 @@ chunk_prep_kernel(PrepParams p)
                         const int i = 8 * ch + 2 * u;
                         w4[u] = pack_f16x2(i <= r ? v[i] : 0.f, i + 1 <= r ? v[i + 1] : 0.f);
                     }
-                    *reinterpret_cast<uint4 *>(blk + kPrepMOff + sw128_offset(r, 8 * ch)) =
+                    *reinterpret_cast<uint4 *>(sm + OFF_M + sw128_offset(r, 8 * ch)) =
                         make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }
             } else {
@@ -350,7 +356,7 @@ chunk_prep_kernel(PrepParams p)
     }
     tc_fence_before();
     __syncthreads();
-    // ---- T = (I + A)^{-1};  Tb = T diag(beta) -> f16 (smem for P3, and workspace)
+    // ---- T = (I + A)^{-1};  Tb = T diag(beta) -> f16 (smem for P3 and P4; -Tb to the workspace)
     inverse64(tid, AT, Tf, Ps);
     {
         const int r = tid >> 2, c0 = (tid & 3) * 16;
@@ -371,7 +377,9 @@ chunk_prep_kernel(PrepParams p)
             }
             const uint4 o = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             *reinterpret_cast<uint4 *>(sm + OFF_TB + sw128_offset(r, cb)) = o;
-            *reinterpret_cast<uint4 *>(blk + kPrepTbOff + sw128_offset(r, cb)) = o;
+            const uint32_t sgn = 0x80008000u;        // f16 sign bits: -Tb
+            *reinterpret_cast<uint4 *>(blk + kPrepYOff + sw128_offset(r, cb)) =
+                make_uint4(o.x ^ sgn, o.y ^ sgn, o.z ^ sgn, o.w ^ sgn);
         }
     }
     fence_proxy_async_smem();
@@ -390,7 +398,8 @@ chunk_prep_kernel(PrepParams p)
     if (tid == 0 && !failed && !mbar_wait(bar, 1)) failed = 1;
     __syncthreads();
     tc_fence_after();
-    // ---- W epilogue (M=64 layout: lanes 0-15 of each quadrant), warps 0-3 cols 0-63, 4-7 cols 64-127
+    // ---- W epilogue (M=64 layout: lanes 0-15 of each quadrant), warps 0-3 cols 0-63, 4-7 cols 64-127:
+    //      W -> workspace (X rows 0-63) and -> smem as N-blocks 1-2 of [Tb | W] (A^T is dead by now)
     {
         const int q4 = warp & 3, half = warp >> 2;
         float w[64];
@@ -404,7 +413,63 @@ chunk_prep_kernel(PrepParams p)
                 o.y = pack_f16x2(w[8 * ch + 2], w[8 * ch + 3]);
                 o.z = pack_f16x2(w[8 * ch + 4], w[8 * ch + 5]);
                 o.w = pack_f16x2(w[8 * ch + 6], w[8 * ch + 7]);
-                *reinterpret_cast<uint4 *>(blk + kPrepWQOff + half * 16384 + sw128_offset(r, 8 * ch)) = o;
+                *reinterpret_cast<uint4 *>(blk + kPrepXOff + half * 16384 + sw128_offset(r, 8 * ch)) = o;
+                *reinterpret_cast<uint4 *>(sm + OFF_KH + half * 8192 + sw128_offset(r, 8 * ch)) = o;
+            }
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // ---- P4: M [Tb | W] (M=64, N=192, K=64; B = [Tb | W] MN-major, N-blocks 8 KiB apart) -> cols 0-191
+    if (tid == 0 && !failed) {
+        const uint32_t id = idesc_f16(64, 192, 0, 1);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            umma_ss(tmem + TM_D1A, smem_desc(sbase + OFF_M + ks * 32, 16, 1024, SW_128B),
+                    smem_desc(sbase + OFF_TB + ks * 2048, 8192, 1024, SW_128B), id, ks > 0);
+        umma_commit(bar);
+        if (!mbar_wait(bar, 0)) failed = 1;
+    }
+    __syncthreads();
+    tc_fence_after();
+    // ---- P4 epilogue: warps 0-3: M Tb (cols 0-63) -> Y rows 64-127, then Qt - M W for channels
+    //      0-63 (cols 64-127); warps 4-7: Qt - M W for channels 64-127 (cols 128-191) -> X rows 64-127
+    {
+        const int q4 = warp & 3, half = warp >> 2;
+        const int r = 16 * q4 + (lane & 15);
+        const int part_end = half ? 3 : 2;
+        for (int part = half ? 2 : 0; part < part_end; ++part) {   // warps 0-3: parts 0, 1; 4-7: part 2
+            float m[64];
+            tmem_ld64_sync(tmem + ((uint32_t)(32 * q4) << 16) + TM_D1A + 64 * part, m);
+            if (lane < 16) {
+                if (part == 0) {
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        uint4 o;
+                        o.x = pack_f16x2(m[8 * ch + 0], m[8 * ch + 1]);
+                        o.y = pack_f16x2(m[8 * ch + 2], m[8 * ch + 3]);
+                        o.z = pack_f16x2(m[8 * ch + 4], m[8 * ch + 5]);
+                        o.w = pack_f16x2(m[8 * ch + 6], m[8 * ch + 7]);
+                        *reinterpret_cast<uint4 *>(blk + kPrepYOff + sw128_offset(64 + r, 8 * ch)) = o;
+                    }
+                } else {
+                    const int kh = part - 1;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        const uint4 qv = *reinterpret_cast<const uint4 *>(sm + OFF_QT + kh * 8192 + sw128_offset(r, 8 * ch));
+                        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+                        uint32_t o[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const float2 qf = __half22float2(*reinterpret_cast<const __half2 *>(&qw[u]));
+                            o[u] = pack_f16x2(qf.x - m[8 * ch + 2 * u], qf.y - m[8 * ch + 2 * u + 1]);
+                        }
+                        *reinterpret_cast<uint4 *>(blk + kPrepXOff + kh * 16384 + 64 * 128 + sw128_offset(r, 8 * ch)) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                }
             }
         }
     }

@@ -1,9 +1,10 @@
 // chunk_scan.cu -- second pass of the two-pass bf16 prefill: the state recurrence over chunks.
 //
 // For each chunk (operands from chunk_prep.cu) with S the state entering the chunk:
-//   D5  = -[Tb; 0] V                      (the Tb V term; seeds the accumulator)
-//   D5 += [W; Qt] S                       rows 0-63: W S - Tb V = -U,  rows 64-127: Qt S
-//   D7  = Kend^T U ;   D5 += [0; M] U     rows 64-127: O = Qt S + M U
+//   D5  = Y V = [-Tb; M Tb] V             (seeds the accumulator; independent of S)
+//   D5 += X S = [W; Qt - M W] S           rows 0-63: W S - Tb V = -U,  rows 64-127: the output
+//                                         O = Qt S + M U = (Qt - M W) S + M Tb V
+//   D7  = Kend^T U
 //   S  <- Diag(gamma) S + D7              (fp32, registers; thread = key channel)
 // (U = Tb V - W S are the chunk's delta-rule writes; chunk-parallel form with a WY/UT
 // representation, KimiLinear KDA/MLA tutorial (icman.com.cn), sec. 3 and 6.)
@@ -11,12 +12,12 @@
 // One CTA per (sequence, head, 32-wide block of d_v): the value columns of S evolve independently.
 // Three roles, coupled only by mbarriers (no group-wide barrier inside the chunk loop):
 //   warp 5 (lane 0)   issues every tcgen05.mma and commit;
-//   warp 4            loader: bulk-copies each chunk's prepared block (W/Qt, Tb, M, Kend, gamma,
-//                     already in the swizzled layout) into a two-stage ring and converts the v
-//                     block to f16 beside it;
-//   warps 0-3         epilogues: U (TMEM -> f16 smem), the fp32 state update, the outputs.
-// Only S1 -> U -> S2 -> S sits on the serial chain; the next chunk's seed and the output product
-// are queued behind S2, and the output epilogue uses the other half of the double-buffered D5.
+//   warp 4            loader: bulk-copies each chunk's prepared block (X, Y, Kend, gamma, already
+//                     in the swizzled layout) into a three-stage ring with one cp.async.bulk, and
+//                     writes the v block beside it as f16 (loaded into registers one chunk ahead);
+//   warps 0-3         epilogues: U (TMEM -> f16 smem), the outputs, the fp32 state update.
+// Only S1 -> U -> S2 -> S sits on the serial chain; the next chunk's seed is queued behind S2 into
+// the other half of the double-buffered D5, and the outputs are read while S2 runs.
 #include "kda_internal.cuh"
 #include "sm100.cuh"
 
@@ -30,39 +31,37 @@ constexpr int DK = kHeadDim;
 constexpr int DVB = 32;
 constexpr int NT = 192;                       // warps 0-3 epilogue, 4 loader, 5 MMA issuer
 
-// one ring stage (offsets inside a stage; stages are 1024-aligned)
-constexpr uint32_t ST_WQ = 0;                 // 32 KB: W rows 0-63, Qt rows 64-127 (two halves)
-constexpr uint32_t ST_Y = 32768;              // 24 KB: Tb (rows 0-63) | zero (64-127) | M (128-191)
-constexpr uint32_t ST_KE = ST_Y + 24576;      // 16 KB: Kend
-constexpr uint32_t ST_V = ST_KE + 16384;      // 4 KB: v block (f16, 64-byte rows)
-constexpr uint32_t ST_G = ST_V + 4096;        // 512 B: gamma
-constexpr uint32_t STAGE = 78848;             // 77 KB
-constexpr uint32_t OFF_SB = 2 * STAGE;        // S (f16), 128 rows x 64 B
+// one ring stage (offsets inside a stage; stages are 1024-aligned). [0, 66048) is a copy of the
+// workspace block.
+constexpr uint32_t ST_X = kPrepXOff;          // 32 KB: W rows 0-63, Qt - M W rows 64-127 (two halves)
+constexpr uint32_t ST_Y = kPrepYOff;          // 16 KB: -Tb rows 0-63, M Tb rows 64-127
+constexpr uint32_t ST_KE = kPrepKEOff;        // 16 KB: Kend
+constexpr uint32_t ST_G = kPrepGammaOff;      // 512 B: gamma
+constexpr uint32_t ST_V = 66560;              // 4 KB: v block (f16, 64-byte rows)
+constexpr uint32_t STAGE = ST_V + 4096;       // 69 KB
+constexpr int NSTAGE = 3;
+constexpr uint32_t OFF_SB = NSTAGE * STAGE;   // S (f16), 128 rows x 64 B
 constexpr uint32_t OFF_UB = OFF_SB + 8192;    // U (f16), 64 rows x 64 B
 constexpr uint32_t OFF_BAR = OFF_UB + 4096;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
 static_assert(SMEM_ALLOC <= 232448, "shared memory plan exceeds 227 KiB");
-static_assert(ST_G + 512 <= STAGE && STAGE % 1024 == 0, "stage layout");
-
-constexpr uint32_t BLOCK_TX = 32768 + 8192 + 8192 + 16384 + 512;   // bytes copied per chunk
+static_assert(kPrepBlockBytes <= ST_V && STAGE % 1024 == 0 && kPrepBlockBytes % 16 == 0, "stage layout");
 
 constexpr uint32_t TMEM_COLS = 128;
-constexpr uint32_t TM_D5 = 0;                 // 2 x 32 columns: -U | O, by chunk parity
+constexpr uint32_t TM_D5 = 0;                 // 2 x 32 columns: [-U; O], by chunk parity
 constexpr uint32_t TM_D7 = 64;                // 32 columns: Kend^T U
 
-// mbarriers: [2] = by stage / chunk parity. A barrier that one role waits on never runs two phases
-// ahead of that role: every arrival on it depends, through another barrier, on the waiter having
-// consumed the previous phase (per-parity barriers where that would not hold otherwise).
+// mbarriers. A barrier that one role waits on never runs two phases ahead of that role: every
+// arrival on it depends, through another barrier, on the waiter having consumed the previous phase.
 enum {
-    B_FULL = 0,      // 2: stage loaded (bulk-copy bytes + loader's v arrival)           count 2
-    B_EMPTY = 2,     // 2: stage consumed (MU commit + 128 epilogue threads)              count 129
-    B_D5FREE = 4,    // 2: outputs of D5[s] read (64 epilogue threads)                    count 64
-    B_MU = 6,        // 2: output product of D5[s] complete (commit)                      count 1
-    B_SREADY = 8,    // state of the next chunk in smem (128 epilogue threads)            count 128
-    B_UREADY = 9,    // U in smem (64 epilogue threads)                                   count 64
-    B_S1 = 10, B_S2 = 11,   // MMA completions (commit)                                   count 1
-    B_DRAIN = 12,    // every MMA of the CTA complete (final commit)                      count 1
+    B_FULL = 0,      // [3] by stage: block copied (tx bytes) + loader's v arrival               count 2
+    B_EMPTY = 3,     // [3] by stage: consumed (S2 commit + 128 epilogue threads, gamma read)    count 129
+    B_D5FREE = 6,    // [2] by chunk parity: D5 read by the U and output epilogues (128 threads) count 128
+    B_SREADY = 8,    // state of the next chunk in smem (128 epilogue threads)                   count 128
+    B_UREADY = 9,    // U in smem (64 epilogue threads)                                          count 64
+    B_S1 = 10, B_S2 = 11,   // MMA completions (commit)                                          count 1
+    B_DRAIN = 12,    // every MMA of the CTA complete (final commit)                             count 1
     N_BARS = 13
 };
 
@@ -110,12 +109,12 @@ chunk_scan_kernel(ScanParams p)
 
     if (warp == 0) { tmem_alloc(tmem_slot, TMEM_COLS); tmem_relinquish(); }
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NSTAGE; ++i) {
             mbar_init(&bars[B_FULL + i], 2);
             mbar_init(&bars[B_EMPTY + i], 129);
-            mbar_init(&bars[B_D5FREE + i], 64);
-            mbar_init(&bars[B_MU + i], 1);
         }
+        mbar_init(&bars[B_D5FREE + 0], 128);
+        mbar_init(&bars[B_D5FREE + 1], 128);
         mbar_init(&bars[B_SREADY], 128);
         mbar_init(&bars[B_UREADY], 64);
         mbar_init(&bars[B_S1], 1);
@@ -124,11 +123,6 @@ chunk_scan_kernel(ScanParams p)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    for (int i = tid; i < 2 * 8192 / 16; i += NT) {      // zero rows 64-127 of both Y regions
-        const int stg = i / (8192 / 16), o = i % (8192 / 16);
-        reinterpret_cast<uint4 *>(sm + stg * STAGE + ST_Y + 8192)[o] = make_uint4(0, 0, 0, 0);
-    }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -145,17 +139,16 @@ chunk_scan_kernel(ScanParams p)
         // ======================================================================== MMA issuer
         if (lane == 0) {
             uint32_t n_issued = 0;
-            const uint32_t id_seed = idesc_f16(128, 32, 0, 1) | (1u << 13);   // -[Tb; 0] V
-            const uint32_t id_s1 = idesc_f16(128, 32, 0, 1);                  // [W; Qt] S
+            const uint32_t id_seed = idesc_f16(128, 32, 0, 1);                // Y V
+            const uint32_t id_s1 = idesc_f16(128, 32, 0, 1);                  // X S
             const uint32_t id_s2 = idesc_f16(128, 32, 1, 1);                  // Kend^T U
-            const uint32_t id_mu = idesc_f16(128, 32, 0, 1);                  // [0; M] U
             for (int c = 0; c < nchunks && !*abort_flag; ++c) {
-                const int s = c & 1;
+                const int s = c % NSTAGE, d = c & 1;
                 const uint32_t astg = sbase + s * STAGE;
-                const uint32_t d5 = tmem + TM_D5 + 32 * s;
-                if (!mbar_wait(&bars[B_FULL + s], (c >> 1) & 1)) { fail(); break; }
+                const uint32_t d5 = tmem + TM_D5 + 32 * d;
+                if (!mbar_wait(&bars[B_FULL + s], (c / NSTAGE) & 1)) { fail(); break; }
                 ++n_issued;
-                if (c >= 2 && !mbar_wait(&bars[B_D5FREE + s], ((c >> 1) - 1) & 1)) { fail(); break; }
+                if (c >= 2 && !mbar_wait(&bars[B_D5FREE + d], ((c >> 1) - 1) & 1)) { fail(); break; }
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
@@ -166,7 +159,7 @@ chunk_scan_kernel(ScanParams p)
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t kh = ks >> 2, ko = (ks & 3) * 32;
-                    umma_ss(d5, smem_desc(astg + ST_WQ + kh * 16384 + ko, 16, 1024, SW_128B),
+                    umma_ss(d5, smem_desc(astg + ST_X + kh * 16384 + ko, 16, 1024, SW_128B),
                             smem_desc(sbase + OFF_SB + ks * 1024, 16, 512, SW_64B), id_s1, 1);
                 }
                 umma_commit(&bars[B_S1]);
@@ -177,12 +170,7 @@ chunk_scan_kernel(ScanParams p)
                     umma_ss(tmem + TM_D7, smem_desc(astg + ST_KE + ks * 2048, 8192, 1024, SW_128B),
                             smem_desc(sbase + OFF_UB + ks * 1024, 16, 512, SW_64B), id_s2, ks > 0);
                 umma_commit(&bars[B_S2]);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    umma_ss(d5, smem_desc(astg + ST_Y + 8192 + ks * 32, 16, 1024, SW_128B),
-                            smem_desc(sbase + OFF_UB + ks * 1024, 16, 512, SW_64B), id_mu, 1);
-                umma_commit(&bars[B_MU + s]);
-                umma_commit(&bars[B_EMPTY + s]);      // its MMA share of releasing stage s
+                umma_commit(&bars[B_EMPTY + s]);      // every MMA reading stage s is complete
             }
             if (n_issued) {                           // every MMA complete before TMEM is freed
                 umma_commit(&bars[B_DRAIN]);
@@ -191,50 +179,54 @@ chunk_scan_kernel(ScanParams p)
         }
     } else if (warp == 4) {
         // ============================================================================ loader
-        uint32_t issued[2] = {0u, 0u};
-        for (int c = 0; c < nchunks; ++c) {
-            const int s = c & 1;
-            unsigned char *stg = sm + s * STAGE;
-            if (warp_abort()) break;
-            int ok = 1;
-            if (c >= 2 && lane == 0) ok = mbar_wait(&bars[B_EMPTY + s], ((c >> 1) - 1) & 1);
-            if (!__shfl_sync(0xffffffffu, ok, 0)) { if (lane == 0) fail(); break; }
-            if (lane == 0) {
-                const unsigned char *blk = p.ws + ((size_t)h * p.n_slots + (first_slot + c)) * kPrepBlockBytes;
-                mbar_arrive_expect_tx(&bars[B_FULL + s], BLOCK_TX);
-                bulk_g2s(stg + ST_WQ, blk + kPrepWQOff, 32768, &bars[B_FULL + s]);
-                bulk_g2s(stg + ST_Y, blk + kPrepTbOff, 8192, &bars[B_FULL + s]);
-                bulk_g2s(stg + ST_Y + 16384, blk + kPrepMOff, 8192, &bars[B_FULL + s]);
-                bulk_g2s(stg + ST_KE, blk + kPrepKEOff, 16384, &bars[B_FULL + s]);
-                bulk_g2s(stg + ST_G, blk + kPrepGammaOff, 512, &bars[B_FULL + s]);
-            }
-            ++issued[s];
-            // v block (bf16 -> f16): lane -> rows 2 lane, 2 lane + 1
+        // v block of chunk c in registers: lane -> rows 2 lane, 2 lane + 1 (32 columns each)
+        uint4 vr[2][4];
+        auto load_v = [&](int c) {
             const int64_t tok0 = t0 + (int64_t)c * C;
             const int L = (t1 - tok0 < C) ? (int)(t1 - tok0) : C;
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) {
                 const int r = 2 * lane + rr;
-                uint4 raw[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
-                    raw[u] = (r < L) ? ldg_nc(p.v + ((size_t)(tok0 + r) * H + h) * DK + j0 + 8 * u)
-                                     : make_uint4(0, 0, 0, 0);
+                    vr[rr][u] = (r < L) ? ldg_nc(p.v + ((size_t)(tok0 + r) * H + h) * DK + j0 + 8 * u)
+                                        : make_uint4(0, 0, 0, 0);
+            }
+        };
+        if (nchunks > 0) load_v(0);
+        int n_loaded = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % NSTAGE;
+            unsigned char *stg = sm + s * STAGE;
+            if (warp_abort()) break;
+            int ok = 1;
+            if (c >= NSTAGE && lane == 0) ok = mbar_wait(&bars[B_EMPTY + s], ((c / NSTAGE) - 1) & 1);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) { if (lane == 0) fail(); break; }
+            if (lane == 0) {
+                const unsigned char *blk = p.ws + ((size_t)h * p.n_slots + (first_slot + c)) * kPrepBlockBytes;
+                mbar_arrive_expect_tx(&bars[B_FULL + s], (uint32_t)kPrepBlockBytes);
+                bulk_g2s(stg, blk, (uint32_t)kPrepBlockBytes, &bars[B_FULL + s]);
+            }
+            n_loaded = c + 1;
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const int r = 2 * lane + rr;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     uint4 o;
-                    o.x = bf16x2_to_f16x2(raw[u].x); o.y = bf16x2_to_f16x2(raw[u].y);
-                    o.z = bf16x2_to_f16x2(raw[u].z); o.w = bf16x2_to_f16x2(raw[u].w);
+                    o.x = bf16x2_to_f16x2(vr[rr][u].x); o.y = bf16x2_to_f16x2(vr[rr][u].y);
+                    o.z = bf16x2_to_f16x2(vr[rr][u].z); o.w = bf16x2_to_f16x2(vr[rr][u].w);
                     *reinterpret_cast<uint4 *>(stg + ST_V + sw64_offset(r, 8 * u)) = o;
                 }
             }
+            if (c + 1 < nchunks) load_v(c + 1);      // lands while the loader waits for a free stage
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_FULL + s]);
         }
         if (lane == 0)       // no copy may still be landing when the CTA exits
-            for (int s = 0; s < 2; ++s)
-                if (issued[s]) mbar_wait(&bars[B_FULL + s], (issued[s] - 1) & 1, 100000000LL);
+            for (int c = (n_loaded > NSTAGE ? n_loaded - NSTAGE : 0); c < n_loaded; ++c)
+                mbar_wait(&bars[B_FULL + c % NSTAGE], (c / NSTAGE) & 1, 100000000LL);
     } else {
         // ========================================================================= epilogues
         const int st = tid;                   // key channel / TMEM lane
@@ -260,67 +252,61 @@ chunk_scan_kernel(ScanParams p)
         fence_proxy_async_smem();
         mbar_arrive(&bars[B_SREADY]);
         for (int c = 0; c < nchunks; ++c) {
-            const int s = c & 1;
+            const int s = c % NSTAGE, d = c & 1;
             const int64_t tok0 = t0 + (int64_t)c * C;
             const int L = (t1 - tok0 < C) ? (int)(t1 - tok0) : C;
-            const uint32_t d5 = tmem + TM_D5 + 32 * s;
+            const uint32_t d5 = tmem + TM_D5 + 32 * d;
             if (warp_abort()) break;
             // gamma of this chunk (read from the stage after observing its arrival directly)
-            if (!warp_wait(&bars[B_FULL + s], (c >> 1) & 1)) { fail(); break; }
+            if (!warp_wait(&bars[B_FULL + s], (c / NSTAGE) & 1)) { fail(); break; }
             const float g = reinterpret_cast<const float *>(sm + s * STAGE + ST_G)[st];
+            if (!warp_wait(&bars[B_S1], c & 1)) { fail(); break; }
+            tc_fence_after();
+            float x[32];
+            tmem_ld32_sync(d5 + ((uint32_t)(32 * warp) << 16), x);
             if (warp < 2) {                   // U = -(D5 rows 0-63) -> f16, MN-major [token][32]
-                if (!warp_wait(&bars[B_S1], c & 1)) { fail(); break; }
-                tc_fence_after();
-                float u[32];
-                tmem_ld32_sync(d5 + ((uint32_t)(32 * warp) << 16), u);
 #pragma unroll
                 for (int j = 0; j < DVB; j += 8) {
                     uint4 o;
-                    o.x = pack_f16x2(-u[j], -u[j + 1]); o.y = pack_f16x2(-u[j + 2], -u[j + 3]);
-                    o.z = pack_f16x2(-u[j + 4], -u[j + 5]); o.w = pack_f16x2(-u[j + 6], -u[j + 7]);
+                    o.x = pack_f16x2(-x[j], -x[j + 1]); o.y = pack_f16x2(-x[j + 2], -x[j + 3]);
+                    o.z = pack_f16x2(-x[j + 4], -x[j + 5]); o.w = pack_f16x2(-x[j + 6], -x[j + 7]);
                     *reinterpret_cast<uint4 *>(sm + OFF_UB + sw64_offset(st, j)) = o;
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
                 mbar_arrive(&bars[B_UREADY]);
+                mbar_arrive(&bars[B_D5FREE + d]);
+            } else {                          // O = D5 rows 64-127, stored after the state update
+                tc_fence_before();
+                mbar_arrive(&bars[B_D5FREE + d]);
             }
             // S <- gamma S + Kend^T U, then hand the new state to the next chunk's S1
             if (!warp_wait(&bars[B_S2], c & 1)) { fail(); break; }
             tc_fence_after();
-            {
-                float d7[32];
-                tmem_ld32_sync(tmem + TM_D7 + ((uint32_t)(32 * warp) << 16), d7);
+            float d7[32];
+            tmem_ld32_sync(tmem + TM_D7 + ((uint32_t)(32 * warp) << 16), d7);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) S[e] = g * S[e] + d7[e];
-                store_state();
-                fence_proxy_async_smem();
-                tc_fence_before();
-                mbar_arrive(&bars[B_SREADY]);
-                mbar_arrive(&bars[B_EMPTY + s]);      // gamma of stage s has been read
-            }
-            if (warp >= 2) {                  // O = D5 rows 64-127 -> out
-                if (!warp_wait(&bars[B_MU + s], (c >> 1) & 1)) { fail(); break; }
-                tc_fence_after();
-                const int r = st - 64;
-                float o32[32];
-                tmem_ld32_sync(d5 + ((uint32_t)(32 * warp) << 16), o32);
-                tc_fence_before();
-                mbar_arrive(&bars[B_D5FREE + s]);
-                if (r < L) {
-                    TO *dst = reinterpret_cast<TO *>(p.out) + ((size_t)(tok0 + r) * H + h) * DK + j0;
-                    if constexpr (sizeof(TO) == 4) {
+            for (int e = 0; e < 32; ++e) S[e] = g * S[e] + d7[e];
+            store_state();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars[B_SREADY]);
+            mbar_arrive(&bars[B_EMPTY + s]);          // gamma of stage s has been read
+            // outputs of this chunk (kept off the chain: global stores here overlap the next S1)
+            if (warp >= 2 && st - 64 < L) {
+                TO *dst = reinterpret_cast<TO *>(p.out) + ((size_t)(tok0 + st - 64) * H + h) * DK + j0;
+                if constexpr (sizeof(TO) == 4) {
 #pragma unroll
-                        for (int j = 0; j < DVB; j += 4)
-                            *reinterpret_cast<float4 *>(reinterpret_cast<float *>(dst) + j) =
-                                make_float4(o32[j], o32[j + 1], o32[j + 2], o32[j + 3]);
-                    } else {
+                    for (int j = 0; j < DVB; j += 4)
+                        *reinterpret_cast<float4 *>(reinterpret_cast<float *>(dst) + j) =
+                            make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+                } else {
 #pragma unroll
-                        for (int j = 0; j < DVB; j += 8) {
-                            uint4 o;
-                            o.x = pack_bf16x2(o32[j], o32[j + 1]); o.y = pack_bf16x2(o32[j + 2], o32[j + 3]);
-                            o.z = pack_bf16x2(o32[j + 4], o32[j + 5]); o.w = pack_bf16x2(o32[j + 6], o32[j + 7]);
-                            *reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(dst) + j) = o;
-                        }
+                    for (int j = 0; j < DVB; j += 8) {
+                        uint4 o;
+                        o.x = pack_bf16x2(x[j], x[j + 1]); o.y = pack_bf16x2(x[j + 2], x[j + 3]);
+                        o.z = pack_bf16x2(x[j + 4], x[j + 5]); o.w = pack_bf16x2(x[j + 6], x[j + 7]);
+                        *reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(dst) + j) = o;
                     }
                 }
             }

@@ -14,10 +14,10 @@ constexpr int kChunk = 64;      // chunk length of the prefill (tokens)
 constexpr size_t kStatusBytes = 256;  // workspace prefix holding the device status word
 
 // Two-pass bf16 prefill: per (chunk slot, head) block of prepared operands in the workspace,
-// laid out as the scan pass wants them in shared memory (see chunk_prep.cu).
-constexpr uint32_t kPrepWQOff = 0;          // W / Qt, 32 KiB
-constexpr uint32_t kPrepTbOff = 32768;      // Tb, 8 KiB
-constexpr uint32_t kPrepMOff = 40960;       // M, 8 KiB
+// laid out as the scan pass wants them in shared memory (see chunk_prep.cu). The first 66048 bytes
+// are contiguous in the same order in the scan's ring stage, so one bulk copy moves a block.
+constexpr uint32_t kPrepXOff = 0;           // X = [W; Qt - M W], 128 x 128 f16, 32 KiB
+constexpr uint32_t kPrepYOff = 32768;       // Y = [-Tb; M Tb], 128 x 64 f16, 16 KiB
 constexpr uint32_t kPrepKEOff = 49152;      // Kend, 16 KiB
 constexpr uint32_t kPrepGammaOff = 65536;   // gamma, 512 B
 constexpr size_t kPrepBlockBytes = 66048;
