@@ -7,7 +7,7 @@ A step is one ``kda_chunk_fwd`` over the 128K-token, 32-head bf16 workload (B=1,
 H=32, d_k=d_v=128, chunk 64, fp32 state, S0 ~ N(0, 0.1^2)); the decode step (256 sequences x 32
 heads, 512 MiB fp32 state, 1000 consecutive steps) is measured in the same run and reported
 under ``decode``. Inputs are synthetic (``kda_inputs``), resident in HBM before timing; one step
-reads 6.5 GB, far more than the 126 MB L2, so no flush is needed between steps.
+reads 5.4 GB of inputs, far more than the 126 MB L2, so no flush is needed between steps.
 
 With N > 1 (torchrun, one process per GPU) every rank runs its own copy of the workload: the
 heads and sequences are independent, so there is no collective on the data path (weak scaling);
@@ -37,9 +37,11 @@ WORKLOAD = "bf16_t128k_h32"
 DECODE = "decode_n256_h32"
 C = 64
 D = 128
-# algorithmic HBM bytes per token*head of the prefill: q, k, v bf16 (3 x 256 B), out fp32
-# (512 B), log_alpha fp32 (512 B), beta fp32 (4 B)
-PREFILL_BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 4 + D * 4 + 4
+# algorithmic HBM bytes per token*head of the prefill: q, k, v bf16 (3 x 256 B), out bf16
+# (256 B; the output takes the inputs' dtype), log_alpha fp32 (512 B), beta fp32 (4 B)
+PREFILL_BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 2 + D * 4 + 4
+# kernels one prefill step launches: the chunk-preparation pass and the state scan
+PREFILL_KERNELS_PER_STEP = 2
 # useful tensor flops per token*head (chunk C): 6 d^2 (W.S, Q.S, Kend^T.U) + 5 C d (triangular
 # K K^T, Q K^T, T.(beta K), T.(beta V), M.U) + C^2 / 3 (triangular inverse)
 PREFILL_FLOPS_PER_TOKEN_HEAD = 6 * D * D + 5 * C * D + C * C // 3
@@ -220,7 +222,7 @@ def run_native(args):
     from kimi_delta_attention_25_b200 import shard
     d = K.make_prefill(w, device=dev, seed=shard.rank_seed(w.seed, rank))
     B, T, H = w.B, w.T, w.H
-    out = torch.empty(B, T, H, D, dtype=torch.float32, device=dev)
+    out = torch.empty(B, T, H, D, dtype=torch.bfloat16, device=dev)
     Sf = torch.empty(B, H, D, D, dtype=torch.float32, device=dev)
     wsz = kda.chunk_fwd_workspace_size(B, T, H, B)
     work = torch.empty(max(256, wsz), dtype=torch.uint8, device=dev)
@@ -278,8 +280,8 @@ def run_native(args):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": WORKLOAD, "global_batch": ws * B, "seq_len": T, "heads": H,
-                       "head_dim": D, "chunk": C, "state": "fp32", "gates": "fp32", "out": "fp32",
-                       "l2": "inputs larger than L2 (6.5 GB per step), no flush",
+                       "head_dim": D, "chunk": C, "state": "fp32", "gates": "fp32", "out": "bf16",
+                       "l2": "inputs larger than L2 (5.4 GB read per step), no flush",
                        "parallelism": "dp%d (independent heads/sequences per GPU)" % ws},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
                          "frac": gbs / pk["hbm"], "traffic": None,
@@ -289,7 +291,7 @@ def run_native(args):
                          "tensor_tflops_useful": tfs, "tensor_frac_useful": tfs / pk["bf16"]},
             "e2e": {"value": e2e_val, "unit": "Mtok/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
-            "gpu_launches": args.steps * 1,
+            "gpu_launches": args.steps * PREFILL_KERNELS_PER_STEP,
             "clocks": clk.summary(),
             "decode": dec,
             "cpu_baseline": cpu,

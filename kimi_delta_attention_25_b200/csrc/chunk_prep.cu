@@ -83,6 +83,43 @@ struct PrepParams {
     int32_t *status;
 };
 
+// The (sequence, chunk) of a chunk slot: slot = floor(first_token / 64) + sequence. Returns false
+// for an unused slot (or for cu_seqlens that the scan pass reports as invalid).
+__device__ __forceinline__ bool slot_chunk(const PrepParams &p, int slot, int64_t *tok0, int *L)
+{
+    int n = 0;
+    int64_t s0, s1;
+    if (p.cu_seqlens) {
+        int lo = 0, hi = p.N - 1;                 // largest n with floor(cu[n]/64) + n <= slot
+        if (hi < 0) return false;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.cu_seqlens[mid] / C + mid <= slot) lo = mid; else hi = mid - 1;
+        }
+        n = lo;
+        s0 = p.cu_seqlens[n];
+        s1 = p.cu_seqlens[n + 1];
+        if (s1 < s0 || s0 < 0 || s1 > p.T) return false;
+    } else {
+        // sequence n = batch row; its first slot is (n * T) / 64 + n
+        int lo = 0, hi = p.N - 1;
+        if (hi < 0) return false;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if ((int)(((int64_t)mid * p.T) / C) + mid <= slot) lo = mid; else hi = mid - 1;
+        }
+        n = lo;
+        s0 = (int64_t)n * p.T;
+        s1 = s0 + p.T;
+    }
+    const int64_t c = slot - (s0 / C + n);
+    *tok0 = s0 + c * C;
+    if (c < 0 || *tok0 >= s1) return false;
+    *L = (s1 - *tok0 < C) ? (int)(s1 - *tok0) : C;
+    return true;
+}
+
+
 // Unit lower-triangular inverse (see chunk_tc.cu): A column-major in AT, T row-major stride LDT.
 __device__ __forceinline__ void inverse64(int pt, const float *AT, float *Tf, float *Ps)
 {
@@ -176,37 +213,9 @@ chunk_prep_kernel(PrepParams p)
     const int slot = blockIdx.x, h = blockIdx.y;
     const int H = p.H;
 
-    // ---- which (sequence, chunk) this slot is: slot = floor(first_token / 64) + sequence
-    int n = 0;
-    int64_t s0, s1;
-    if (p.cu_seqlens) {
-        int lo = 0, hi = p.N - 1;                 // largest n with floor(cu[n]/64) + n <= slot
-        if (hi < 0) return;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (p.cu_seqlens[mid] / C + mid <= slot) lo = mid; else hi = mid - 1;
-        }
-        n = lo;
-        s0 = p.cu_seqlens[n];
-        s1 = p.cu_seqlens[n + 1];
-        if (s1 < s0 || s0 < 0 || s1 > p.T) return;    // reported by the scan pass
-    } else {
-        // sequence n = batch row; its first slot is (n * T) / 64 + n
-        int lo = 0, hi = p.N - 1;
-        if (hi < 0) return;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if ((int)(((int64_t)mid * p.T) / C) + mid <= slot) lo = mid; else hi = mid - 1;
-        }
-        n = lo;
-        s0 = (int64_t)n * p.T;
-        s1 = s0 + p.T;
-    }
-    const int64_t first_slot = s0 / C + n;
-    const int64_t c = slot - first_slot;
-    const int64_t tok0 = s0 + c * C;
-    if (c < 0 || tok0 >= s1) return;              // unused slot
-    const int L = (s1 - tok0 < C) ? (int)(s1 - tok0) : C;
+    int64_t tok0;
+    int L;
+    if (!slot_chunk(p, slot, &tok0, &L)) return;  // unused slot
     unsigned char *blk = p.ws + ((size_t)h * p.n_slots + slot) * kPrepBlockBytes;
 
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
@@ -487,6 +496,7 @@ cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slo
     p.q = (const __nv_bfloat16 *)a.q; p.k = (const __nv_bfloat16 *)a.k;
     p.log_alpha = a.log_alpha; p.beta = a.beta; p.cu_seqlens = a.cu_seqlens;
     p.ws = ws; p.T = a.T; p.H = a.H; p.N = a.N; p.n_slots = n_slots; p.status = a.status;
+
     cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
