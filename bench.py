@@ -42,6 +42,14 @@ D = 128
 PREFILL_BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 2 + D * 4 + 4
 # kernels one prefill step launches: the chunk-preparation pass and the state scan
 PREFILL_KERNELS_PER_STEP = 2
+# the same algorithmic bytes, split by the pass that moves them: the preparation pass reads q, k,
+# log_alpha and beta; the scan reads v and writes out (its other traffic is the workspace)
+PREP_BYTES_PER_TOKEN_HEAD = 2 * D * 2 + D * 4 + 4
+SCAN_BYTES_PER_TOKEN_HEAD = D * 2 + D * 2
+# DRAM traffic per token*head measured by Nsight Compute (profiles/dram_traffic.json), valid for
+# the kernel source it was taken from
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
+CSRC = os.path.join(ROOT, "kimi_delta_attention_25_b200", "csrc")
 # useful tensor flops per token*head (chunk C): 6 d^2 (W.S, Q.S, Kend^T.U) + 5 C d (triangular
 # K K^T, Q K^T, T.(beta K), T.(beta V), M.U) + C^2 / 3 (triangular inverse)
 PREFILL_FLOPS_PER_TOKEN_HEAD = 6 * D * D + 5 * C * D + C * C // 3
@@ -137,6 +145,20 @@ def max_over_ranks(x, ws):
     return shard.max_over_ranks(x, device="cuda") if ws > 1 else x
 
 
+def measured_traffic(kernel, unit="dram_bytes_per_token_head"):
+    """DRAM bytes per unit of `kernel` from the committed ncu summary, or None when the kernel's
+    source has changed since the counters were taken."""
+    import hashlib
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)[kernel]
+        with open(os.path.join(CSRC, t["source"]), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except (OSError, KeyError, ValueError):
+        return None
+    return float(t[unit]) if sha == t["source_sha256"] else None
+
+
 def time_loop(fn, steps, warmup, ws):
     """CUDA-event time of `steps` calls of fn on the current stream, after `warmup` calls."""
     for _ in range(warmup):
@@ -164,7 +186,7 @@ def cpu_oracle_sample(budget_s=12.0):
     from oracle import ref
     cores = ref.online_cores()
     w = K.WORKLOADS[WORKLOAD]
-    Hs = max(1, min(w.H, cores))
+    Hs = w.H
     cal_T = 1024
     d = K.make_prefill(w, T=cal_T, H=1)
     args = [d[x].float().numpy() for x in ("q", "k", "v", "log_alpha", "beta")]
@@ -172,10 +194,11 @@ def cpu_oracle_sample(budget_s=12.0):
     ref.forward(*args, S0=d["S0"].double().numpy(), nthreads=1)
     per_tok_head = (time.perf_counter() - t0) / cal_T
     Ts = int(max(1024, min(w.T, budget_s / per_tok_head * min(Hs, cores) / Hs)))
+    Ts -= Ts % C
     d = K.make_prefill(w, T=Ts, H=Hs)
     args = [d[x].float().numpy() for x in ("q", "k", "v", "log_alpha", "beta")]
     t0 = time.perf_counter()
-    ref.forward(*args, S0=d["S0"].double().numpy(), nthreads=Hs)
+    ref.forward(*args, S0=d["S0"].double().numpy(), nthreads=min(Hs, cores))
     dt = time.perf_counter() - t0
     tok_equiv = Ts * Hs / w.H                 # tokens of the full 32-head workload
     return {"value": tok_equiv / dt / 1e6, "unit": "Mtok/s", "cores": min(Hs, cores),
@@ -234,9 +257,38 @@ def run_native(args):
     step()
     torch.cuda.synchronize()
     assert kda.workspace_status(work) == kda.KDA_OK
+
+    # One timed step = the two passes through their own entry points (exactly what chunk_fwd
+    # runs), with CUDA events on the launching stream around each pass.
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+
+    def step_passes(ev=None):
+        if ev is not None:
+            ev[0].record()
+        kda.chunk_prep(d["q"], d["k"], d["log_alpha"], d["beta"], work)
+        if ev is not None:
+            ev[1].record()
+        kda.chunk_scan(d["v"], work, S0=d["S0"], out=out, S_final=Sf)
+        if ev is not None:
+            ev[2].record()
+
     with Clocks(local) as clk:
-        ms = time_loop(step, args.steps, args.warmup, ws)
-    ms = max_over_ranks(ms, ws)
+        for _ in range(args.warmup):
+            step_passes()
+        torch.cuda.synchronize()
+        barrier(ws)
+        torch.cuda.synchronize()
+        t_s, t_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t_s.record()
+        for i in range(args.steps):
+            step_passes(evs[i])
+        t_e.record()
+        torch.cuda.synchronize()
+        barrier(ws)
+    assert kda.workspace_status(work) == kda.KDA_OK
+    ms = max_over_ranks(t_s.elapsed_time(t_e) / args.steps, ws)
+    ms_prep = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    ms_scan = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     tokens = B * T
     value = ws * tokens / (ms * 1e-3) / 1e6                   # Mtok/s, whole job
     th = B * T * H
@@ -244,6 +296,15 @@ def run_native(args):
     flops = th * PREFILL_FLOPS_PER_TOKEN_HEAD
     gbs = alg_bytes / (ms * 1e-3) / 1e9
     tfs = flops / (ms * 1e-3) / 1e12
+    kern = {}
+    for name, t_ms, per in (("chunk_prep", ms_prep, PREP_BYTES_PER_TOKEN_HEAD),
+                            ("chunk_scan", ms_scan, SCAN_BYTES_PER_TOKEN_HEAD)):
+        tr = measured_traffic(name)
+        a = th * per / (t_ms * 1e-3) / 1e9
+        kern[name] = {"ms": t_ms, "achieved": a, "frac": a / pk["hbm"],
+                      "algorithmic_bytes_per_launch": th * per,
+                      "traffic": None if tr is None else tr * th}
+    dom = max(kern, key=lambda k: kern[k]["ms"])
 
     # ---- end to end through the public call with pinned host buffers
     host = {x: d[x].cpu().pin_memory() for x in ("q", "k", "v", "log_alpha", "beta", "S0")}
@@ -283,12 +344,15 @@ def run_native(args):
                        "head_dim": D, "chunk": C, "state": "fp32", "gates": "fp32", "out": "bf16",
                        "l2": "inputs larger than L2 (5.4 GB read per step), no flush",
                        "parallelism": "dp%d (independent heads/sequences per GPU)" % ws},
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm"], "traffic": None,
-                         "peak_source": "of %s" % pk["src"],
-                         "kernel": "kda chunk prefill",
-                         "algorithmic_bytes_per_launch": alg_bytes,
-                         "tensor_tflops_useful": tfs, "tensor_frac_useful": tfs / pk["bf16"]},
+            "roofline": {"bound": "hbm", "achieved": kern[dom]["achieved"], "peak": pk["hbm"],
+                         "unit": "GB/s", "frac": kern[dom]["frac"], "traffic": kern[dom]["traffic"],
+                         "peak_source": "of %s" % pk["src"], "kernel": dom,
+                         "ms_per_launch": kern[dom]["ms"],
+                         "algorithmic_bytes_per_launch": kern[dom]["algorithmic_bytes_per_launch"],
+                         "kernels": kern,
+                         "step": {"achieved": gbs, "frac": gbs / pk["hbm"],
+                                  "algorithmic_bytes": alg_bytes,
+                                  "tensor_tflops_useful": tfs, "tensor_frac_useful": tfs / pk["bf16"]}},
             "e2e": {"value": e2e_val, "unit": "Mtok/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
             "gpu_launches": args.steps * PREFILL_KERNELS_PER_STEP,
@@ -318,15 +382,37 @@ def run_decode(kda, dev, pk, ws, local, args):
     with Clocks(local) as clk:
         ms = time_loop(one, nsteps, 5, ws)
     ms = max_over_ranks(ms, ws)
+
+    # the same 1000 launches captured once in a CUDA graph and replayed (launch overhead removed)
+    g = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream()
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cs):
+        with torch.cuda.graph(g, stream=cs):
+            for x in xs:
+                kda.decode_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S, out=out)
+    torch.cuda.current_stream().wait_stream(cs)
+    g.replay()
+    torch.cuda.synchronize()
+    gs, ge = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gs.record()
+    g.replay()
+    ge.record()
+    torch.cuda.synchronize()
+    ms_graph = max_over_ranks(gs.elapsed_time(ge) / nsteps, ws)
+    del g
     heads = N * H
     state_b = heads * DECODE_STATE_BYTES_PER_HEAD
     io_b = heads * DECODE_IO_BYTES_PER_HEAD
     us = ms * 1e3
     gbs = state_b / (ms * 1e-3) / 1e9
     return {"workload": DECODE, "us_per_step": us, "steps": nsteps,
+            "graph_us_per_step": ms_graph * 1e3,
             "state_gbs": gbs, "total_gbs": (state_b + io_b) / (ms * 1e-3) / 1e9,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm"], "traffic": None, "peak_source": "of %s" % pk["src"]},
+                         "frac": gbs / pk["hbm"], "peak_source": "of %s" % pk["src"],
+                         "traffic": (lambda t: None if t is None else t * heads)(
+                             measured_traffic("decode", "dram_bytes_per_head"))},
             "tokens_per_s_whole_job": ws * N / (ms * 1e-3),
             "gpu_launches": nsteps, "clocks": clk.summary()}
 
@@ -342,7 +428,8 @@ def run_profile_case(args):
         w = K.WORKLOADS[WORKLOAD]
         d = K.make_prefill(w, device=dev, T=args.tokens)
         for _ in range(2):
-            kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"])
+            kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"],
+                          out_dtype=torch.bfloat16)
         torch.cuda.synchronize()
         assert kda.workspace_status(kda.chunk_fwd.last_workspace) == kda.KDA_OK
     else:

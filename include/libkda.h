@@ -101,6 +101,34 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v,
                            kda_dtype_t dtype, kda_dtype_t out_dtype,
                            void *workspace, size_t workspace_bytes, void *stream);
 
+/* The two passes kda_chunk_fwd runs for bf16 inputs, callable one by one (the same
+ * chunked form as kda_chunk_fwd; the split is this library's, the pages name no passes).
+ * kda_chunk_prep does every step that does not depend on the running state, for all
+ * chunks at once (decay scaling, the intra-chunk products, the triangular inverse, the
+ * WY factors) and writes the results to the workspace; kda_chunk_scan then runs the
+ * state recurrence over the chunks and writes out and S_final. Together they compute
+ * exactly what one kda_chunk_fwd call does. A caller can run the passes of different
+ * batches on different streams, or time them separately.
+ *
+ *   Arguments mean what they mean for kda_chunk_fwd with dtype = KDA_BF16; the
+ *   workspace is sized by kda_chunk_fwd_workspace_size(..., KDA_BF16).
+ *   kda_chunk_prep reads q, k, log_alpha, beta (and cu_seqlens) and clears the
+ *   workspace status word before it enqueues its kernel.
+ *   kda_chunk_scan reads v, S0 and the prepared workspace, writes out and S_final, and
+ *   leaves the status word as it is, so that it reports errors of both passes.
+ * kda_chunk_scan must follow a kda_chunk_prep with the same B, T, H, N, cu_seqlens and
+ * workspace, ordered after it (same stream, or an event); it reads whatever the
+ * workspace holds, so a scan without its prep returns garbage, not an error. */
+kda_status_t kda_chunk_prep(const void *q, const void *k,
+                            const float *log_alpha, const float *beta,
+                            const int32_t *cu_seqlens,
+                            int B, int T, int H, int N, int dk, int dv,
+                            void *workspace, size_t workspace_bytes, void *stream);
+kda_status_t kda_chunk_scan(const void *v, const float *S0, const int32_t *cu_seqlens,
+                            void *out, float *S_final,
+                            int B, int T, int H, int N, int dk, int dv, kda_dtype_t out_dtype,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
 /* One decode step for N independent sequences (one token each), updating the
  * state in place: the recurrent ("fused_recurrent") mode the layer uses for
  * short queries and generation (lpnh.cn article, sec. 2 and 5); the per-step

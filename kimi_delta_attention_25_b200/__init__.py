@@ -9,6 +9,8 @@ Names follow the C entry points:
 
 * ``chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None)`` -> ``(out, S_final)``
 * ``decode_step(q, k, v, log_alpha, beta, S)`` -> ``out`` (``S`` updated in place)
+* ``chunk_prep(q, k, log_alpha, beta, workspace, ...)`` and ``chunk_scan(v, workspace, ...)``:
+  the two passes of ``chunk_fwd`` for bf16 inputs, one call each
 * ``chunk_fwd_workspace_size``, ``workspace_status``, ``status_string``
 """
 from __future__ import annotations
@@ -19,7 +21,7 @@ from typing import Optional
 
 import torch
 
-__all__ = ["chunk_fwd", "decode_step", "chunk_fwd_workspace_size", "workspace_status",
+__all__ = ["chunk_fwd", "chunk_prep", "chunk_scan", "decode_step", "chunk_fwd_workspace_size", "workspace_status",
            "status_string", "library_path", "load", "KDAError",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA", "KDA_ERR_TIMEOUT"]
 
@@ -32,7 +34,8 @@ _lib = None
 
 # Every entry point declared in include/libkda.h.
 EXPORTS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
-           "kda_workspace_status", "kda_status_string", "kda_version", "kda_chunk_fwd_noalloc")
+           "kda_workspace_status", "kda_status_string", "kda_version", "kda_chunk_fwd_noalloc",
+           "kda_chunk_prep", "kda_chunk_scan")
 
 
 class KDAError(RuntimeError):
@@ -64,6 +67,10 @@ def load():
     lib.kda_version.restype = I
     lib.kda_chunk_fwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P]
     lib.kda_chunk_fwd_noalloc.restype = I
+    lib.kda_chunk_prep.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, Z, P]
+    lib.kda_chunk_prep.restype = I
+    lib.kda_chunk_scan.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, Z, P]
+    lib.kda_chunk_scan.restype = I
     _lib = lib
     return lib
 
@@ -128,6 +135,44 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, S_fi
     if st != KDA_OK:
         raise KDAError(st, "kda_chunk_fwd")
     chunk_fwd.last_workspace = workspace
+    return out, S_final
+
+
+def chunk_prep(q, k, log_alpha, beta, workspace, cu_seqlens=None):
+    """``kda_chunk_prep``: first pass of the bf16 prefill (everything that does not depend on the
+    state), written into ``workspace`` (uint8, ``chunk_fwd_workspace_size(...)`` bytes)."""
+    lib = load()
+    B, T, H, dk = q.shape
+    N = B if cu_seqlens is None else cu_seqlens.shape[0] - 1
+    _need_cuda(q, k, log_alpha, beta, cu_seqlens, workspace)
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16:
+        raise TypeError("chunk_prep takes bfloat16 q and k")
+    st = lib.kda_chunk_prep(_ptr(q), _ptr(k), _ptr(log_alpha), _ptr(beta), _ptr(cu_seqlens),
+                            B, T, H, N, dk, dk, _ptr(workspace), workspace.numel(), _stream(q.device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_prep")
+    return workspace
+
+
+def chunk_scan(v, workspace, S0=None, cu_seqlens=None, out=None, S_final=None, want_state=True,
+               out_dtype=torch.float32):
+    """``kda_chunk_scan``: second pass of the bf16 prefill, after ``chunk_prep`` on the same
+    workspace and sizes. Returns (out, S_final) like ``chunk_fwd``."""
+    lib = load()
+    B, T, H, dv = v.shape
+    N = B if cu_seqlens is None else cu_seqlens.shape[0] - 1
+    if out is None:
+        out = torch.empty(B, T, H, dv, dtype=out_dtype, device=v.device)
+    if S_final is None and want_state:
+        S_final = torch.empty(N, H, dv, dv, dtype=torch.float32, device=v.device)
+    _need_cuda(v, S0, cu_seqlens, out, S_final, workspace)
+    if v.dtype != torch.bfloat16:
+        raise TypeError("chunk_scan takes bfloat16 v")
+    st = lib.kda_chunk_scan(_ptr(v), _ptr(S0), _ptr(cu_seqlens), _ptr(out), _ptr(S_final),
+                            B, T, H, N, dv, dv, _dtype_code(out), _ptr(workspace), workspace.numel(),
+                            _stream(v.device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_scan")
     return out, S_final
 
 

@@ -42,13 +42,17 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int N, int dk, int dv, 
     return kStatusBytes + (size_t)H * (size_t)prep_slots((long long)B * T, N) * kPrepBlockBytes;
 }
 
-kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v,
-                           const float *log_alpha, const float *beta,
-                           const float *S0, const int32_t *cu_seqlens,
-                           void *out, float *S_final,
-                           int B, int T, int H, int N, int dk, int dv,
-                           kda_dtype_t dtype, kda_dtype_t out_dtype,
-                           void *workspace, size_t workspace_bytes, void *stream)
+}  // extern "C"
+
+namespace {
+
+// Host-side checks shared by the prefill entry points. `need_*` selects which tensors the caller
+// passes (the two passes of the bf16 path each take a subset).
+kda_status_t check_prefill(const void *q, const void *k, const void *v, const float *log_alpha,
+                           const float *beta, const float *S0, const int32_t *cu_seqlens, const void *out,
+                           const float *S_final, int B, int T, int H, int N, int dk, int dv,
+                           kda_dtype_t dtype, kda_dtype_t out_dtype, const void *workspace,
+                           size_t workspace_bytes, bool need_qk, bool need_vout)
 {
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (out_dtype != KDA_F32 && out_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
@@ -61,22 +65,23 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v,
         return KDA_ERR_INVALID_ARG;
     }
     if ((long long)B * T > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
-    const bool has_tokens = (long long)B * T > 0;
-    if (has_tokens) {
-        if (!q || !k || !v || !log_alpha || !beta || !out) return KDA_ERR_INVALID_ARG;
-        if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
-            !aligned(log_alpha, 16) || !aligned(beta, 4))
+    if ((long long)B * T > 0) {
+        if (need_qk && (!q || !k || !log_alpha || !beta)) return KDA_ERR_INVALID_ARG;
+        if (need_vout && (!v || !out)) return KDA_ERR_INVALID_ARG;
+        if ((need_qk && (!aligned(q, 16) || !aligned(k, 16) || !aligned(log_alpha, 16) || !aligned(beta, 4))) ||
+            (need_vout && (!aligned(v, 16) || !aligned(out, 16))))
             return KDA_ERR_INVALID_ARG;
     }
     if ((S0 && !aligned(S0, 16)) || (S_final && !aligned(S_final, 16))) return KDA_ERR_INVALID_ARG;
     const size_t need = kda_chunk_fwd_workspace_size(B, T, H, N, dk, dv, dtype);
     if (!workspace || !aligned(workspace, 16) || workspace_bytes < need) return KDA_ERR_INVALID_ARG;
+    return KDA_OK;
+}
 
-    cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, st);
-    if (e != cudaSuccess) return KDA_ERR_CUDA;
-    if (N == 0) return KDA_OK;
-
+PrefillArgs prefill_args(const void *q, const void *k, const void *v, const float *log_alpha,
+                         const float *beta, const float *S0, const int32_t *cu_seqlens, void *out,
+                         float *S_final, int B, int T, int H, int N, void *workspace, size_t workspace_bytes)
+{
     PrefillArgs a;
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.S0 = S0;
     a.cu_seqlens = cu_seqlens; a.out = out; a.S_final = S_final;
@@ -84,14 +89,67 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v,
     a.status = (int32_t *)workspace;
     a.scratch = (unsigned char *)workspace + kStatusBytes;
     a.scratch_bytes = workspace_bytes - kStatusBytes;
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const float *beta,
+                           const float *S0, const int32_t *cu_seqlens,
+                           void *out, float *S_final,
+                           int B, int T, int H, int N, int dk, int dv,
+                           kda_dtype_t dtype, kda_dtype_t out_dtype,
+                           void *workspace, size_t workspace_bytes, void *stream)
+{
+    kda_status_t s = check_prefill(q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, N,
+                                   dk, dv, dtype, out_dtype, workspace, workspace_bytes, true, true);
+    if (s != KDA_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemsetAsync(workspace, 0, kStatusBytes, st) != cudaSuccess) return KDA_ERR_CUDA;
+    if (N == 0) return KDA_OK;
+    const PrefillArgs a = prefill_args(q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final,
+                                       B, T, H, N, workspace, workspace_bytes);
     if (dtype == KDA_BF16) {
         const int n_slots = (int)prep_slots((long long)B * T, N);
-        unsigned char *ws = (unsigned char *)workspace + kStatusBytes;
-        cudaError_t e2 = launch_chunk_prep(a, ws, n_slots, st);
-        if (e2 == cudaSuccess) e2 = launch_chunk_scan(a, ws, n_slots, out_dtype, st);
-        return map_cuda(e2);
+        cudaError_t e = launch_chunk_prep(a, (unsigned char *)a.scratch, n_slots, st);
+        if (e == cudaSuccess) e = launch_chunk_scan(a, (const unsigned char *)a.scratch, n_slots, out_dtype, st);
+        return map_cuda(e);
     }
     return map_cuda(launch_chunk_fp32(a, dtype, out_dtype, st));
+}
+
+kda_status_t kda_chunk_prep(const void *q, const void *k, const float *log_alpha, const float *beta,
+                            const int32_t *cu_seqlens, int B, int T, int H, int N, int dk, int dv,
+                            void *workspace, size_t workspace_bytes, void *stream)
+{
+    kda_status_t s = check_prefill(q, k, nullptr, log_alpha, beta, nullptr, cu_seqlens, nullptr, nullptr,
+                                   B, T, H, N, dk, dv, KDA_BF16, KDA_BF16, workspace, workspace_bytes,
+                                   true, false);
+    if (s != KDA_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemsetAsync(workspace, 0, kStatusBytes, st) != cudaSuccess) return KDA_ERR_CUDA;
+    if (N == 0) return KDA_OK;
+    const PrefillArgs a = prefill_args(q, k, nullptr, log_alpha, beta, nullptr, cu_seqlens, nullptr,
+                                       nullptr, B, T, H, N, workspace, workspace_bytes);
+    return map_cuda(launch_chunk_prep(a, (unsigned char *)a.scratch, (int)prep_slots((long long)B * T, N), st));
+}
+
+kda_status_t kda_chunk_scan(const void *v, const float *S0, const int32_t *cu_seqlens, void *out,
+                            float *S_final, int B, int T, int H, int N, int dk, int dv,
+                            kda_dtype_t out_dtype, void *workspace, size_t workspace_bytes, void *stream)
+{
+    kda_status_t s = check_prefill(nullptr, nullptr, v, nullptr, nullptr, S0, cu_seqlens, out, S_final,
+                                   B, T, H, N, dk, dv, KDA_BF16, out_dtype, workspace, workspace_bytes,
+                                   false, true);
+    if (s != KDA_OK) return s;
+    if (N == 0) return KDA_OK;
+    const PrefillArgs a = prefill_args(nullptr, nullptr, v, nullptr, nullptr, S0, cu_seqlens, out, S_final,
+                                       B, T, H, N, workspace, workspace_bytes);
+    return map_cuda(launch_chunk_scan(a, (const unsigned char *)a.scratch, (int)prep_slots((long long)B * T, N), out_dtype,
+                                      (cudaStream_t)stream));
 }
 
 kda_status_t kda_decode_step(const void *q, const void *k, const void *v,

@@ -107,3 +107,39 @@ def test_binding_refuses_cpu_tensors(lib):
     x = torch.zeros(1, 64, 2, 128)
     with pytest.raises(ValueError):
         kda.chunk_fwd(x, x, x, x, torch.zeros(1, 64, 2))
+
+
+def _prep(lib, **kw):
+    P = ctypes.c_void_p
+    a = dict(q=FAKE, k=FAKE, la=FAKE, beta=FAKE, cu=None, B=1, T=64, H=2, N=1, dk=128, dv=128,
+             ws=FAKE, wsb=256)
+    a.update(kw)
+    return lib.kda_chunk_prep(P(a["q"]), P(a["k"]), P(a["la"]), P(a["beta"]), P(a["cu"]), a["B"], a["T"],
+                              a["H"], a["N"], a["dk"], a["dv"], P(a["ws"]), a["wsb"], None)
+
+
+def _scan(lib, **kw):
+    P = ctypes.c_void_p
+    a = dict(v=FAKE, S0=None, cu=None, out=FAKE, Sf=None, B=1, T=64, H=2, N=1, dk=128, dv=128, odt=1,
+             ws=FAKE, wsb=256)
+    a.update(kw)
+    return lib.kda_chunk_scan(P(a["v"]), P(a["S0"]), P(a["cu"]), P(a["out"]), P(a["Sf"]), a["B"], a["T"],
+                              a["H"], a["N"], a["dk"], a["dv"], a["odt"], P(a["ws"]), a["wsb"], None)
+
+
+def test_two_pass_host_checks(lib):
+    need = kda.chunk_fwd_workspace_size(1, 64, 2, 1)
+    assert need > 256
+    # the first failing check decides; none of these reaches a CUDA call
+    assert _prep(lib, dk=64) == kda.KDA_ERR_UNSUPPORTED
+    assert _prep(lib, q=None) == kda.KDA_ERR_INVALID_ARG
+    assert _prep(lib, la=FAKE + 4) == kda.KDA_ERR_INVALID_ARG
+    assert _prep(lib, N=3) == kda.KDA_ERR_INVALID_ARG
+    assert _prep(lib) == kda.KDA_ERR_INVALID_ARG                          # workspace too small
+    assert _scan(lib, dv=64) == kda.KDA_ERR_UNSUPPORTED
+    assert _scan(lib, v=None) == kda.KDA_ERR_INVALID_ARG
+    assert _scan(lib, out=FAKE + 2) == kda.KDA_ERR_INVALID_ARG
+    assert _scan(lib, Sf=FAKE + 8) == kda.KDA_ERR_INVALID_ARG
+    assert _scan(lib, odt=9) == kda.KDA_ERR_INVALID_ARG
+    assert _scan(lib, B=2, cu=FAKE) == kda.KDA_ERR_INVALID_ARG
+    assert _scan(lib) == kda.KDA_ERR_INVALID_ARG                          # workspace too small

@@ -118,6 +118,24 @@ def test_causality_bitwise():
     assert not torch.equal(o1[:, t + 1:], o2[:, t + 1:])
 
 
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_two_pass_calls_equal_chunk_fwd_bitwise(out_dtype):
+    """kda_chunk_prep then kda_chunk_scan (varlen, ragged, with an empty sequence) give exactly
+    what one kda_chunk_fwd call gives."""
+    w = K.Workload("twopass", B=1, T=700, H=3, dtype="bf16", s0_std=0.1)
+    d = to_device(K.make_prefill(w, seed=11), DEV)
+    cu = torch.tensor([0, 130, 130, 451, 700], dtype=torch.int32, device=DEV)
+    S0 = torch.randn(4, 3, 128, 128, device=DEV) * 0.1
+    o1, s1 = kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=S0, cu_seqlens=cu,
+                           out_dtype=out_dtype)
+    ws = torch.empty(kda.chunk_fwd_workspace_size(1, 700, 3, 4), dtype=torch.uint8, device=DEV)
+    kda.chunk_prep(d["q"], d["k"], d["log_alpha"], d["beta"], ws, cu_seqlens=cu)
+    o2, s2 = kda.chunk_scan(d["v"], ws, S0=S0, cu_seqlens=cu, out_dtype=out_dtype)
+    assert kda.workspace_status(ws) == kda.KDA_OK
+    assert torch.equal(o1, o2)
+    assert torch.equal(s1, s2)
+
+
 def test_split_continuation():
     w = K.Workload("split", B=1, T=300, H=2, dtype="f32", s0_std=0.1)
     d = to_device(K.make_prefill(w, seed=8), DEV)
