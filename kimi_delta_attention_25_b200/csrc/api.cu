@@ -65,6 +65,9 @@ kda_status_t check_prefill(const void *q, const void *k, const void *v, const fl
         return KDA_ERR_INVALID_ARG;
     }
     if ((long long)B * T > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    // the preparation pass launches one CTA per (chunk slot, head)
+    if (dtype == KDA_BF16 && (long long)H * prep_slots((long long)B * T, N) > 0x7fffffffLL)
+        return KDA_ERR_UNSUPPORTED;
     if ((long long)B * T > 0) {
         if (need_qk && (!q || !k || !log_alpha || !beta)) return KDA_ERR_INVALID_ARG;
         if (need_vout && (!v || !out)) return KDA_ERR_INVALID_ARG;

@@ -47,6 +47,11 @@ constexpr uint32_t OFF_TB = 32768;           // Tb (f16), 64 x 128 B; N-block 0 
 constexpr uint32_t OFF_KH = 40960;           // Kh; after P1: A^T (fp32, column-major);
                                              // after P3: W (f16), N-blocks 1-2 of [Tb | W]
 constexpr uint32_t OFF_M = 57344;            // M (f16), 64 x 128 B
+// input staging of the chunk (bulk copies), dead once the rows are in registers: aliases the
+// operand tiles above, all of which are written later
+constexpr uint32_t STG_Q = 0;                // q rows, 64 x 256 B
+constexpr uint32_t STG_K = 16384;            // k rows
+constexpr uint32_t STG_LA = 32768;           // log_alpha rows, 64 x 512 B
 constexpr int LDT = 68;
 constexpr uint32_t OFF_TF = 65536;           // T (fp32, stride LDT) = 17408 B
 constexpr uint32_t OFF_PS = OFF_TF + 17408;  // 4 KB: row-block products, then inverse scratch
@@ -60,6 +65,10 @@ constexpr uint32_t TM_D1A = 0;               // Qt Kh^T  (M=64 layout), later W 
                                              // then M [Tb | W] (cols 0-191)
 constexpr uint32_t TM_D1B = 64;              // Kt Kh^T
 
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
 __device__ __forceinline__ uint2 ldg_nc_u2(const void *p) {
@@ -210,7 +219,10 @@ chunk_prep_kernel(PrepParams p)
     unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int slot = blockIdx.x, h = blockIdx.y;
+    // head fastest: the CTAs resident at one time cover all heads of a few consecutive chunks, so
+    // together they read whole [token][head][channel] rows of q, k and log_alpha (DRAM pages are
+    // used in full; with one head per row window each 8 KB row would give up 256 bytes)
+    const int h = (int)(blockIdx.x % (unsigned)p.H), slot = (int)(blockIdx.x / (unsigned)p.H);
     const int H = p.H;
 
     int64_t tok0;
@@ -225,10 +237,30 @@ chunk_prep_kernel(PrepParams p)
     float *Ps = reinterpret_cast<float *>(sm + OFF_PS);
     float *bet = reinterpret_cast<float *>(sm + OFF_BET);
 
+    uint64_t *bar_in = bar + 2;
     if (warp == 0) { tmem_alloc(tmem_slot, TMEM_COLS); tmem_relinquish(); }
-    if (tid == 0) { mbar_init(bar, 1); fence_mbar_init(); }
-
-    // ---- loads: warp w -> rows 8w..8w+7, lane -> channels 4 lane..4 lane+3 (a warp reads whole rows)
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_init(bar_in, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(bar_in, (uint32_t)L * (2 * DK * 2 + DK * 4));
+    }
+    __syncthreads();
+    // ---- loads: one bulk copy per row of q, k (256 B) and log_alpha (512 B) into the staging
+    //      area, then warp w -> rows 8w..8w+7, lane -> channels 4 lane..4 lane+3 into registers
+    if (tid < 3 * C) {
+        const int arr = tid / C, r = tid % C;
+        if (r < L) {
+            const size_t row = ((size_t)(tok0 + r) * H + h) * DK;
+            if (arr == 0) bulk_g2s(sbase + STG_Q + r * 256, p.q + row, 256, bar_in);
+            else if (arr == 1) bulk_g2s(sbase + STG_K + r * 256, p.k + row, 256, bar_in);
+            else bulk_g2s(sbase + STG_LA + r * 512, p.log_alpha + row, 512, bar_in);
+        }
+    }
+    if (!mbar_wait(bar_in, 0)) {
+        set_status(p.status, KDA_ERR_TIMEOUT);
+        mbar_wait(bar_in, 0, 100000000LL);         // copies still landing must not outlive the CTA
+    }
     const int cq = lane, kh = cq >> 4, lc4 = cq & 15;
     float4 la[8];
     uint2 kr[8], qr[8];
@@ -236,10 +268,9 @@ chunk_prep_kernel(PrepParams p)
     for (int x = 0; x < 8; ++x) {
         const int r = 8 * warp + x;
         if (r < L) {
-            const size_t row = ((size_t)(tok0 + r) * H + h) * DK + 4 * cq;
-            la[x] = ldg_nc_f4(p.log_alpha + row);
-            kr[x] = ldg_nc_u2(p.k + row);
-            qr[x] = ldg_nc_u2(p.q + row);
+            la[x] = *reinterpret_cast<const float4 *>(sm + STG_LA + r * 512 + 16 * cq);
+            kr[x] = *reinterpret_cast<const uint2 *>(sm + STG_K + r * 256 + 8 * cq);
+            qr[x] = *reinterpret_cast<const uint2 *>(sm + STG_Q + r * 256 + 8 * cq);
         } else {
             la[x] = make_float4(0.f, 0.f, 0.f, 0.f);
             kr[x] = make_uint2(0u, 0u);
@@ -279,12 +310,9 @@ chunk_prep_kernel(PrepParams p)
         g[e] = before[e] * pre[7][e] * after[e];
         rg[e] = __frcp_rn(g[e]);
     }
-    if (warp == 0) {
-        float *gw = reinterpret_cast<float *>(blk + kPrepGammaOff);
-        *reinterpret_cast<float4 *>(gw + 4 * cq) = make_float4(g[0], g[1], g[2], g[3]);
-        if (g[0] < kMinChunkDecay || g[1] < kMinChunkDecay || g[2] < kMinChunkDecay || g[3] < kMinChunkDecay)
-            set_status(p.status, KDA_ERR_UNSUPPORTED);
-    }
+    // Workspace (global) stores of each phase are issued after that phase's proxy fence and MMA
+    // issue: a fence.proxy.async would otherwise also wait for them to complete.
+    uint2 kend[8];
     {
         float suf[4] = {1.f, 1.f, 1.f, 1.f};
 #pragma unroll
@@ -312,7 +340,7 @@ chunk_prep_kernel(PrepParams p)
             *reinterpret_cast<uint2 *>(sm + OFF_KT + kh * 8192 + off) = make_uint2(okt[0], okt[1]);
             *reinterpret_cast<uint2 *>(sm + OFF_QT + kh * 8192 + off) = make_uint2(oqt[0], oqt[1]);
             *reinterpret_cast<uint2 *>(sm + OFF_KH + kh * 8192 + off) = make_uint2(okh[0], okh[1]);
-            *reinterpret_cast<uint2 *>(blk + kPrepKEOff + kh * 8192 + off) = make_uint2(oke[0], oke[1]);
+            kend[x] = make_uint2(oke[0], oke[1]);
         }
     }
     fence_proxy_async_smem();
@@ -332,6 +360,18 @@ chunk_prep_kernel(PrepParams p)
             umma_ss(tmem + TM_D1B, smem_desc(sbase + OFF_KT + k2 * 8192 + ko, 16, 1024, SW_128B), bd, id, ks > 0);
         }
         umma_commit(bar);
+    }
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+        const int r = 8 * warp + x;
+        const uint32_t off = r * 128 + ((((lc4 >> 1) ^ (r & 7)) & 7) << 4) + ((lc4 & 1) << 3);
+        *reinterpret_cast<uint2 *>(blk + kPrepKEOff + kh * 8192 + off) = kend[x];
+    }
+    if (warp == 0) {
+        float *gw = reinterpret_cast<float *>(blk + kPrepGammaOff);
+        *reinterpret_cast<float4 *>(gw + 4 * cq) = make_float4(g[0], g[1], g[2], g[3]);
+        if (g[0] < kMinChunkDecay || g[1] < kMinChunkDecay || g[2] < kMinChunkDecay || g[3] < kMinChunkDecay)
+            set_status(p.status, KDA_ERR_UNSUPPORTED);
     }
     int32_t failed = 0;
     if (tid == 0 && !mbar_wait(bar, 0)) failed = 1;
@@ -386,9 +426,6 @@ chunk_prep_kernel(PrepParams p)
             }
             const uint4 o = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             *reinterpret_cast<uint4 *>(sm + OFF_TB + sw128_offset(r, cb)) = o;
-            const uint32_t sgn = 0x80008000u;        // f16 sign bits: -Tb
-            *reinterpret_cast<uint4 *>(blk + kPrepYOff + sw128_offset(r, cb)) =
-                make_uint4(o.x ^ sgn, o.y ^ sgn, o.z ^ sgn, o.w ^ sgn);
         }
     }
     fence_proxy_async_smem();
@@ -403,6 +440,16 @@ chunk_prep_kernel(PrepParams p)
             umma_ss(tmem + TM_D1A, smem_desc(sbase + OFF_TB + ks * 32, 16, 1024, SW_128B),
                     smem_desc(sbase + OFF_KT + ks * 2048, 8192, 1024, SW_128B), id, ks > 0);
         umma_commit(bar);
+    }
+    {   // -Tb to the workspace (Y rows 0-63), from its shared-memory copy
+        const int r = tid >> 2, c0 = (tid & 3) * 16;
+        const uint32_t sgn = 0x80008000u;            // f16 sign bits
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const uint32_t o = sw128_offset(r, c0 + 8 * hh);
+            const uint4 t = *reinterpret_cast<const uint4 *>(sm + OFF_TB + o);
+            *reinterpret_cast<uint4 *>(blk + kPrepYOff + o) = make_uint4(t.x ^ sgn, t.y ^ sgn, t.z ^ sgn, t.w ^ sgn);
+        }
     }
     if (tid == 0 && !failed && !mbar_wait(bar, 1)) failed = 1;
     __syncthreads();
@@ -422,7 +469,6 @@ chunk_prep_kernel(PrepParams p)
                 o.y = pack_f16x2(w[8 * ch + 2], w[8 * ch + 3]);
                 o.z = pack_f16x2(w[8 * ch + 4], w[8 * ch + 5]);
                 o.w = pack_f16x2(w[8 * ch + 6], w[8 * ch + 7]);
-                *reinterpret_cast<uint4 *>(blk + kPrepXOff + half * 16384 + sw128_offset(r, 8 * ch)) = o;
                 *reinterpret_cast<uint4 *>(sm + OFF_KH + half * 8192 + sw128_offset(r, 8 * ch)) = o;
             }
         }
@@ -439,8 +485,20 @@ chunk_prep_kernel(PrepParams p)
             umma_ss(tmem + TM_D1A, smem_desc(sbase + OFF_M + ks * 32, 16, 1024, SW_128B),
                     smem_desc(sbase + OFF_TB + ks * 2048, 8192, 1024, SW_128B), id, ks > 0);
         umma_commit(bar);
-        if (!mbar_wait(bar, 0)) failed = 1;
     }
+    {   // W to the workspace (X rows 0-63), from its shared-memory copy
+        const int q4 = warp & 3, half = warp >> 2;
+        if (lane < 16) {
+            const int r = 16 * q4 + lane;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                const uint32_t o = sw128_offset(r, 8 * ch);
+                *reinterpret_cast<uint4 *>(blk + kPrepXOff + half * 16384 + o) =
+                    *reinterpret_cast<const uint4 *>(sm + OFF_KH + half * 8192 + o);
+            }
+        }
+    }
+    if (tid == 0 && !failed && !mbar_wait(bar, 0)) failed = 1;
     __syncthreads();
     tc_fence_after();
     // ---- P4 epilogue: warps 0-3: M Tb (cols 0-63) -> Y rows 64-127, then Qt - M W for channels
@@ -500,7 +558,7 @@ cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slo
     cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    const dim3 grid(n_slots, a.H);
+    const dim3 grid((unsigned)n_slots * (unsigned)a.H);
     chunk_prep_kernel<<<grid, NT, SMEM_ALLOC, stream>>>(p);
     return cudaGetLastError();
 }
