@@ -22,7 +22,10 @@
 //   [64K, +512) gamma (fp32)
 // A chunk slot is floor(first_token / 64) + sequence, which is unique per (sequence, chunk) and
 // below floor(total_tokens / 64) + N + 1.
+#include <cuda.h>
 #include <cuda_fp16.h>
+
+#include <mutex>
 
 #include "kda_internal.cuh"
 #include "sm100.cuh"
@@ -65,10 +68,6 @@ constexpr uint32_t TM_D1A = 0;               // Qt Kh^T  (M=64 layout), later W 
                                              // then M [Tb | W] (cols 0-191)
 constexpr uint32_t TM_D1B = 64;              // Kt Kh^T
 
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
-}
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
 __device__ __forceinline__ uint2 ldg_nc_u2(const void *p) {
@@ -213,7 +212,8 @@ __device__ __forceinline__ void inverse64(int pt, const float *AT, float *Tf, fl
 }
 
 __global__ void __launch_bounds__(NT, 2)
-chunk_prep_kernel(PrepParams p)
+chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_la)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -240,23 +240,18 @@ chunk_prep_kernel(PrepParams p)
     uint64_t *bar_in = bar + 2;
     if (warp == 0) { tmem_alloc(tmem_slot, TMEM_COLS); tmem_relinquish(); }
     if (tid == 0) {
+        // ---- loads: the chunk's 64 rows of q, k and log_alpha for this head, one tensor copy each
+        //      (rows past the end of the tensor read as zero; rows of the next sequence are masked
+        //      below); then warp w -> rows 8w..8w+7, lane -> channels 4 lane..4 lane+3 into registers
         mbar_init(bar, 1);
         mbar_init(bar_in, 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(bar_in, (uint32_t)L * (2 * DK * 2 + DK * 4));
+        mbar_arrive_expect_tx(bar_in, (uint32_t)C * (2 * DK * 2 + DK * 4));
+        tma_load_3d(sm + STG_Q, &tm_q, bar_in, 0, h, (int)tok0);
+        tma_load_3d(sm + STG_K, &tm_k, bar_in, 0, h, (int)tok0);
+        tma_load_3d(sm + STG_LA, &tm_la, bar_in, 0, h, (int)tok0);
     }
     __syncthreads();
-    // ---- loads: one bulk copy per row of q, k (256 B) and log_alpha (512 B) into the staging
-    //      area, then warp w -> rows 8w..8w+7, lane -> channels 4 lane..4 lane+3 into registers
-    if (tid < 3 * C) {
-        const int arr = tid / C, r = tid % C;
-        if (r < L) {
-            const size_t row = ((size_t)(tok0 + r) * H + h) * DK;
-            if (arr == 0) bulk_g2s(sbase + STG_Q + r * 256, p.q + row, 256, bar_in);
-            else if (arr == 1) bulk_g2s(sbase + STG_K + r * 256, p.k + row, 256, bar_in);
-            else bulk_g2s(sbase + STG_LA + r * 512, p.log_alpha + row, 512, bar_in);
-        }
-    }
     if (!mbar_wait(bar_in, 0)) {
         set_status(p.status, KDA_ERR_TIMEOUT);
         mbar_wait(bar_in, 0, 100000000LL);         // copies still landing must not outlive the CTA
@@ -546,6 +541,39 @@ chunk_prep_kernel(PrepParams p)
     if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
 }
 
+// Tensor map of a [tokens][H][128] row-major tensor whose box is the 64 token rows of one head.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, []() {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+bool token_rows_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint32_t elem_bytes, int H,
+                    long long tokens)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)DK, (cuuint64_t)H, (cuuint64_t)tokens};
+    const cuuint64_t strides[2] = {(cuuint64_t)DK * elem_bytes, (cuuint64_t)DK * elem_bytes * H};
+    const cuuint32_t box[3] = {(cuuint32_t)DK, 1u, (cuuint32_t)C};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slots, cudaStream_t stream)
@@ -554,12 +582,19 @@ cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slo
     p.q = (const __nv_bfloat16 *)a.q; p.k = (const __nv_bfloat16 *)a.k;
     p.log_alpha = a.log_alpha; p.beta = a.beta; p.cu_seqlens = a.cu_seqlens;
     p.ws = ws; p.T = a.T; p.H = a.H; p.N = a.N; p.n_slots = n_slots; p.status = a.status;
+    const long long tokens = (long long)a.B * a.T;
+    if (tokens == 0) return cudaSuccess;          // no chunk to prepare
+    CUtensorMap tq, tk, tla;
+    if (!token_rows_map(&tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, tokens) ||
+        !token_rows_map(&tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, tokens) ||
+        !token_rows_map(&tla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.H, tokens))
+        return cudaErrorNotSupported;
 
     cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)n_slots * (unsigned)a.H);
-    chunk_prep_kernel<<<grid, NT, SMEM_ALLOC, stream>>>(p);
+    chunk_prep_kernel<<<grid, NT, SMEM_ALLOC, stream>>>(p, tq, tk, tla);
     return cudaGetLastError();
 }
 
