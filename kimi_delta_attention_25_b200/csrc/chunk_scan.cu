@@ -48,6 +48,11 @@ constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
 static_assert(SMEM_ALLOC <= 232448, "shared memory plan exceeds 227 KiB");
 static_assert(kPrepBlockBytes <= ST_V && STAGE % 1024 == 0 && kPrepBlockBytes % 16 == 0, "stage layout");
 
+// The blocks come from DRAM (the workspace is far larger than L2) and the ring holds three chunks,
+// so with copies issued only as stages free up the DRAM latency divided by the ring depth would set
+// the chunk rate. Each block is also asked into L2 this many chunks ahead.
+constexpr int PREFETCH_AHEAD = 6;
+
 constexpr uint32_t TMEM_COLS = 128;
 constexpr uint32_t TM_D5 = 0;                 // 2 x 32 columns: [-U; O], by chunk parity
 constexpr uint32_t TM_D7 = 64;                // 32 columns: Kend^T U
@@ -79,6 +84,9 @@ struct ScanParams {
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                  ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 __device__ __forceinline__ uint4 ldg_nc(const void *p) {
     uint4 r;
@@ -194,16 +202,24 @@ chunk_scan_kernel(ScanParams p)
             }
         };
         if (nchunks > 0) load_v(0);
+        auto block_of = [&](int c) {
+            return p.ws + ((size_t)h * p.n_slots + (first_slot + c)) * kPrepBlockBytes;
+        };
+        // one CTA of the four that share a head's blocks asks for them into L2
+        if (jb == 0 && lane == 0)
+            for (int c = 0; c < PREFETCH_AHEAD && c < nchunks; ++c) prefetch_l2(block_of(c), (uint32_t)kPrepBlockBytes);
         int n_loaded = 0;
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % NSTAGE;
             unsigned char *stg = sm + s * STAGE;
+            if (jb == 0 && lane == 0 && c + PREFETCH_AHEAD < nchunks)
+                prefetch_l2(block_of(c + PREFETCH_AHEAD), (uint32_t)kPrepBlockBytes);
             if (warp_abort()) break;
             int ok = 1;
             if (c >= NSTAGE && lane == 0) ok = mbar_wait(&bars[B_EMPTY + s], ((c / NSTAGE) - 1) & 1);
             if (!__shfl_sync(0xffffffffu, ok, 0)) { if (lane == 0) fail(); break; }
             if (lane == 0) {
-                const unsigned char *blk = p.ws + ((size_t)h * p.n_slots + (first_slot + c)) * kPrepBlockBytes;
+                const unsigned char *blk = block_of(c);
                 mbar_arrive_expect_tx(&bars[B_FULL + s], (uint32_t)kPrepBlockBytes);
                 bulk_g2s(stg, blk, (uint32_t)kPrepBlockBytes, &bars[B_FULL + s]);
             }
