@@ -88,6 +88,7 @@ struct PrepParams {
     const int32_t *cu_seqlens;
     unsigned char *ws;              // chunk blocks, [H][n_slots][kPrepBlockBytes]
     int T, H, N, n_slots;
+    int prefetch_wave;              // CTAs resident at once; > 0: prefetch that many units ahead
     int32_t *status;
 };
 
@@ -250,6 +251,19 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
         tma_load_3d(sm + STG_Q, &tm_q, bar_in, 0, h, (int)tok0);
         tma_load_3d(sm + STG_K, &tm_k, bar_in, 0, h, (int)tok0);
         tma_load_3d(sm + STG_LA, &tm_la, bar_in, 0, h, (int)tok0);
+        // ask for the inputs of the unit one wave of resident CTAs ahead into L2, so that its
+        // tensor copies are served from L2 instead of waiting on DRAM
+        if (p.prefetch_wave > 0) {
+            const long long nxt = (long long)blockIdx.x + p.prefetch_wave;
+            int64_t ptok;
+            int pL;
+            if (nxt < (long long)gridDim.x && slot_chunk(p, (int)(nxt / H), &ptok, &pL)) {
+                const int ph = (int)(nxt % H);
+                tma_prefetch_3d(&tm_q, 0, ph, (int)ptok);
+                tma_prefetch_3d(&tm_k, 0, ph, (int)ptok);
+                tma_prefetch_3d(&tm_la, 0, ph, (int)ptok);
+            }
+        }
     }
     __syncthreads();
     if (!mbar_wait(bar_in, 0)) {
@@ -582,6 +596,11 @@ cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slo
     p.q = (const __nv_bfloat16 *)a.q; p.k = (const __nv_bfloat16 *)a.k;
     p.log_alpha = a.log_alpha; p.beta = a.beta; p.cu_seqlens = a.cu_seqlens;
     p.ws = ws; p.T = a.T; p.H = a.H; p.N = a.N; p.n_slots = n_slots; p.status = a.status;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sms = 0;
+    p.prefetch_wave = 2 * sms;                    // two CTAs per SM
     const long long tokens = (long long)a.B * a.T;
     if (tokens == 0) return cudaSuccess;          // no chunk to prepare
     CUtensorMap tq, tk, tla;
