@@ -175,6 +175,18 @@ kda_status_t kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
                                    int B, int T, int H, int N, int dk, int dv,
                                    kda_dtype_t dtype, kda_dtype_t out_dtype, void *stream);
 
+/* Self-test of the library's failure detection (the pages have no counterpart): every device-side
+ * wait of the kernels (on an mbarrier or a copy) is bounded and, when it runs out, records
+ * KDA_ERR_TIMEOUT in the workspace status word and lets the kernel return, so that the CUDA context
+ * stays usable. This call launches one tiny kernel that makes such a wait on a barrier nothing
+ * arrives on, with a limit of budget_cycles SM clock cycles (1 .. KDA_SELFTEST_MAX_BUDGET), so the
+ * caller can read KDA_ERR_TIMEOUT back with kda_workspace_status. workspace: at least 256 bytes,
+ * 16-byte aligned; its status word is cleared first. Returns KDA_ERR_INVALID_ARG for a bad
+ * workspace or budget. */
+#define KDA_SELFTEST_MAX_BUDGET 2000000000LL
+kda_status_t kda_selftest_wait_timeout(void *workspace, size_t workspace_bytes,
+                                       long long budget_cycles, void *stream);
+
 /* Waits for `stream`, then copies the workspace status word to *status
  * (KDA_OK when every device-side check passed). */
 kda_status_t kda_workspace_status(const void *workspace, void *stream, int32_t *status);

@@ -35,7 +35,7 @@ _lib = None
 # Every entry point declared in include/libkda.h.
 EXPORTS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
            "kda_workspace_status", "kda_status_string", "kda_version", "kda_chunk_fwd_noalloc",
-           "kda_chunk_prep", "kda_chunk_scan")
+           "kda_chunk_prep", "kda_chunk_scan", "kda_selftest_wait_timeout")
 
 
 class KDAError(RuntimeError):
@@ -71,6 +71,8 @@ def load():
     lib.kda_chunk_prep.restype = I
     lib.kda_chunk_scan.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, Z, P]
     lib.kda_chunk_scan.restype = I
+    lib.kda_selftest_wait_timeout.argtypes = [P, Z, ctypes.c_longlong, P]
+    lib.kda_selftest_wait_timeout.restype = I
     _lib = lib
     return lib
 
@@ -174,6 +176,16 @@ def chunk_scan(v, workspace, S0=None, cu_seqlens=None, out=None, S_final=None, w
     if st != KDA_OK:
         raise KDAError(st, "kda_chunk_scan")
     return out, S_final
+
+
+def selftest_wait_timeout(workspace: torch.Tensor, budget_cycles: int) -> None:
+    """``kda_selftest_wait_timeout``: one bounded device wait on a barrier nothing arrives on; the
+    workspace status word then reads ``KDA_ERR_TIMEOUT`` (check it with ``workspace_status``)."""
+    _need_cuda(workspace)
+    st = load().kda_selftest_wait_timeout(_ptr(workspace), workspace.numel(), int(budget_cycles),
+                                          _stream(workspace.device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_selftest_wait_timeout")
 
 
 def workspace_status(workspace: torch.Tensor) -> int:

@@ -143,3 +143,13 @@ def test_two_pass_host_checks(lib):
     assert _scan(lib, odt=9) == kda.KDA_ERR_INVALID_ARG
     assert _scan(lib, B=2, cu=FAKE) == kda.KDA_ERR_INVALID_ARG
     assert _scan(lib) == kda.KDA_ERR_INVALID_ARG                          # workspace too small
+
+
+def test_selftest_host_checks(lib):
+    P = ctypes.c_void_p
+    f = lib.kda_selftest_wait_timeout
+    assert f(None, 256, 1000, None) == kda.KDA_ERR_INVALID_ARG
+    assert f(P(FAKE), 128, 1000, None) == kda.KDA_ERR_INVALID_ARG          # smaller than the status header
+    assert f(P(FAKE + 8), 256, 1000, None) == kda.KDA_ERR_INVALID_ARG      # misaligned
+    assert f(P(FAKE), 256, 0, None) == kda.KDA_ERR_INVALID_ARG
+    assert f(P(FAKE), 256, 2000000001, None) == kda.KDA_ERR_INVALID_ARG
