@@ -44,8 +44,10 @@ constexpr int NT = 256;
 constexpr float kMinChunkDecay = 3.0517578125e-05f;
 
 // shared memory (1024-aligned base)
-constexpr uint32_t OFF_QT = 0;               // Qt (f16), two halves of 64 x 128 B
-constexpr uint32_t OFF_KT = 16384;           // Kt
+constexpr uint32_t OFF_QK = 0;               // [Qt; Kt] (f16): per 64-channel half (16 KB apart),
+                                             // rows 0-63 Qt then rows 64-127 Kt, 128 B per row
+constexpr uint32_t QK_HALF = 16384;
+constexpr uint32_t OFF_KT = OFF_QK + 8192;   // Kt rows of half 0 (half 1 at + QK_HALF)
 constexpr uint32_t OFF_TB = 32768;           // Tb (f16), 64 x 128 B; N-block 0 of [Tb | W]
 constexpr uint32_t OFF_KH = 40960;           // Kh; after P1: A^T (fp32, column-major);
                                              // after P3: W (f16), N-blocks 1-2 of [Tb | W]
@@ -64,9 +66,8 @@ constexpr uint32_t SMEM_BYTES = OFF_BAR + 64;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
 
 constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t TM_D1A = 0;               // Qt Kh^T  (M=64 layout), later W (cols 0-127),
+constexpr uint32_t TM_D1A = 0;               // [Qt; Kt] Kh^T (M=128, 64 cols), later W (cols 0-127),
                                              // then M [Tb | W] (cols 0-191)
-constexpr uint32_t TM_D1B = 64;              // Kt Kh^T
 
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
@@ -346,8 +347,8 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) suf[e] *= a[x][e];
-            *reinterpret_cast<uint2 *>(sm + OFF_KT + kh * 8192 + off) = make_uint2(okt[0], okt[1]);
-            *reinterpret_cast<uint2 *>(sm + OFF_QT + kh * 8192 + off) = make_uint2(oqt[0], oqt[1]);
+            *reinterpret_cast<uint2 *>(sm + OFF_KT + kh * QK_HALF + off) = make_uint2(okt[0], okt[1]);
+            *reinterpret_cast<uint2 *>(sm + OFF_QK + kh * QK_HALF + off) = make_uint2(oqt[0], oqt[1]);
             *reinterpret_cast<uint2 *>(sm + OFF_KH + kh * 8192 + off) = make_uint2(okh[0], okh[1]);
             kend[x] = make_uint2(oke[0], oke[1]);
         }
@@ -358,15 +359,14 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // ---- P1: D1A = Qt Kh^T, D1B = Kt Kh^T (M=64, N=64, K=128)
+    // ---- P1: D1A = [Qt; Kt] Kh^T (M=128, N=64, K=128): rows 0-63 Qt Kh^T, rows 64-127 Kt Kh^T
     if (tid == 0) {
-        const uint32_t id = idesc_f16(64, 64, 0, 0);
+        const uint32_t id = idesc_f16(128, 64, 0, 0);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
             const uint32_t k2 = ks >> 2, ko = (ks & 3) * 32;
-            const uint64_t bd = smem_desc(sbase + OFF_KH + k2 * 8192 + ko, 16, 1024, SW_128B);
-            umma_ss(tmem + TM_D1A, smem_desc(sbase + OFF_QT + k2 * 8192 + ko, 16, 1024, SW_128B), bd, id, ks > 0);
-            umma_ss(tmem + TM_D1B, smem_desc(sbase + OFF_KT + k2 * 8192 + ko, 16, 1024, SW_128B), bd, id, ks > 0);
+            umma_ss(tmem + TM_D1A, smem_desc(sbase + OFF_QK + k2 * QK_HALF + ko, 16, 1024, SW_128B),
+                    smem_desc(sbase + OFF_KH + k2 * 8192 + ko, 16, 1024, SW_128B), id, ks > 0);
         }
         umma_commit(bar);
     }
@@ -386,30 +386,31 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
     if (tid == 0 && !mbar_wait(bar, 0)) failed = 1;
     __syncthreads();
     tc_fence_after();
-    // ---- P1 epilogue: warps 0-3 -> M (f16, smem); warps 4-7 -> A^T (fp32, smem)
+    // ---- P1 epilogue (M=128: lane = row): rows 0-63 -> M (f16, smem), rows 64-127 -> A^T (fp32,
+    //      smem); warp w takes columns 32 (w / 4) .. +31 of its rows
     {
         const int q4 = warp & 3, half = warp >> 2;
-        float v[64];
-        tmem_ld64_sync(tmem + ((uint32_t)(32 * q4) << 16) + (half ? TM_D1B : TM_D1A), v);
-        if (lane < 16) {
-            const int r = 16 * q4 + lane;
-            if (half == 0) {
+        const int row = 32 * q4 + lane, c0 = 32 * half;
+        float v[32];
+        tmem_ld32_sync(tmem + ((uint32_t)(32 * q4) << 16) + TM_D1A + c0, v);
+        if (q4 < 2) {
+            const int r = row;
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t w4[4];
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t w4[4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int i = 8 * ch + 2 * u;
-                        w4[u] = pack_f16x2(i <= r ? v[i] : 0.f, i + 1 <= r ? v[i + 1] : 0.f);
-                    }
-                    *reinterpret_cast<uint4 *>(sm + OFF_M + sw128_offset(r, 8 * ch)) =
-                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                for (int u = 0; u < 4; ++u) {
+                    const int i = c0 + 8 * ch + 2 * u;
+                    w4[u] = pack_f16x2(i <= r ? v[8 * ch + 2 * u] : 0.f, i + 1 <= r ? v[8 * ch + 2 * u + 1] : 0.f);
                 }
-            } else {
-                const float br = bet[r];
-#pragma unroll
-                for (int i = 0; i < 64; ++i) AT[i * 64 + r] = (i < r) ? br * v[i] : 0.f;
+                *reinterpret_cast<uint4 *>(sm + OFF_M + sw128_offset(r, c0 + 8 * ch)) =
+                    make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
+        } else {
+            const int r = row - 64;
+            const float br = bet[r];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) AT[(c0 + j) * 64 + r] = (c0 + j < r) ? br * v[j] : 0.f;
         }
     }
     tc_fence_before();
@@ -447,7 +448,7 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
             umma_ss(tmem + TM_D1A, smem_desc(sbase + OFF_TB + ks * 32, 16, 1024, SW_128B),
-                    smem_desc(sbase + OFF_KT + ks * 2048, 8192, 1024, SW_128B), id, ks > 0);
+                    smem_desc(sbase + OFF_KT + ks * 2048, QK_HALF, 1024, SW_128B), id, ks > 0);
         umma_commit(bar);
     }
     {   // -Tb to the workspace (Y rows 0-63), from its shared-memory copy
@@ -534,7 +535,7 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
                     const int kh = part - 1;
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) {
-                        const uint4 qv = *reinterpret_cast<const uint4 *>(sm + OFF_QT + kh * 8192 + sw128_offset(r, 8 * ch));
+                        const uint4 qv = *reinterpret_cast<const uint4 *>(sm + OFF_QK + kh * QK_HALF + sw128_offset(r, 8 * ch));
                         const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
                         uint32_t o[4];
 #pragma unroll
