@@ -511,39 +511,37 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
     if (tid == 0 && !failed && !mbar_wait(bar, 0)) failed = 1;
     __syncthreads();
     tc_fence_after();
-    // ---- P4 epilogue: warps 0-3: M Tb (cols 0-63) -> Y rows 64-127, then Qt - M W for channels
-    //      0-63 (cols 64-127); warps 4-7: Qt - M W for channels 64-127 (cols 128-191) -> X rows 64-127
+    // ---- P4 epilogue (M=64 layout: lanes 0-15 of each quadrant), warps 0-3 cols 0-95, 4-7 cols
+    //      96-191, in 32-column groups: M Tb (cols 0-63) -> Y rows 64-127; Qt - M W (cols 64-191,
+    //      channel = col - 64) -> X rows 64-127
     {
         const int q4 = warp & 3, half = warp >> 2;
         const int r = 16 * q4 + (lane & 15);
-        const int part_end = half ? 3 : 2;
-        for (int part = half ? 2 : 0; part < part_end; ++part) {   // warps 0-3: parts 0, 1; 4-7: part 2
-            float m[64];
-            tmem_ld64_sync(tmem + ((uint32_t)(32 * q4) << 16) + TM_D1A + 64 * part, m);
+#pragma unroll
+        for (int grp = 0; grp < 3; ++grp) {
+            const int c0 = 96 * half + 32 * grp;
+            float m[32];
+            tmem_ld32_sync(tmem + ((uint32_t)(32 * q4) << 16) + TM_D1A + c0, m);
             if (lane < 16) {
-                if (part == 0) {
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        uint4 o;
-                        o.x = pack_f16x2(m[8 * ch + 0], m[8 * ch + 1]);
-                        o.y = pack_f16x2(m[8 * ch + 2], m[8 * ch + 3]);
-                        o.z = pack_f16x2(m[8 * ch + 4], m[8 * ch + 5]);
-                        o.w = pack_f16x2(m[8 * ch + 6], m[8 * ch + 7]);
-                        *reinterpret_cast<uint4 *>(blk + kPrepYOff + sw128_offset(64 + r, 8 * ch)) = o;
-                    }
-                } else {
-                    const int kh = part - 1;
+                for (int u8 = 0; u8 < 4; ++u8) {
+                    const int c = c0 + 8 * u8;                 // 8 columns c .. c + 7
+                    uint32_t o[4];
+                    if (c < 64) {
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        const uint4 qv = *reinterpret_cast<const uint4 *>(sm + OFF_QK + kh * QK_HALF + sw128_offset(r, 8 * ch));
+                        for (int u = 0; u < 4; ++u) o[u] = pack_f16x2(m[8 * u8 + 2 * u], m[8 * u8 + 2 * u + 1]);
+                        *reinterpret_cast<uint4 *>(blk + kPrepYOff + sw128_offset(64 + r, c)) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
+                    } else {
+                        const int kh = (c - 64) >> 6, cc = (c - 64) & 63;
+                        const uint4 qv = *reinterpret_cast<const uint4 *>(sm + OFF_QK + kh * QK_HALF + sw128_offset(r, cc));
                         const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-                        uint32_t o[4];
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
                             const float2 qf = __half22float2(*reinterpret_cast<const __half2 *>(&qw[u]));
-                            o[u] = pack_f16x2(qf.x - m[8 * ch + 2 * u], qf.y - m[8 * ch + 2 * u + 1]);
+                            o[u] = pack_f16x2(qf.x - m[8 * u8 + 2 * u], qf.y - m[8 * u8 + 2 * u + 1]);
                         }
-                        *reinterpret_cast<uint4 *>(blk + kPrepXOff + kh * 16384 + 64 * 128 + sw128_offset(r, 8 * ch)) =
+                        *reinterpret_cast<uint4 *>(blk + kPrepXOff + kh * 16384 + 64 * 128 + sw128_offset(r, cc)) =
                             make_uint4(o[0], o[1], o[2], o[3]);
                     }
                 }
