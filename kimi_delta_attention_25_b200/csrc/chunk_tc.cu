@@ -16,14 +16,17 @@
 //   W  = Tb Kt;   U = Tb V - W S;   O = Qt S + M U;   S <- Diag(gamma) S + Kend^T U
 // f and b are running products of alpha = exp(log_alpha) (forward and backward within the chunk).
 //
+// This single-kernel form needs no workspace beyond the status word, so kda_chunk_fwd_noalloc runs
+// it; kda_chunk_fwd runs the faster two-pass form (chunk_prep.cu, chunk_scan.cu).
+//
 // Work split: one CTA per (sequence, head, 32-column block of d_v). The value columns of S evolve
 // independently, so the four blocks of a head never communicate; each recomputes the
 // d_v-independent part of a chunk. Inside a CTA two warp groups run a two-stage pipeline:
 //
 //   prep group (8 warps) for chunk c+1            scan group (4 warps) for chunk c
 //   --------------------------------------        ------------------------------------------
-//   coalesced loads (next chunk prefetched         S1: D5 += [W; Qt] S          (M=128,N=32,K=128)
-//     to L2 one chunk ahead)                       U  = -(D5 rows 0-63) -> f16
+//   coalesced loads of the chunk's rows            S1: D5 += [W; Qt] S          (M=128,N=32,K=128)
+//                                                  U  = -(D5 rows 0-63) -> f16
 //   decay scaling (fp32) -> Kt Qt Kh Kend (f16)    S2: D7 = Kend^T U            (M=128,N=32,K=64)
 //   P1: Qt Kh^T, Kt Kh^T  (two M=64, N=64, K=128)  MU: D5 += [0; M] U           (M=128,N=32,K=64)
 //   M (f16), A (fp32); T = (I + A)^{-1} (fp32,     S <- gamma S + D7 (fp32 registers), S -> f16
@@ -107,9 +110,6 @@ struct TcParams {
 
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
-__device__ __forceinline__ void prefetch_l2(const void *p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
 __device__ __forceinline__ uint4 ldg_nc(const void *p) {
     uint4 r;
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
