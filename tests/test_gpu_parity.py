@@ -250,3 +250,74 @@ def test_tensor_core_path_reports_out_of_range_decay():
     ro, rs = oracle_prefill(f)
     assert_close(np32(out), ro, TOL[torch.float32], "out")
     assert_close(np32(Sf), rs, TOL[torch.float32], "S_final")
+
+
+# ---- degenerate cases of the method, against closed forms ----------------------------------
+
+def _closed_form_out(S_seq, q):
+    """o_t = S_t^T q_t for a list of per-token states [T, dk, dv] and queries [T, dk]."""
+    return np.einsum("tkv,tk->tv", S_seq, q)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_beta_zero_is_pure_decay(dtype):
+    """With beta = 0 the delta-rule write vanishes and the recurrence is S_t = Diag(alpha_t) S_{t-1}:
+    the state is S0 scaled per key channel by the running product of the decays, and the output
+    reads that state (the gated delta rule of Kimi Linear, section 3.1, with the write term zero)."""
+    w = K.Workload("beta0", B=1, T=200, H=2, dtype=dtype, alpha_lo=0.9, alpha_hi=0.999, s0_std=0.5)
+    d = K.make_prefill(w, seed=21)
+    d["beta"] = torch.zeros_like(d["beta"])
+    g = to_device(d, DEV)
+    out, Sf = kda.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], S0=g["S0"])
+    assert kda.workspace_status(kda.chunk_fwd.last_workspace) == kda.KDA_OK
+    tol = TOL[K.to_dtype(dtype)]
+    q = d["q"].double().numpy()[0]
+    G = np.cumsum(d["log_alpha"].double().numpy()[0], axis=0)       # [T, H, dk]
+    S0 = d["S0"].double().numpy()[0]                                 # [H, dk, dv]
+    for h in range(w.H):
+        S_seq = np.exp(G[:, h, :, None]) * S0[h][None]
+        assert_close(np32(out[0, :, h]), _closed_form_out(S_seq, q[:, h]), tol, "out h%d" % h)
+        assert_close(np32(Sf[0, h]), S_seq[-1], tol, "S_final h%d" % h)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T", [100, 128])
+def test_no_decay_unit_beta_one_hot_keys_overwrite_rows(dtype, T):
+    """alpha = 1 (DeltaNet) and beta = 1 with one-hot keys k_t = e_{p(t)}: each update
+    (I - k k^T) S + k v^T replaces row p(t) of the state by v_t, so S_t is S0 with the rows
+    p(1..t) overwritten (the delta rule of Kimi Linear, section 3.1, at its fixed point)."""
+    w = K.Workload("overwrite", B=1, T=T, H=2, dtype=dtype, s0_std=0.5)
+    d = K.make_prefill(w, seed=22)
+    dt = K.to_dtype(dtype)
+    gen = torch.Generator().manual_seed(22)
+    k = torch.zeros(1, T, w.H, 128)
+    perms = [torch.randperm(128, generator=gen)[:T] for _ in range(w.H)]
+    for h in range(w.H):
+        k[0, torch.arange(T), h, perms[h]] = 1.0
+    d["k"] = k.to(dt)
+    d["log_alpha"] = torch.zeros_like(d["log_alpha"])
+    d["beta"] = torch.ones_like(d["beta"])
+    g = to_device(d, DEV)
+    out, Sf = kda.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], S0=g["S0"])
+    assert kda.workspace_status(kda.chunk_fwd.last_workspace) == kda.KDA_OK
+    tol = TOL[dt]
+    q = d["q"].double().numpy()[0]
+    v = d["v"].double().numpy()[0]
+    for h in range(w.H):
+        S = d["S0"].double().numpy()[0, h].copy()
+        S_seq = np.empty((T, 128, 128))
+        for t in range(T):
+            S[int(perms[h][t])] = v[t, h]
+            S_seq[t] = S
+        assert_close(np32(out[0, :, h]), _closed_form_out(S_seq, q[:, h]), tol, "out h%d" % h)
+        assert_close(np32(Sf[0, h]), S, tol, "S_final h%d" % h)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_no_decay_is_deltanet(dtype):
+    """log alpha = 0: the per-chunk decay factors are all 1 and the path computes DeltaNet;
+    checked against the oracle on random inputs with a ragged tail."""
+    w = K.Workload("deltanet", B=2, T=150, H=2, dtype=dtype, s0_std=0.1)
+    d = K.make_prefill(w, seed=23)
+    d["log_alpha"] = torch.zeros_like(d["log_alpha"])
+    _run_check(d, TOL[K.to_dtype(dtype)])
