@@ -92,3 +92,88 @@ def decode_step(S, q, k, v, log_alpha, beta):
     S_new = Sp + k[..., :, None] * u[..., None, :]
     o = np.einsum("nhi,nhij->nhj", q, Sp) + np.einsum("nhi,nhi->nh", q, k)[..., None] * u
     return o, S_new
+
+
+def _chunk_backward(S, dSn, dO, q, k, v, la, be):
+    """Gradients through one chunk of the chunk form above, given the state S entering it, the
+    gradient dSn reaching the state leaving it and the gradient dO of its outputs. Reverse-mode
+    chain rule through the chunk-form lines, last line first. Returns (dq, dk, dv, dla, dbe, dS)
+    with dS the gradient reaching S."""
+    L = q.shape[0]
+    g = np.cumsum(la, axis=0)
+    E = np.exp(g)
+    Kt, Kh, Qt = k * E, k / E, q * E
+    Kend = k * np.exp(g[L - 1][None, :] - g)
+    gam = np.exp(g[L - 1])
+    Pm = Kt @ Kh.T
+    Tm = np.linalg.inv(np.eye(L) + np.tril(be[:, None] * Pm, -1))
+    Tb = Tm * be[None, :]
+    R = v - Kt @ S
+    U = Tb @ R
+    Mm = np.tril(Qt @ Kh.T)
+    # S_next = Diag(gam) S + Kend^T U ;  O = Qt S + Mm U
+    dU = Mm.T @ dO + Kend @ dSn
+    dMm = np.tril(dO @ U.T)
+    dQt = dO @ S.T + dMm @ Kh
+    dKh = dMm.T @ Qt
+    dKend = U @ dSn.T
+    dgam = np.sum(dSn * S, axis=1)
+    # U = Tb R,  R = V - Kt S
+    dR = Tb.T @ dU
+    dTb = dU @ R.T
+    dS = gam[:, None] * dSn + Qt.T @ dO - Kt.T @ dR
+    dv = dR
+    dKt = -dR @ S.T
+    # Tb = Tm diag(beta),  Tm = (I + A)^{-1},  A = StrictLower(diag(beta) Kt Kh^T)
+    dbe = np.sum(dTb * Tm, axis=0)
+    dTm = dTb * be[None, :]
+    dA = np.tril(-Tm.T @ dTm @ Tm.T, -1)
+    dbe += np.sum(dA * Pm, axis=1)
+    dPm = be[:, None] * dA
+    dKt += dPm @ Kh
+    dKh += dPm.T @ Kt
+    # back to the raw inputs through the decay scalings and g = cumsum(log_alpha)
+    dq = dQt * E
+    dk = dKt * E + dKh / E + dKend * np.exp(g[L - 1][None, :] - g)
+    dg = dQt * Qt + dKt * Kt - dKh * Kh - dKend * Kend
+    dg[L - 1] += np.sum(dKend * Kend, axis=0) + dgam * gam
+    dla = np.cumsum(dg[::-1], axis=0)[::-1]
+    return dq, dk, dv, dla, dbe, dS
+
+
+def backward(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens=None, chunk=64):
+    """The gradients of ``backward.backward`` (same arguments and result), computed chunk by
+    chunk: a forward sweep keeps the state entering every chunk, then a reverse sweep over the
+    chunks carries the state gradient dS and differentiates each chunk on its own."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    la = np.asarray(log_alpha, dtype=np.float64)
+    be = np.asarray(beta, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is None:
+        spans = [(b, 0, T) for b in range(B)]
+    else:
+        cu = [int(x) for x in cu_seqlens]
+        spans = [(0, cu[n], cu[n + 1]) for n in range(len(cu) - 1)]
+    res = dict(dq=np.zeros_like(q), dk=np.zeros_like(k), dv=np.zeros_like(v), dlog_alpha=np.zeros_like(la),
+               dbeta=np.zeros_like(be), dS0=np.zeros((len(spans), H, dk, dv)))
+    for n, (b, t0, t1) in enumerate(spans):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if S0 is None else np.array(S0[n, h], dtype=np.float64)
+            bounds = [(s, min(s + chunk, t1)) for s in range(t0, t1, chunk)]
+            states = []
+            for s, e in bounds:
+                states.append(S)
+                S = _chunk(S, q[b, s:e, h], k[b, s:e, h], v[b, s:e, h], la[b, s:e, h], be[b, s:e, h])[1]
+            dS = np.zeros((dk, dv)) if dS_final is None else np.array(dS_final[n, h], dtype=np.float64)
+            for (s, e), Sc in zip(reversed(bounds), reversed(states)):
+                r = _chunk_backward(Sc, dS, dout[b, s:e, h], q[b, s:e, h], k[b, s:e, h], v[b, s:e, h],
+                                    la[b, s:e, h], be[b, s:e, h])
+                res["dq"][b, s:e, h], res["dk"][b, s:e, h], res["dv"][b, s:e, h] = r[0], r[1], r[2]
+                res["dlog_alpha"][b, s:e, h], res["dbeta"][b, s:e, h] = r[3], r[4]
+                dS = r[5]
+            res["dS0"][n, h] = dS
+    return res
