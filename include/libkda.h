@@ -129,6 +129,40 @@ kda_status_t kda_chunk_scan(const void *v, const float *S0, const int32_t *cu_se
                             int B, int T, int H, int N, int dk, int dv, kda_dtype_t out_dtype,
                             void *workspace, size_t workspace_bytes, void *stream);
 
+/* Backward pass of kda_chunk_fwd: the gradients of a scalar loss with respect to every
+ * input, given its gradients with respect to every output o_t and to the final states.
+ * The pages print no backward pass (training uses the chunk mode: lpnh.cn article, sec. 5);
+ * these are the chain rule through the recurrence above, computed through the same chunk
+ * form (chunk 64) in fp32 arithmetic on CUDA cores, for either input dtype.
+ *
+ *   q, k, v, log_alpha, beta, S0, cu_seqlens, B, T, H, N, dk, dv, dtype:
+ *              exactly as passed to kda_chunk_fwd (the forward is recomputed here).
+ *   dout       [B, T, H, dv]  dtype: dL/do_t for every token.
+ *   dS_final   [N, H, dk, dv] float32: dL/dS_final, or NULL for zero.
+ *   dq, dk_out, dlog_alpha  [B, T, H, dk] float32 (written)
+ *   dv_out     [B, T, H, dv]  float32 (written)
+ *   dbeta      [B, T, H]      float32 (written)
+ *   dS0        [N, H, dk, dv] float32 (written: dL/dS0), or NULL (not computed).
+ *   workspace  device buffer of kda_chunk_bwd_workspace_size(...) bytes (fp32 records
+ *              of the forward and of the reverse sweep: 224 KiB per chunk slot and head,
+ *              see kda_chunk_fwd_workspace_size for chunk slots). Its status word is
+ *              cleared by this call; cu_seqlens is checked on the device as for
+ *              kda_chunk_fwd.
+ * Gradient buffers must not overlap each other or the inputs. Every pointer except S0,
+ * dS_final and dS0 must be non-NULL when B * T > 0; alignment as for kda_chunk_fwd
+ * (16 bytes; 4 for beta and dbeta). Errors: KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED
+ * (dk, dv other than 128, or more chunk slots times heads than one launch grid holds),
+ * KDA_ERR_CUDA. */
+size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int N, int dk, int dv);
+kda_status_t kda_chunk_bwd(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const float *beta,
+                           const float *S0, const int32_t *cu_seqlens,
+                           const void *dout, const float *dS_final,
+                           float *dq, float *dk_out, float *dv_out,
+                           float *dlog_alpha, float *dbeta, float *dS0,
+                           int B, int T, int H, int N, int dk, int dv, kda_dtype_t dtype,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
 /* One decode step for N independent sequences (one token each), updating the
  * state in place: the recurrent ("fused_recurrent") mode the layer uses for
  * short queries and generation (lpnh.cn article, sec. 2 and 5); the per-step

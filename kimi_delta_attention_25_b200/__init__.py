@@ -35,7 +35,8 @@ _lib = None
 # Every entry point declared in include/libkda.h.
 EXPORTS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
            "kda_workspace_status", "kda_status_string", "kda_version", "kda_chunk_fwd_noalloc",
-           "kda_chunk_prep", "kda_chunk_scan", "kda_selftest_wait_timeout")
+           "kda_chunk_prep", "kda_chunk_scan", "kda_selftest_wait_timeout",
+           "kda_chunk_bwd_workspace_size", "kda_chunk_bwd")
 
 
 class KDAError(RuntimeError):
@@ -73,6 +74,10 @@ def load():
     lib.kda_chunk_scan.restype = I
     lib.kda_selftest_wait_timeout.argtypes = [P, Z, ctypes.c_longlong, P]
     lib.kda_selftest_wait_timeout.restype = I
+    lib.kda_chunk_bwd_workspace_size.argtypes = [I, I, I, I, I, I]
+    lib.kda_chunk_bwd_workspace_size.restype = Z
+    lib.kda_chunk_bwd.argtypes = [P] * 15 + [I] * 7 + [P, Z, P]
+    lib.kda_chunk_bwd.restype = I
     _lib = lib
     return lib
 
@@ -176,6 +181,54 @@ def chunk_scan(v, workspace, S0=None, cu_seqlens=None, out=None, S_final=None, w
     if st != KDA_OK:
         raise KDAError(st, "kda_chunk_scan")
     return out, S_final
+
+
+def chunk_bwd_workspace_size(B, T, H, N, dk=128, dv=128) -> int:
+    return int(load().kda_chunk_bwd_workspace_size(B, T, H, N, dk, dv))
+
+
+def chunk_bwd(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens=None,
+              want_dS0=True, grads=None, workspace=None):
+    """``kda_chunk_bwd``: gradients of a loss with gradients ``dout`` (w.r.t. every output, dtype of
+    q) and ``dS_final`` (w.r.t. the final states, fp32 or None) through ``chunk_fwd`` with the same
+    inputs. Returns a dict of fp32 tensors dq, dk, dv, dlog_alpha, dbeta and dS0 (None unless
+    ``want_dS0``). ``grads`` may supply those tensors (same keys) to be written in place."""
+    lib = load()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = B if cu_seqlens is None else cu_seqlens.shape[0] - 1
+    dev = q.device
+    g = dict(grads) if grads is not None else {}
+    f32 = dict(dtype=torch.float32, device=dev)
+    g.setdefault("dq", torch.empty(B, T, H, dk, **f32))
+    g.setdefault("dk", torch.empty(B, T, H, dk, **f32))
+    g.setdefault("dv", torch.empty(B, T, H, dv, **f32))
+    g.setdefault("dlog_alpha", torch.empty(B, T, H, dk, **f32))
+    g.setdefault("dbeta", torch.empty(B, T, H, **f32))
+    if want_dS0:
+        g.setdefault("dS0", torch.empty(N, H, dk, dv, **f32))
+    else:
+        g["dS0"] = None
+    _need_cuda(q, k, v, log_alpha, beta, dout, S0, dS_final, cu_seqlens, *g.values())
+    if dout.dtype != q.dtype:
+        raise TypeError("dout must have the dtype of q")
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    for key in ("dq", "dk", "dv", "dlog_alpha", "dbeta", "dS0"):
+        if g[key] is not None and g[key].dtype != torch.float32:
+            raise TypeError("%s must be float32" % key)
+    ws_bytes = lib.kda_chunk_bwd_workspace_size(B, T, H, N, dk, dv)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    st = lib.kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                           _ptr(cu_seqlens), _ptr(dout), _ptr(dS_final), _ptr(g["dq"]), _ptr(g["dk"]),
+                           _ptr(g["dv"]), _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]), _ptr(g["dS0"]),
+                           B, T, H, N, dk, dv, _dtype_code(q), _ptr(workspace), workspace.numel(),
+                           _stream(dev))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_bwd")
+    chunk_bwd.last_workspace = workspace
+    return g
 
 
 def selftest_wait_timeout(workspace: torch.Tensor, budget_cycles: int) -> None:

@@ -155,6 +155,78 @@ kda_status_t kda_chunk_scan(const void *v, const float *S0, const int32_t *cu_se
                                       (cudaStream_t)stream));
 }
 
+size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int N, int dk, int dv)
+{
+    if (B < 0 || T < 0 || H <= 0 || N < 0 || dk != kHeadDim || dv != kHeadDim) return 0;
+    const size_t per = 2 * kBwdStateFloats + 3 * kBwdRowsFloats;      // S, dS'; R, U, Y
+    return kStatusBytes + (size_t)H * (size_t)prep_slots((long long)B * T, N) * per * sizeof(float);
+}
+
+kda_status_t kda_chunk_bwd(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const float *beta,
+                           const float *S0, const int32_t *cu_seqlens,
+                           const void *dout, const float *dS_final,
+                           float *dq, float *dk_out, float *dv_out,
+                           float *dlog_alpha, float *dbeta, float *dS0,
+                           int B, int T, int H, int N, int dk, int dv, kda_dtype_t dtype,
+                           void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || H <= 0 || N < 0) return KDA_ERR_INVALID_ARG;
+    if (dk != kHeadDim || dv != kHeadDim) return KDA_ERR_UNSUPPORTED;
+    if (cu_seqlens) {
+        if (B != 1 || !aligned(cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
+    } else if (N != B) {
+        return KDA_ERR_INVALID_ARG;
+    }
+    const long long total = (long long)B * T;
+    if (total > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    const long long n_slots = prep_slots(total, N);
+    if ((long long)H * n_slots > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    if (total > 0) {
+        if (!q || !k || !v || !log_alpha || !beta || !dout || !dq || !dk_out || !dv_out || !dlog_alpha || !dbeta)
+            return KDA_ERR_INVALID_ARG;
+        if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(log_alpha, 16) ||
+            !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk_out, 16) || !aligned(dv_out, 16) ||
+            !aligned(dlog_alpha, 16) || !aligned(beta, 4) || !aligned(dbeta, 4))
+            return KDA_ERR_INVALID_ARG;
+    }
+    if ((S0 && !aligned(S0, 16)) || (dS_final && !aligned(dS_final, 16)) || (dS0 && !aligned(dS0, 16)))
+        return KDA_ERR_INVALID_ARG;
+    const size_t need = kda_chunk_bwd_workspace_size(B, T, H, N, dk, dv);
+    if (!workspace || !aligned(workspace, 16) || workspace_bytes < need) return KDA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemsetAsync(workspace, 0, kStatusBytes, st) != cudaSuccess) return KDA_ERR_CUDA;
+    if (N == 0) return KDA_OK;
+
+    // records: S and dS' per (head, slot), then R, U, Y
+    float *base = (float *)((unsigned char *)workspace + kStatusBytes);
+    const size_t hs = (size_t)H * (size_t)n_slots;
+    float *ck_S = base;
+    float *ck_dS = ck_S + hs * kBwdStateFloats;
+    float *ck_R = ck_dS + hs * kBwdStateFloats;
+    float *ck_U = ck_R + hs * kBwdRowsFloats;
+    float *ck_Y = ck_U + hs * kBwdRowsFloats;
+
+    // 1. forward sweep with records (outputs not needed)
+    PrefillArgs a = prefill_args(q, k, v, log_alpha, beta, S0, cu_seqlens, nullptr, nullptr, B, T, H, N,
+                                 workspace, workspace_bytes);
+    a.ck_S = ck_S; a.ck_R = ck_R; a.ck_U = ck_U; a.n_slots = (int)n_slots;
+    cudaError_t e = launch_chunk_fp32(a, dtype, KDA_F32, st);
+    // 2. reverse scan of the state gradient; 3. per-chunk gradients
+    BwdArgs b;
+    b.q = q; b.k = k; b.v = v; b.dout = dout;
+    b.log_alpha = log_alpha; b.beta = beta; b.dS_final = dS_final;
+    b.cu_seqlens = cu_seqlens;
+    b.dq = dq; b.dk = dk_out; b.dv = dv_out; b.dlog_alpha = dlog_alpha; b.dbeta = dbeta; b.dS0 = dS0;
+    b.ck_S = ck_S; b.ck_R = ck_R; b.ck_U = ck_U; b.ck_dS = ck_dS; b.ck_Y = ck_Y;
+    b.B = B; b.T = T; b.H = H; b.N = N; b.n_slots = (int)n_slots;
+    b.status = (int32_t *)workspace;
+    if (e == cudaSuccess) e = launch_chunk_bwd_scan(b, dtype, st);
+    if (e == cudaSuccess) e = launch_chunk_bwd_local(b, dtype, st);
+    return map_cuda(e);
+}
+
 kda_status_t kda_decode_step(const void *q, const void *k, const void *v,
                              const float *log_alpha, const float *beta,
                              float *S_inout, void *out,

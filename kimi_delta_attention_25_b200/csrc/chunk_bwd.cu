@@ -1,0 +1,561 @@
+// chunk_bwd.cu -- backward pass of the chunked KDA prefill on CUDA cores, fp32 arithmetic.
+//
+// Forward chunk form (chunk C = 64; chunk-parallel prefill with a WY representation: KimiLinear
+// KDA/MLA tutorial (icman.com.cn), sec. 3 and 6; the algebra is derived from the recurrence of
+// sec. 2 and 5). For a chunk of L <= C tokens entering with state S, per key channel c,
+//   g_r = sum_{j<=r} log_alpha_j,  E = e^g,  Kt = K E,  Kh = K / E,  Qt = Q E,  gamma = E_{L-1},
+//   Ke = Kh gamma,  A = StrictLower(diag(beta) Kt Kh^T),  M = tril(Qt Kh^T),
+//   R = V - Kt S,  U = (I + A)^{-1} diag(beta) R,  O = Qt S + M U,  S' = Diag(gamma) S + Ke^T U.
+// The pages give no backward pass; the gradients are the chain rule through these lines. With dO
+// the output gradient and dS' the gradient reaching the state that leaves the chunk:
+//   dU  = M^T dO + Ke dS'                Y = (I + A)^{-T} dU   (back substitution)
+//   dV  = diag(beta) Y                   dS = Diag(gamma) dS' + Qt^T dO - Kt^T dV
+// and, with every sum over the value channels gathered into dense products,
+//   dM  = tril(dO U^T)                   dA = -StrictLower(Y U^T)     dP = diag(beta) dA
+//   dQt = dO S^T + dM Kh                 dKt = -diag(beta) Y S^T + dP Kh
+//   dKh = dM^T Qt + dP^T Kt              dKe = U dS'^T                dgamma = rowsum(dS' * S)
+//   dbeta_r = sum_v R_rv Y_rv + sum_{i<r} dA_ri (Kt Kh^T)_ri
+//   dq = dQt E,  dk = dKt E + dKh / E + dKe gamma / E,
+//   dg = dQt Qt + dKt Kt - dKh Kh - dKe Ke,  plus (sum_r dKe Ke + dgamma gamma) on the last row,
+//   dlog_alpha = reverse cumulative sum of dg over the chunk's rows.
+//
+// Three launches (the host calls them in order on one stream):
+//  1. the fp32 forward kernel (chunk_fp32.cu) with records on: the state entering every chunk and
+//     each chunk's R and U, per (head, chunk slot);
+//  2. chunk_bwd_scan_kernel: the state gradient, chunk by chunk from the end of each sequence
+//     (one CTA per (sequence, head, 32 value columns); the columns are independent). It writes dV,
+//     dS0, Y and the gradient dS' reaching the end of every chunk;
+//  3. chunk_bwd_local_kernel: everything else, one CTA per (chunk slot, head), no chunk-to-chunk
+//     dependence (data-parallel over the whole grid).
+// Rows past a chunk's end are zero-filled (log_alpha = 0, k = q = v = dO = 0), which leaves every
+// gradient of the real rows unchanged.
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int C = kChunk;
+constexpr int DK = kHeadDim;
+constexpr int DVB = 32;          // value columns per block
+constexpr int LD = DK + 1;       // padded row stride of the 64 x 128 operand tiles
+constexpr int LDC = C + 1;       // padded row stride of the 64 x 64 tiles
+constexpr int LDV = DVB + 1;     // padded row stride of the 32-column blocks
+
+// ------------------------------------------------------------------------------------------
+// 2. reverse scan of the state gradient
+// ------------------------------------------------------------------------------------------
+constexpr int NT_SCAN = 256;
+
+struct ScanSmem {
+    float Kt[C * LD];
+    float Kh[C * LD];
+    float Qt[C * LD];
+    float Ke[C * LD];
+    float dS[DK * DVB];
+    float A[C * LDC];
+    float M[C * LDC];
+    float dO[C * DVB];
+    float dU[C * DVB];
+    float Y[C * DVB];
+    float gam[DK];
+    float beta[C];
+};
+
+template <typename T>
+__global__ void __launch_bounds__(NT_SCAN, 1)
+chunk_bwd_scan_kernel(BwdArgs a)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    ScanSmem &sm = *reinterpret_cast<ScanSmem *>(smem_raw);
+    const int tid = threadIdx.x;
+    const int j0 = blockIdx.x * DVB;
+    const int h = blockIdx.y;
+    const int n = blockIdx.z;
+    const int H = a.H;
+    const T *q = (const T *)a.q;
+    const T *k = (const T *)a.k;
+    const T *dout = (const T *)a.dout;
+
+    int64_t t0, t1;
+    if (!sequence_span(a.cu_seqlens, n, a.N, a.T, &t0, &t1, a.status)) return;
+
+    const size_t sbase = ((size_t)n * H + h) * DK * DK;
+    for (int idx = tid; idx < DK * DVB; idx += NT_SCAN) {
+        const int c = idx / DVB, j = idx % DVB;
+        sm.dS[idx] = a.dS_final ? a.dS_final[sbase + (size_t)c * DK + j0 + j] : 0.f;
+    }
+
+    const int64_t n_chunks = (t1 - t0 + C - 1) / C;
+    for (int64_t ci = n_chunks - 1; ci >= 0; --ci) {
+        const int64_t s = t0 + ci * C;
+        const int L = (t1 - s < C) ? (int)(t1 - s) : C;
+        const size_t rec = (size_t)h * a.n_slots + (size_t)chunk_slot(s, n);
+        __syncthreads();
+        // ---- load the chunk (k -> Kt, q -> Qt, log_alpha -> Kh, dO block) and record dS'
+        for (int idx = tid; idx < C * DK; idx += NT_SCAN) {
+            const int r = idx / DK, c = idx % DK;
+            float kk = 0.f, qq = 0.f, la = 0.f;
+            if (r < L) {
+                const size_t off = ((size_t)(s + r) * H + h) * DK + c;
+                kk = to_f32(k[off]);
+                qq = to_f32(q[off]);
+                la = a.log_alpha[off];
+            }
+            sm.Kt[r * LD + c] = kk;
+            sm.Qt[r * LD + c] = qq;
+            sm.Kh[r * LD + c] = la;
+        }
+        for (int idx = tid; idx < C * DVB; idx += NT_SCAN) {
+            const int r = idx / DVB, j = idx % DVB;
+            sm.dO[idx] = (r < L) ? to_f32(dout[((size_t)(s + r) * H + h) * DK + j0 + j]) : 0.f;
+        }
+        if (tid < C) sm.beta[tid] = (tid < L) ? a.beta[(size_t)(s + tid) * H + h] : 0.f;
+        {
+            float *dst = a.ck_dS + rec * kBwdStateFloats;
+            for (int idx = tid; idx < DK * DVB; idx += NT_SCAN) {
+                const int c = idx / DVB, j = idx % DVB;
+                dst[(size_t)c * DK + j0 + j] = sm.dS[idx];
+            }
+        }
+        __syncthreads();
+
+        // ---- cumulative log-decay and the decay-scaled operands (one thread per key channel)
+        if (tid < DK) {
+            const int c = tid;
+            float g = 0.f;
+            for (int r = 0; r < C; ++r) { g += sm.Kh[r * LD + c]; sm.Kh[r * LD + c] = g; }
+            const float gl = g;
+            sm.gam[c] = expf(gl);
+            for (int r = 0; r < C; ++r) {
+                const float gr = sm.Kh[r * LD + c];
+                const float kk = sm.Kt[r * LD + c];
+                const float e = expf(gr);
+                sm.Kt[r * LD + c] = kk * e;
+                sm.Qt[r * LD + c] *= e;
+                sm.Kh[r * LD + c] = kk * expf(-gr);
+                sm.Ke[r * LD + c] = kk * expf(gl - gr);
+            }
+        }
+        __syncthreads();
+
+        // ---- A = StrictLower(diag(beta) Kt Kh^T), M = tril(Qt Kh^T); 4x4 register tiles
+        {
+            const int rb = tid / 16, ib = tid % 16;
+            float accA[4][4], accM[4][4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) { accA[x][y] = 0.f; accM[x][y] = 0.f; }
+            if (ib <= rb) {
+                for (int c = 0; c < DK; ++c) {
+                    float kt[4], qt[4], kh[4];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        kt[x] = sm.Kt[(4 * rb + x) * LD + c];
+                        qt[x] = sm.Qt[(4 * rb + x) * LD + c];
+                        kh[x] = sm.Kh[(4 * ib + x) * LD + c];
+                    }
+#pragma unroll
+                    for (int x = 0; x < 4; ++x)
+#pragma unroll
+                        for (int y = 0; y < 4; ++y) {
+                            accA[x][y] += kt[x] * kh[y];
+                            accM[x][y] += qt[x] * kh[y];
+                        }
+                }
+            }
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    const int r = 4 * rb + x, i = 4 * ib + y;
+                    sm.A[r * LDC + i] = (i < r) ? sm.beta[r] * accA[x][y] : 0.f;
+                    sm.M[r * LDC + i] = (i <= r) ? accM[x][y] : 0.f;
+                }
+        }
+        __syncthreads();
+
+        // ---- dU = M^T dO + Ke dS': thread -> row r, 8 columns
+        {
+            const int r = tid / 4, jg = (tid % 4) * 8;
+            float acc[8];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) acc[x] = 0.f;
+            for (int i = r; i < C; ++i) {
+                const float m = sm.M[i * LDC + r];
+#pragma unroll
+                for (int x = 0; x < 8; ++x) acc[x] += m * sm.dO[i * DVB + jg + x];
+            }
+            for (int c = 0; c < DK; ++c) {
+                const float ke = sm.Ke[r * LD + c];
+#pragma unroll
+                for (int x = 0; x < 8; ++x) acc[x] += ke * sm.dS[c * DVB + jg + x];
+            }
+#pragma unroll
+            for (int x = 0; x < 8; ++x) sm.dU[r * DVB + jg + x] = acc[x];
+        }
+        __syncthreads();
+
+        // ---- Y = (I + A)^{-T} dU by back substitution: Y_r = dU_r - sum_{i>r} A_ir Y_i.
+        //      Warp w owns columns 4w..4w+3; eight lanes per column split the sum.
+        {
+            const int warp = tid >> 5, lane = tid & 31;
+            const int j = warp * 4 + lane / 8, p = lane % 8;
+            for (int r = C - 1; r >= 0; --r) {
+                float part = 0.f;
+                for (int i = r + 1 + p; i < C; i += 8) part += sm.A[i * LDC + r] * sm.Y[i * DVB + j];
+                part += __shfl_xor_sync(0xffffffffu, part, 1);
+                part += __shfl_xor_sync(0xffffffffu, part, 2);
+                part += __shfl_xor_sync(0xffffffffu, part, 4);
+                if (p == 0) sm.Y[r * DVB + j] = sm.dU[r * DVB + j] - part;
+                __syncwarp();
+            }
+        }
+        __syncthreads();
+
+        // ---- dV = diag(beta) Y -> dv (rows < L); Y -> record (all rows)
+        {
+            float *ydst = a.ck_Y + rec * kBwdRowsFloats;
+            for (int idx = tid; idx < C * DVB; idx += NT_SCAN) {
+                const int r = idx / DVB, j = idx % DVB;
+                const float y = sm.Y[idx];
+                ydst[(size_t)r * DK + j0 + j] = y;
+                if (r < L) a.dv[((size_t)(s + r) * H + h) * DK + j0 + j] = sm.beta[r] * y;
+            }
+        }
+
+        // ---- dS <- Diag(gamma) dS' + Qt^T dO - Kt^T diag(beta) Y: thread -> key channel c, 16 columns
+        {
+            const int c = tid / 2, jh = (tid % 2) * 16;
+            float acc[16];
+            const float gm = sm.gam[c];
+#pragma unroll
+            for (int x = 0; x < 16; ++x) acc[x] = gm * sm.dS[c * DVB + jh + x];
+            for (int r = 0; r < C; ++r) {
+                const float qt = sm.Qt[r * LD + c];
+                const float kb = sm.Kt[r * LD + c] * sm.beta[r];
+#pragma unroll
+                for (int x = 0; x < 16; ++x) acc[x] += qt * sm.dO[r * DVB + jh + x] - kb * sm.Y[r * DVB + jh + x];
+            }
+#pragma unroll
+            for (int x = 0; x < 16; ++x) sm.dS[c * DVB + jh + x] = acc[x];
+        }
+    }
+    __syncthreads();
+    if (a.dS0) {
+        for (int idx = tid; idx < DK * DVB; idx += NT_SCAN) {
+            const int c = idx / DVB, j = idx % DVB;
+            a.dS0[sbase + (size_t)c * DK + j0 + j] = sm.dS[idx];
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// 3. per-chunk gradients (data-parallel)
+// ------------------------------------------------------------------------------------------
+constexpr int NT_LOC = 512;
+
+struct LocalSmem {
+    float Kt[C * LD];
+    float Kh[C * LD];        // after the last products: dg
+    float Qt[C * LD];
+    float E[C * LD];
+    // one 32-column block of the value axis at a time; after the loop: dM and dP (64 x LDC each)
+    float S[DK * LDV];
+    float dSn[DK * LDV];
+    float dO[C * LDV];
+    float U[C * LDV];
+    float Y[C * LDV];
+    float R[C * LDV];
+    float P[C * LDC];        // Kt Kh^T (strictly lower part used)
+    float beta[C];
+    float gam[DK];
+    float dgam[DK];
+    float dgl[DK];
+    float ry[C];
+};
+
+template <typename T>
+__global__ void __launch_bounds__(NT_LOC, 1)
+chunk_bwd_local_kernel(BwdArgs a)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    LocalSmem &sm = *reinterpret_cast<LocalSmem *>(smem_raw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = a.H;
+    const int h = (int)(blockIdx.x % (unsigned)H), slot = (int)(blockIdx.x / (unsigned)H);
+    int n, L;
+    int64_t s;
+    if (!slot_to_chunk(a.cu_seqlens, a.N, a.T, slot, &n, &s, &L)) return;
+    const size_t rec = (size_t)h * a.n_slots + (size_t)slot;
+    const T *q = (const T *)a.q;
+    const T *k = (const T *)a.k;
+    const T *dout = (const T *)a.dout;
+
+    // ---- load q, k, log_alpha (zero past L), beta
+    for (int idx = tid; idx < C * DK; idx += NT_LOC) {
+        const int r = idx / DK, c = idx % DK;
+        float kk = 0.f, qq = 0.f, la = 0.f;
+        if (r < L) {
+            const size_t off = ((size_t)(s + r) * H + h) * DK + c;
+            kk = to_f32(k[off]);
+            qq = to_f32(q[off]);
+            la = a.log_alpha[off];
+        }
+        sm.Kt[r * LD + c] = kk;
+        sm.Qt[r * LD + c] = qq;
+        sm.E[r * LD + c] = la;
+    }
+    if (tid < C) sm.beta[tid] = (tid < L) ? a.beta[(size_t)(s + tid) * H + h] : 0.f;
+    if (tid < DK) { sm.dgam[tid] = 0.f; sm.dgl[tid] = 0.f; }
+    if (tid < C) sm.ry[tid] = 0.f;
+    __syncthreads();
+    if (tid < DK) {
+        const int c = tid;
+        float g = 0.f;
+        for (int r = 0; r < C; ++r) {
+            g += sm.E[r * LD + c];
+            const float e = expf(g), kk = sm.Kt[r * LD + c];
+            sm.E[r * LD + c] = e;
+            sm.Kt[r * LD + c] = kk * e;
+            sm.Kh[r * LD + c] = kk * expf(-g);
+            sm.Qt[r * LD + c] *= e;
+        }
+        sm.gam[c] = expf(g);
+    }
+    __syncthreads();
+
+    // thread tile: rows 4 rb .. 4 rb + 3 (rb = warp), key columns lane + 32 x, token columns lane + 32 x
+    const int rb = warp, cb = lane;
+    // ---- P = Kt Kh^T, strictly lower part
+    {
+        float acc[4][2];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) { acc[x][0] = 0.f; acc[x][1] = 0.f; }
+        for (int c = 0; c < DK; ++c) {
+            float kt[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) kt[x] = sm.Kt[(4 * rb + x) * LD + c];
+            const float kh0 = sm.Kh[cb * LD + c], kh1 = sm.Kh[(cb + 32) * LD + c];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) { acc[x][0] += kt[x] * kh0; acc[x][1] += kt[x] * kh1; }
+        }
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+            for (int y = 0; y < 2; ++y) {
+                const int r = 4 * rb + x, i = cb + 32 * y;
+                sm.P[r * LDC + i] = (i < r) ? acc[x][y] : 0.f;
+            }
+    }
+
+    // ---- sums over the value axis, 32 columns at a time
+    float aQ[4][4], aY[4][4], aE[4][4], aM[4][2], aA[4][2];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+#pragma unroll
+        for (int y = 0; y < 4; ++y) { aQ[x][y] = 0.f; aY[x][y] = 0.f; aE[x][y] = 0.f; }
+        aM[x][0] = aM[x][1] = aA[x][0] = aA[x][1] = 0.f;
+    }
+    const float *gS = a.ck_S + rec * kBwdStateFloats;
+    const float *gdS = a.ck_dS + rec * kBwdStateFloats;
+    const float *gU = a.ck_U + rec * kBwdRowsFloats;
+    const float *gY = a.ck_Y + rec * kBwdRowsFloats;
+    const float *gR = a.ck_R + rec * kBwdRowsFloats;
+    float dgam_acc = 0.f, ry_acc = 0.f;
+    for (int j0 = 0; j0 < DK; j0 += DVB) {
+        __syncthreads();
+        for (int idx = tid; idx < DK * DVB; idx += NT_LOC) {
+            const int c = idx / DVB, v = idx % DVB;
+            sm.S[c * LDV + v] = gS[(size_t)c * DK + j0 + v];
+            sm.dSn[c * LDV + v] = gdS[(size_t)c * DK + j0 + v];
+        }
+        for (int idx = tid; idx < C * DVB; idx += NT_LOC) {
+            const int r = idx / DVB, v = idx % DVB;
+            sm.U[r * LDV + v] = gU[(size_t)r * DK + j0 + v];
+            sm.Y[r * LDV + v] = gY[(size_t)r * DK + j0 + v];
+            sm.R[r * LDV + v] = gR[(size_t)r * DK + j0 + v];
+            sm.dO[r * LDV + v] = (r < L) ? to_f32(dout[((size_t)(s + r) * H + h) * DK + j0 + v]) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int v = 0; v < DVB; ++v) {
+            float o[4], y[4], u[4], sv[4], dv[4], ui[2];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                o[x] = sm.dO[(4 * rb + x) * LDV + v];
+                y[x] = sm.Y[(4 * rb + x) * LDV + v];
+                u[x] = sm.U[(4 * rb + x) * LDV + v];
+                sv[x] = sm.S[(cb + 32 * x) * LDV + v];
+                dv[x] = sm.dSn[(cb + 32 * x) * LDV + v];
+            }
+            ui[0] = sm.U[cb * LDV + v];
+            ui[1] = sm.U[(cb + 32) * LDV + v];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+#pragma unroll
+                for (int z = 0; z < 4; ++z) {
+                    aQ[x][z] += o[x] * sv[z];
+                    aY[x][z] += y[x] * sv[z];
+                    aE[x][z] += u[x] * dv[z];
+                }
+#pragma unroll
+                for (int z = 0; z < 2; ++z) {
+                    aM[x][z] += o[x] * ui[z];
+                    aA[x][z] += y[x] * ui[z];
+                }
+            }
+        }
+        if (tid < DK) {
+            for (int v = 0; v < DVB; ++v) dgam_acc += sm.dSn[tid * LDV + v] * sm.S[tid * LDV + v];
+        } else if (tid < DK + C) {
+            const int r = tid - DK;
+            for (int v = 0; v < DVB; ++v) ry_acc += sm.R[r * LDV + v] * sm.Y[r * LDV + v];
+        }
+    }
+    __syncthreads();                                   // the value blocks are dead from here on
+    float *dM = sm.S;                                  // 64 x LDC, aliases the staging area
+    float *dP = sm.S + C * LDC;
+    if (tid < DK) sm.dgam[tid] = dgam_acc;
+    else if (tid < DK + C) sm.ry[tid - DK] = ry_acc;
+    {
+        // dM = tril(dO U^T); dA = -StrictLower(Y U^T); dP = diag(beta) dA; dbeta's A part
+        float part[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int r = 4 * rb + x;
+            part[x] = 0.f;
+#pragma unroll
+            for (int z = 0; z < 2; ++z) {
+                const int i = cb + 32 * z;
+                const float da = (i < r) ? -aA[x][z] : 0.f;
+                dM[r * LDC + i] = (i <= r) ? aM[x][z] : 0.f;
+                dP[r * LDC + i] = sm.beta[r] * da;
+                part[x] += da * sm.P[r * LDC + i];
+            }
+        }
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) part[x] += __shfl_xor_sync(0xffffffffu, part[x], m);
+        }
+        __syncthreads();                               // ry, dM, dP complete
+        if (lane == 0) {
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const int r = 4 * rb + x;
+                if (r < L) a.dbeta[(size_t)(s + r) * H + h] = sm.ry[r] + part[x];
+            }
+        }
+    }
+
+    // ---- dQt, dKt, dKh for the thread's 4 x 4 tile, then dq, dk and dg
+    float dg[4][4], colp[4];
+#pragma unroll
+    for (int z = 0; z < 4; ++z) colp[z] = 0.f;
+    {
+        float dQ[4][4], dKt[4][4], dKh[4][4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const float br = sm.beta[4 * rb + x];
+#pragma unroll
+            for (int z = 0; z < 4; ++z) { dQ[x][z] = aQ[x][z]; dKt[x][z] = -br * aY[x][z]; dKh[x][z] = 0.f; }
+        }
+        for (int i = 0; i < C; ++i) {
+            float kh[4], qt[4], kt[4];
+#pragma unroll
+            for (int z = 0; z < 4; ++z) {
+                kh[z] = sm.Kh[i * LD + cb + 32 * z];
+                qt[z] = sm.Qt[i * LD + cb + 32 * z];
+                kt[z] = sm.Kt[i * LD + cb + 32 * z];
+            }
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const int r = 4 * rb + x;
+                const float m_ri = dM[r * LDC + i], p_ri = dP[r * LDC + i];     // row r: dQt, dKt
+                const float m_ir = dM[i * LDC + r], p_ir = dP[i * LDC + r];     // column r: dKh
+#pragma unroll
+                for (int z = 0; z < 4; ++z) {
+                    dQ[x][z] += m_ri * kh[z];
+                    dKt[x][z] += p_ri * kh[z];
+                    dKh[x][z] += m_ir * qt[z] + p_ir * kt[z];
+                }
+            }
+        }
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int r = 4 * rb + x;
+#pragma unroll
+            for (int z = 0; z < 4; ++z) {
+                const int c = cb + 32 * z;
+                const float e = sm.E[r * LD + c], gm = sm.gam[c];
+                const float ktv = sm.Kt[r * LD + c], khv = sm.Kh[r * LD + c], qtv = sm.Qt[r * LD + c];
+                const float dke = aE[x][z], ke = khv * gm;
+                if (r < L) {
+                    const size_t off = ((size_t)(s + r) * H + h) * DK + c;
+                    a.dq[off] = dQ[x][z] * e;
+                    a.dk[off] = dKt[x][z] * e + (dKh[x][z] + dke * gm) / e;
+                }
+                dg[x][z] = dQ[x][z] * qtv + dKt[x][z] * ktv - dKh[x][z] * khv - dke * ke;
+                colp[z] += dke * ke;
+            }
+        }
+    }
+    __syncthreads();                                   // Kh is free: it takes dg
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int z = 0; z < 4; ++z) sm.Kh[(4 * rb + x) * LD + cb + 32 * z] = dg[x][z];
+#pragma unroll
+    for (int z = 0; z < 4; ++z) atomicAdd(&sm.dgl[cb + 32 * z], colp[z]);
+    __syncthreads();
+    // ---- dlog_alpha: reverse cumulative sum over rows, the last row also carrying the terms of
+    //      g_{L-1} (through Ke and gamma)
+    if (tid < DK) {
+        const int c = tid;
+        float run = sm.dgl[c] + sm.dgam[c] * sm.gam[c];
+        for (int r = C - 1; r >= 0; --r) {
+            run += sm.Kh[r * LD + c];
+            if (r < L) a.dlog_alpha[((size_t)(s + r) * H + h) * DK + c] = run;
+        }
+    }
+}
+
+template <typename T>
+cudaError_t launch_scan_typed(const BwdArgs &a, cudaStream_t stream)
+{
+    const size_t smem = sizeof(ScanSmem);
+    cudaError_t e = cudaFuncSetAttribute(chunk_bwd_scan_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    chunk_bwd_scan_kernel<T><<<dim3(DK / DVB, a.H, a.N), NT_SCAN, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_local_typed(const BwdArgs &a, cudaStream_t stream)
+{
+    const size_t smem = sizeof(LocalSmem);
+    cudaError_t e = cudaFuncSetAttribute(chunk_bwd_local_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const long long blocks = (long long)a.n_slots * a.H;
+    chunk_bwd_local_kernel<T><<<(unsigned)blocks, NT_LOC, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_bwd_scan(const BwdArgs &a, kda_dtype_t dtype, cudaStream_t stream)
+{
+    if (a.N == 0) return cudaSuccess;
+    return dtype == KDA_BF16 ? launch_scan_typed<__nv_bfloat16>(a, stream) : launch_scan_typed<float>(a, stream);
+}
+
+cudaError_t launch_chunk_bwd_local(const BwdArgs &a, kda_dtype_t dtype, cudaStream_t stream)
+{
+    if (a.N == 0 || a.n_slots == 0) return cudaSuccess;
+    return dtype == KDA_BF16 ? launch_local_typed<__nv_bfloat16>(a, stream) : launch_local_typed<float>(a, stream);
+}
+
+}  // namespace kda

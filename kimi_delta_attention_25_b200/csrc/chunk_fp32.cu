@@ -17,6 +17,9 @@
 // Work split: one CTA per (sequence, head, 32-column block of d_v); the columns of S evolve
 // independently, so blocks never communicate. Chunks are processed in order; everything stays
 // in shared memory (about 198 KiB).
+//
+// For the backward pass the same kernel also records, per (head, chunk slot), the state entering
+// each chunk and the chunk's R = V - Kt S and U (PrefillArgs::ck_*), and may skip the outputs.
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -91,6 +94,15 @@ chunk_fp32_kernel(PrefillArgs a)
             sm.R[idx] = (r < L) ? to_f32(v[((size_t)(s + r) * H + h) * DK + j0 + j]) : 0.f;
         }
         if (tid < C) sm.beta[tid] = (tid < L) ? a.beta[(size_t)(s + tid) * H + h] : 0.f;
+        // backward records of this chunk: (head, chunk slot) blocks
+        const size_t rec = (size_t)h * a.n_slots + (size_t)chunk_slot(s, n);
+        if (a.ck_S) {
+            float *dst = a.ck_S + rec * kBwdStateFloats;
+            for (int idx = tid; idx < DK * DVB; idx += NT) {
+                const int c = idx / DVB, j = idx % DVB;
+                dst[(size_t)c * DK + j0 + j] = sm.S[idx];
+            }
+        }
         __syncthreads();
 
         // ---- cumulative log-decay and the decay-scaled operands (one thread per key channel)
@@ -159,6 +171,11 @@ chunk_fp32_kernel(PrefillArgs a)
                 for (int x = 0; x < 8; ++x) acc[x] += kt * sm.S[c * DVB + jg + x];
             }
             const float b = sm.beta[r];
+            if (a.ck_R) {
+                float *dst = a.ck_R + rec * kBwdRowsFloats + (size_t)r * DK + j0 + jg;
+#pragma unroll
+                for (int x = 0; x < 8; ++x) dst[x] = sm.R[r * DVB + jg + x] - acc[x];
+            }
 #pragma unroll
             for (int x = 0; x < 8; ++x) sm.R[r * DVB + jg + x] = b * (sm.R[r * DVB + jg + x] - acc[x]);
         }
@@ -180,9 +197,16 @@ chunk_fp32_kernel(PrefillArgs a)
             }
         }
         __syncthreads();
+        if (a.ck_U) {
+            float *dst = a.ck_U + rec * kBwdRowsFloats;
+            for (int idx = tid; idx < C * DVB; idx += NT) {
+                const int r = idx / DVB, j = idx % DVB;
+                dst[(size_t)r * DK + j0 + j] = sm.U[idx];
+            }
+        }
 
-        // ---- O = Qt S + M U  -> out (rows < L)
-        {
+        // ---- O = Qt S + M U  -> out (rows < L); skipped when only the records are wanted
+        if (out) {
             const int r = tid / 4, jg = (tid % 4) * 8;
             float acc[8];
 #pragma unroll

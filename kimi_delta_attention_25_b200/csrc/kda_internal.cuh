@@ -74,7 +74,52 @@ struct PrefillArgs {
     int32_t *status;      // device status word (workspace prefix)
     void *scratch;        // workspace after the status prefix
     size_t scratch_bytes;
+    // Backward-pass records written by the fp32 chunk kernel when non-null (one block per
+    // (head, chunk slot), see chunk_bwd.cu): the state entering each chunk (d_k x d_v) and the
+    // chunk's R = V - Kt S and U (64 x d_v each, rows past the chunk's end zero).
+    float *ck_S = nullptr, *ck_R = nullptr, *ck_U = nullptr;
+    int n_slots = 0;
 };
+
+// Backward-pass record sizes (floats) per (head, chunk slot).
+constexpr size_t kBwdStateFloats = (size_t)kHeadDim * kHeadDim;   // 128 x 128
+constexpr size_t kBwdRowsFloats = (size_t)kChunk * kHeadDim;       // 64 x 128
+
+// The chunk slot of a chunk starting at absolute token s in sequence n (unique per chunk, below
+// prep_slots(total_tokens, N)).
+__host__ __device__ inline long long chunk_slot(int64_t s, int n) { return s / kChunk + n; }
+
+// Inverse of chunk_slot: the sequence n, first token and length of chunk slot `slot`. Returns
+// false for a slot that no chunk uses, or when cu_seqlens is inconsistent (without flagging it:
+// the kernels that walk the sequences flag that).
+__device__ __forceinline__ bool slot_to_chunk(const int32_t *cu_seqlens, int N, int T, int slot,
+                                              int *n_out, int64_t *tok0, int *L)
+{
+    if (N <= 0) return false;
+    int lo = 0, hi = N - 1;                 // largest n with floor(first token of n / 64) + n <= slot
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        const int64_t st = cu_seqlens ? (int64_t)cu_seqlens[mid] : (int64_t)mid * T;
+        if (st / kChunk + mid <= slot) lo = mid; else hi = mid - 1;
+    }
+    const int n = lo;
+    int64_t s0, s1;
+    if (cu_seqlens) {
+        s0 = cu_seqlens[n];
+        s1 = cu_seqlens[n + 1];
+        if (s1 < s0 || s0 < 0 || s1 > T) return false;
+    } else {
+        s0 = (int64_t)n * T;
+        s1 = s0 + T;
+    }
+    const int64_t c = slot - (s0 / kChunk + n);
+    if (c < 0) return false;
+    *tok0 = s0 + c * kChunk;
+    if (*tok0 >= s1) return false;
+    *L = (s1 - *tok0 < kChunk) ? (int)(s1 - *tok0) : kChunk;
+    *n_out = n;
+    return true;
+}
 
 // CUDA-core fp32 chunk path (any input dtype; fp32 arithmetic throughout).
 cudaError_t launch_chunk_fp32(const PrefillArgs &a, kda_dtype_t dtype, kda_dtype_t out_dtype,
@@ -88,6 +133,20 @@ cudaError_t launch_chunk_tc(const PrefillArgs &a, kda_dtype_t out_dtype, cudaStr
 cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slots, cudaStream_t stream);
 cudaError_t launch_chunk_scan(const PrefillArgs &a, const unsigned char *ws, int n_slots,
                               kda_dtype_t out_dtype, cudaStream_t stream);
+
+// Backward pass (chunk_bwd.cu). Gradient pointers and the records of the forward kernel.
+struct BwdArgs {
+    const void *q, *k, *v, *dout;
+    const float *log_alpha, *beta, *dS_final;
+    const int32_t *cu_seqlens;
+    float *dq, *dk, *dv, *dlog_alpha, *dbeta, *dS0;
+    const float *ck_S, *ck_R, *ck_U;   // from the forward sweep
+    float *ck_dS, *ck_Y;               // from the reverse scan
+    int B, T, H, N, n_slots;
+    int32_t *status;
+};
+cudaError_t launch_chunk_bwd_scan(const BwdArgs &a, kda_dtype_t dtype, cudaStream_t stream);
+cudaError_t launch_chunk_bwd_local(const BwdArgs &a, kda_dtype_t dtype, cudaStream_t stream);
 
 // Decode step (memory-bound state update in place).
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,

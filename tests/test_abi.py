@@ -153,3 +153,33 @@ def test_selftest_host_checks(lib):
     assert f(P(FAKE + 8), 256, 1000, None) == kda.KDA_ERR_INVALID_ARG      # misaligned
     assert f(P(FAKE), 256, 0, None) == kda.KDA_ERR_INVALID_ARG
     assert f(P(FAKE), 256, 2000000001, None) == kda.KDA_ERR_INVALID_ARG
+
+
+def _bwd(lib, **kw):
+    P = ctypes.c_void_p
+    a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, S0=None, cu=None, do=FAKE, dSf=None,
+             dq=FAKE, dk_=FAKE, dv_=FAKE, dla=FAKE, dbe=FAKE, dS0=None,
+             B=1, T=64, H=2, N=1, dk=128, dv=128, dtype=1, ws=FAKE, wsb=256)
+    a.update(kw)
+    return lib.kda_chunk_bwd(*[P(a[x]) for x in ("q", "k", "v", "la", "beta", "S0", "cu", "do", "dSf", "dq",
+                                                 "dk_", "dv_", "dla", "dbe", "dS0")],
+                             a["B"], a["T"], a["H"], a["N"], a["dk"], a["dv"], a["dtype"], P(a["ws"]), a["wsb"],
+                             None)
+
+
+def test_backward_host_checks(lib):
+    need = kda.chunk_bwd_workspace_size(1, 64, 2, 1)
+    # 2 heads x (64 / 64 + 1 + 1) slots x (2 states + 3 row blocks) of fp32, after the status prefix
+    assert need == 256 + 2 * 3 * (2 * 128 * 128 + 3 * 64 * 128) * 4
+    assert kda.chunk_bwd_workspace_size(1, 64, 2, 1, dk=64) == 0
+    # the first failing check decides; none of these reaches a CUDA call
+    assert _bwd(lib, dk=64) == kda.KDA_ERR_UNSUPPORTED
+    assert _bwd(lib, dtype=7) == kda.KDA_ERR_INVALID_ARG
+    assert _bwd(lib, do=None) == kda.KDA_ERR_INVALID_ARG
+    assert _bwd(lib, dla=None) == kda.KDA_ERR_INVALID_ARG
+    assert _bwd(lib, dq=FAKE + 4) == kda.KDA_ERR_INVALID_ARG
+    assert _bwd(lib, dS0=FAKE + 8) == kda.KDA_ERR_INVALID_ARG
+    assert _bwd(lib, N=2) == kda.KDA_ERR_INVALID_ARG
+    assert _bwd(lib, B=2, N=2, cu=FAKE) == kda.KDA_ERR_INVALID_ARG
+    assert _bwd(lib) == kda.KDA_ERR_INVALID_ARG                           # workspace too small
+    assert _bwd(lib, ws=FAKE + 8, wsb=need) == kda.KDA_ERR_INVALID_ARG    # misaligned workspace
