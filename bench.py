@@ -53,6 +53,23 @@ CSRC = os.path.join(ROOT, "kimi_delta_attention_25_b200", "csrc")
 # useful tensor flops per token*head (chunk C): 6 d^2 (W.S, Q.S, Kend^T.U) + 5 C d (triangular
 # K K^T, Q K^T, T.(beta K), T.(beta V), M.U) + C^2 / 3 (triangular inverse)
 PREFILL_FLOPS_PER_TOKEN_HEAD = 6 * D * D + 5 * C * D + C * C // 3
+# backward (kda_chunk_bwd, fp32 arithmetic on CUDA cores): flops per (64-token chunk, head) that
+# each of its three kernels must do in this design, triangular products counted once
+# (TRI = a 64 x 64 triangle times 128 columns, FULL = 64 x 128 x 128, 2 flops per multiply-add):
+#   forward sweep: A, the solve for U (TRI each); Kt S, Ke^T U (FULL each)
+#   reverse scan:  A, M, M^T dO, the solve for Y (TRI); Ke dS', Qt^T dO, Kt^T dV (FULL)
+#   per chunk:     Kt Kh^T, dO U^T, Y U^T, dM Kh, dP Kh, dM^T Qt, dP^T Kt (TRI); dO S^T, Y S^T,
+#                  U dS'^T (FULL)
+BWD_TRI = C * C // 2 * D * 2
+BWD_FULL = C * D * D * 2
+BWD_FLOPS_PER_CHUNK_HEAD = {"bwd_forward_records": 2 * BWD_TRI + 2 * BWD_FULL,
+                            "bwd_scan": 4 * BWD_TRI + 3 * BWD_FULL,
+                            "bwd_local": 7 * BWD_TRI + 3 * BWD_FULL}
+# algorithmic HBM bytes per token*head: q, k, v, dout bf16 and log_alpha, beta read; dq, dk, dv,
+# dlog_alpha, dbeta fp32 written
+BWD_BYTES_PER_TOKEN_HEAD = 4 * D * 2 + D * 4 + 4 + 4 * D * 4 + 4
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz (max SM clock)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # decode: state read + written once per step
 DECODE_STATE_BYTES_PER_HEAD = 2 * D * D * 4
 DECODE_IO_BYTES_PER_HEAD = 3 * D * 2 + D * 4 + 4 + D * 4
@@ -330,6 +347,11 @@ def run_native(args):
     # ---- decode step
     dec = run_decode(kda, dev, pk, ws, local, args)
 
+    # ---- backward of the same prefill
+    del work
+    torch.cuda.empty_cache()
+    bwd = run_backward(kda, dev, pk, ws, local, args, d)
+
     del d, out
     torch.cuda.empty_cache()
     cpu = None
@@ -358,6 +380,7 @@ def run_native(args):
             "gpu_launches": args.steps * PREFILL_KERNELS_PER_STEP,
             "clocks": clk.summary(),
             "decode": dec,
+            "backward": bwd,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
@@ -417,10 +440,75 @@ def run_decode(kda, dev, pk, ws, local, args):
             "gpu_launches": nsteps, "clocks": clk.summary()}
 
 
+def run_backward(kda, dev, pk, ws, local, args, d):
+    """kda_chunk_bwd on the headline workload (gradients of every input for a random output
+    gradient and final-state gradient), its three kernels timed one by one with CUDA events."""
+    B, T, H = d["v"].shape[:3]
+    g = torch.Generator(device=dev).manual_seed(1234)
+    dout = torch.randn(B, T, H, D, generator=g, device=dev).to(torch.bfloat16)
+    dSf = torch.randn(B, H, D, D, generator=g, device=dev)
+    args_ = (d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], dout)
+    kw = dict(S0=d["S0"], dS_final=dSf)
+    grads = kda.chunk_bwd(*args_, **kw)
+    work = kda.chunk_bwd.last_workspace
+    torch.cuda.synchronize()
+    assert kda.workspace_status(work) == kda.KDA_OK
+    steps = max(1, min(args.steps, 3))
+    names = ("bwd_forward_records", "bwd_scan", "bwd_local")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+
+    def step(ev=None):
+        for p in range(3):
+            if ev is not None:
+                ev[p].record()
+            kda.chunk_bwd(*args_, **kw, grads=grads, workspace=work, phase=p)
+        if ev is not None:
+            ev[3].record()
+
+    with Clocks(local) as clk:
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        barrier(ws)
+        torch.cuda.synchronize()
+        t_s, t_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t_s.record()
+        for i in range(steps):
+            step(evs[i])
+        t_e.record()
+        torch.cuda.synchronize()
+        barrier(ws)
+    assert kda.workspace_status(work) == kda.KDA_OK
+    ms = max_over_ranks(t_s.elapsed_time(t_e) / steps, ws)
+    chunk_heads = B * (T // C) * H
+    kern = {}
+    for p, name in enumerate(names):
+        t_ms = statistics.mean(e[p].elapsed_time(e[p + 1]) for e in evs)
+        fl = chunk_heads * BWD_FLOPS_PER_CHUNK_HEAD[name]
+        a = fl / (t_ms * 1e-3) / 1e12
+        kern[name] = {"ms": t_ms, "achieved": a, "frac": a / FP32_ALU_TFLOPS, "flops_per_launch": fl}
+    dom = max(kern, key=lambda k: kern[k]["ms"])
+    th = B * T * H
+    gbs = th * BWD_BYTES_PER_TOKEN_HEAD / (ms * 1e-3) / 1e9
+    del grads, work, dout
+    torch.cuda.empty_cache()
+    return {"workload": WORKLOAD, "ms_per_step": ms, "Mtok_s": ws * B * T / (ms * 1e-3) / 1e6,
+            "steps": steps, "grads": "fp32", "arithmetic": "fp32 (CUDA cores)",
+            "roofline": {"bound": "alu", "achieved": kern[dom]["achieved"], "peak": FP32_ALU_TFLOPS,
+                         "unit": "TFLOP/s", "frac": kern[dom]["frac"], "traffic": None,
+                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz",
+                         "kernel": dom, "ms_per_launch": kern[dom]["ms"],
+                         "flops_per_launch": kern[dom]["flops_per_launch"], "kernels": kern,
+                         "step": {"hbm_gbs_algorithmic": gbs, "hbm_frac": gbs / pk["hbm"],
+                                  "algorithmic_bytes": th * BWD_BYTES_PER_TOKEN_HEAD}},
+            "gpu_launches": 3 * steps, "clocks": clk.summary()}
+
+
 def run_profile_case(args):
     """One small invocation for Nsight Compute captures: `prefill` runs kda_chunk_fwd on the
     first `--tokens` tokens of the 32-head bf16 workload (inputs > L2, a few GB at most) twice;
-    `decode` runs 8 decode steps of the 256 x 32 decode workload."""
+    `backward` runs kda_chunk_bwd twice on the same tokens; `decode` runs 8 decode steps of the
+    256 x 32 decode workload."""
     import kimi_delta_attention_25_b200 as kda
     kda.load()
     dev = torch.device("cuda", 0)
@@ -432,6 +520,15 @@ def run_profile_case(args):
                           out_dtype=torch.bfloat16)
         torch.cuda.synchronize()
         assert kda.workspace_status(kda.chunk_fwd.last_workspace) == kda.KDA_OK
+    elif args.profile == "backward":
+        w = K.WORKLOADS[WORKLOAD]
+        d = K.make_prefill(w, device=dev, T=args.tokens)
+        g = torch.Generator(device=dev).manual_seed(1234)
+        dout = torch.randn(d["v"].shape, generator=g, device=dev).to(torch.bfloat16)
+        for _ in range(2):
+            kda.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], dout, S0=d["S0"])
+        torch.cuda.synchronize()
+        assert kda.workspace_status(kda.chunk_bwd.last_workspace) == kda.KDA_OK
     else:
         w = K.WORKLOADS[DECODE]
         S = K.make_decode_state(w, device=dev)
@@ -449,7 +546,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--profile", choices=["prefill", "decode", "backward"], default=None,
                     help="run one small case for an Nsight Compute capture instead of the benchmark")
     ap.add_argument("--tokens", type=int, default=32768, help="tokens of the --profile prefill case")
     args = ap.parse_args()

@@ -163,6 +163,26 @@ kda_status_t kda_chunk_bwd(const void *q, const void *k, const void *v,
                            int B, int T, int H, int N, int dk, int dv, kda_dtype_t dtype,
                            void *workspace, size_t workspace_bytes, void *stream);
 
+/* The three kernels kda_chunk_bwd runs, one at a time (for timing them separately, or for
+ * running the phases of different batches on different streams), with the arguments of
+ * kda_chunk_bwd and the same checks:
+ *   phase 0  the forward sweep, recording into the workspace the state entering every chunk
+ *            and each chunk's R = V - Kt S and U; clears the workspace status word first;
+ *   phase 1  the reverse scan of the state gradient: writes dv_out and dS0, and records Y and
+ *            the gradient reaching the end of every chunk;
+ *   phase 2  every other gradient (dq, dk_out, dlog_alpha, dbeta), chunk by chunk.
+ * Each phase reads what the earlier ones recorded, so they must run in this order on the same
+ * workspace and arguments (same stream, or ordered by events); a phase run without the earlier
+ * ones returns garbage, not an error. Any other phase number: KDA_ERR_INVALID_ARG. */
+kda_status_t kda_chunk_bwd_phase(int phase, const void *q, const void *k, const void *v,
+                                 const float *log_alpha, const float *beta,
+                                 const float *S0, const int32_t *cu_seqlens,
+                                 const void *dout, const float *dS_final,
+                                 float *dq, float *dk_out, float *dv_out,
+                                 float *dlog_alpha, float *dbeta, float *dS0,
+                                 int B, int T, int H, int N, int dk, int dv, kda_dtype_t dtype,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
 /* One decode step for N independent sequences (one token each), updating the
  * state in place: the recurrent ("fused_recurrent") mode the layer uses for
  * short queries and generation (lpnh.cn article, sec. 2 and 5); the per-step

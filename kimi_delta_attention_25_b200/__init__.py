@@ -36,7 +36,7 @@ _lib = None
 EXPORTS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
            "kda_workspace_status", "kda_status_string", "kda_version", "kda_chunk_fwd_noalloc",
            "kda_chunk_prep", "kda_chunk_scan", "kda_selftest_wait_timeout",
-           "kda_chunk_bwd_workspace_size", "kda_chunk_bwd")
+           "kda_chunk_bwd_workspace_size", "kda_chunk_bwd", "kda_chunk_bwd_phase")
 
 
 class KDAError(RuntimeError):
@@ -78,6 +78,8 @@ def load():
     lib.kda_chunk_bwd_workspace_size.restype = Z
     lib.kda_chunk_bwd.argtypes = [P] * 15 + [I] * 7 + [P, Z, P]
     lib.kda_chunk_bwd.restype = I
+    lib.kda_chunk_bwd_phase.argtypes = [I] + [P] * 15 + [I] * 7 + [P, Z, P]
+    lib.kda_chunk_bwd_phase.restype = I
     _lib = lib
     return lib
 
@@ -188,11 +190,13 @@ def chunk_bwd_workspace_size(B, T, H, N, dk=128, dv=128) -> int:
 
 
 def chunk_bwd(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens=None,
-              want_dS0=True, grads=None, workspace=None):
+              want_dS0=True, grads=None, workspace=None, phase=None):
     """``kda_chunk_bwd``: gradients of a loss with gradients ``dout`` (w.r.t. every output, dtype of
     q) and ``dS_final`` (w.r.t. the final states, fp32 or None) through ``chunk_fwd`` with the same
     inputs. Returns a dict of fp32 tensors dq, dk, dv, dlog_alpha, dbeta and dS0 (None unless
-    ``want_dS0``). ``grads`` may supply those tensors (same keys) to be written in place."""
+    ``want_dS0``). ``grads`` may supply those tensors (same keys) to be written in place.
+    ``phase`` (0, 1 or 2) runs one of the three kernels only (``kda_chunk_bwd_phase``); the phases
+    must then run in order on the same ``grads`` and ``workspace``."""
     lib = load()
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -220,11 +224,14 @@ def chunk_bwd(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens
     ws_bytes = lib.kda_chunk_bwd_workspace_size(B, T, H, N, dk, dv)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
-    st = lib.kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
-                           _ptr(cu_seqlens), _ptr(dout), _ptr(dS_final), _ptr(g["dq"]), _ptr(g["dk"]),
-                           _ptr(g["dv"]), _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]), _ptr(g["dS0"]),
-                           B, T, H, N, dk, dv, _dtype_code(q), _ptr(workspace), workspace.numel(),
-                           _stream(dev))
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(cu_seqlens), _ptr(dout),
+            _ptr(dS_final), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]),
+            _ptr(g["dbeta"]), _ptr(g["dS0"]), B, T, H, N, dk, dv, _dtype_code(q), _ptr(workspace),
+            workspace.numel(), _stream(dev))
+    if phase is None:
+        st = lib.kda_chunk_bwd(*args)
+    else:
+        st = lib.kda_chunk_bwd_phase(int(phase), *args)
     if st != KDA_OK:
         raise KDAError(st, "kda_chunk_bwd")
     chunk_bwd.last_workspace = workspace

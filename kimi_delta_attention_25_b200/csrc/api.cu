@@ -162,14 +162,19 @@ size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int N, int dk, int dv)
     return kStatusBytes + (size_t)H * (size_t)prep_slots((long long)B * T, N) * per * sizeof(float);
 }
 
-kda_status_t kda_chunk_bwd(const void *q, const void *k, const void *v,
-                           const float *log_alpha, const float *beta,
-                           const float *S0, const int32_t *cu_seqlens,
-                           const void *dout, const float *dS_final,
-                           float *dq, float *dk_out, float *dv_out,
-                           float *dlog_alpha, float *dbeta, float *dS0,
-                           int B, int T, int H, int N, int dk, int dv, kda_dtype_t dtype,
-                           void *workspace, size_t workspace_bytes, void *stream)
+}  // extern "C"
+
+namespace {
+
+// The backward's host checks and launches; `phases` selects which of the three kernels to enqueue
+// (bit 0: forward sweep with records, also clearing the status word; bit 1: reverse scan of the
+// state gradient; bit 2: per-chunk gradients).
+kda_status_t chunk_bwd_impl(unsigned phases, const void *q, const void *k, const void *v,
+                            const float *log_alpha, const float *beta, const float *S0,
+                            const int32_t *cu_seqlens, const void *dout, const float *dS_final,
+                            float *dq, float *dk_out, float *dv_out, float *dlog_alpha, float *dbeta,
+                            float *dS0, int B, int T, int H, int N, int dk, int dv, kda_dtype_t dtype,
+                            void *workspace, size_t workspace_bytes, void *stream)
 {
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || H <= 0 || N < 0) return KDA_ERR_INVALID_ARG;
@@ -196,7 +201,7 @@ kda_status_t kda_chunk_bwd(const void *q, const void *k, const void *v,
     const size_t need = kda_chunk_bwd_workspace_size(B, T, H, N, dk, dv);
     if (!workspace || !aligned(workspace, 16) || workspace_bytes < need) return KDA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
-    if (cudaMemsetAsync(workspace, 0, kStatusBytes, st) != cudaSuccess) return KDA_ERR_CUDA;
+    if ((phases & 1u) && cudaMemsetAsync(workspace, 0, kStatusBytes, st) != cudaSuccess) return KDA_ERR_CUDA;
     if (N == 0) return KDA_OK;
 
     // records: S and dS' per (head, slot), then R, U, Y
@@ -208,12 +213,13 @@ kda_status_t kda_chunk_bwd(const void *q, const void *k, const void *v,
     float *ck_U = ck_R + hs * kBwdRowsFloats;
     float *ck_Y = ck_U + hs * kBwdRowsFloats;
 
-    // 1. forward sweep with records (outputs not needed)
-    PrefillArgs a = prefill_args(q, k, v, log_alpha, beta, S0, cu_seqlens, nullptr, nullptr, B, T, H, N,
-                                 workspace, workspace_bytes);
-    a.ck_S = ck_S; a.ck_R = ck_R; a.ck_U = ck_U; a.n_slots = (int)n_slots;
-    cudaError_t e = launch_chunk_fp32(a, dtype, KDA_F32, st);
-    // 2. reverse scan of the state gradient; 3. per-chunk gradients
+    cudaError_t e = cudaSuccess;
+    if (phases & 1u) {              // 1. forward sweep with records (outputs not needed)
+        PrefillArgs a = prefill_args(q, k, v, log_alpha, beta, S0, cu_seqlens, nullptr, nullptr, B, T, H, N,
+                                     workspace, workspace_bytes);
+        a.ck_S = ck_S; a.ck_R = ck_R; a.ck_U = ck_U; a.n_slots = (int)n_slots;
+        e = launch_chunk_fp32(a, dtype, KDA_F32, st);
+    }
     BwdArgs b;
     b.q = q; b.k = k; b.v = v; b.dout = dout;
     b.log_alpha = log_alpha; b.beta = beta; b.dS_final = dS_final;
@@ -222,9 +228,41 @@ kda_status_t kda_chunk_bwd(const void *q, const void *k, const void *v,
     b.ck_S = ck_S; b.ck_R = ck_R; b.ck_U = ck_U; b.ck_dS = ck_dS; b.ck_Y = ck_Y;
     b.B = B; b.T = T; b.H = H; b.N = N; b.n_slots = (int)n_slots;
     b.status = (int32_t *)workspace;
-    if (e == cudaSuccess) e = launch_chunk_bwd_scan(b, dtype, st);
-    if (e == cudaSuccess) e = launch_chunk_bwd_local(b, dtype, st);
+    if (e == cudaSuccess && (phases & 2u)) e = launch_chunk_bwd_scan(b, dtype, st);   // 2. reverse scan
+    if (e == cudaSuccess && (phases & 4u)) e = launch_chunk_bwd_local(b, dtype, st);  // 3. per chunk
     return map_cuda(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status_t kda_chunk_bwd(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const float *beta,
+                           const float *S0, const int32_t *cu_seqlens,
+                           const void *dout, const float *dS_final,
+                           float *dq, float *dk_out, float *dv_out,
+                           float *dlog_alpha, float *dbeta, float *dS0,
+                           int B, int T, int H, int N, int dk, int dv, kda_dtype_t dtype,
+                           void *workspace, size_t workspace_bytes, void *stream)
+{
+    return chunk_bwd_impl(7u, q, k, v, log_alpha, beta, S0, cu_seqlens, dout, dS_final, dq, dk_out, dv_out,
+                          dlog_alpha, dbeta, dS0, B, T, H, N, dk, dv, dtype, workspace, workspace_bytes, stream);
+}
+
+kda_status_t kda_chunk_bwd_phase(int phase, const void *q, const void *k, const void *v,
+                                 const float *log_alpha, const float *beta,
+                                 const float *S0, const int32_t *cu_seqlens,
+                                 const void *dout, const float *dS_final,
+                                 float *dq, float *dk_out, float *dv_out,
+                                 float *dlog_alpha, float *dbeta, float *dS0,
+                                 int B, int T, int H, int N, int dk, int dv, kda_dtype_t dtype,
+                                 void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (phase < 0 || phase > 2) return KDA_ERR_INVALID_ARG;
+    return chunk_bwd_impl(1u << phase, q, k, v, log_alpha, beta, S0, cu_seqlens, dout, dS_final, dq, dk_out,
+                          dv_out, dlog_alpha, dbeta, dS0, B, T, H, N, dk, dv, dtype, workspace, workspace_bytes,
+                          stream);
 }
 
 kda_status_t kda_decode_step(const void *q, const void *k, const void *v,

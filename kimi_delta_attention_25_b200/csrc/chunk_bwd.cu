@@ -29,6 +29,7 @@
 //     dependence (data-parallel over the whole grid).
 // Rows past a chunk's end are zero-filled (log_alpha = 0, k = q = v = dO = 0), which leaves every
 // gradient of the real rows unchanged.
+#include "chunk_fp32_common.cuh"
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -55,8 +56,7 @@ struct ScanSmem {
     float A[C * LDC];
     float M[C * LDC];
     float dO[C * DVB];
-    float dU[C * DVB];
-    float Y[C * DVB];
+    float Y[C * DVB];        // dU, then Y in place
     float gam[DK];
     float beta[C];
 };
@@ -92,41 +92,19 @@ chunk_bwd_scan_kernel(BwdArgs a)
         const size_t rec = (size_t)h * a.n_slots + (size_t)chunk_slot(s, n);
         __syncthreads();
         // ---- load the chunk (k -> Kt, q -> Qt, log_alpha -> Kh, dO block) and record dS'
-        for (int idx = tid; idx < C * DK; idx += NT_SCAN) {
-            const int r = idx / DK, c = idx % DK;
-            float kk = 0.f, qq = 0.f, la = 0.f;
-            if (r < L) {
-                const size_t off = ((size_t)(s + r) * H + h) * DK + c;
-                kk = to_f32(k[off]);
-                qq = to_f32(q[off]);
-                la = a.log_alpha[off];
-            }
-            sm.Kt[r * LD + c] = kk;
-            sm.Qt[r * LD + c] = qq;
-            sm.Kh[r * LD + c] = la;
-        }
-        for (int idx = tid; idx < C * DVB; idx += NT_SCAN) {
-            const int r = idx / DVB, j = idx % DVB;
-            sm.dO[idx] = (r < L) ? to_f32(dout[((size_t)(s + r) * H + h) * DK + j0 + j]) : 0.f;
-        }
+        fp32c::load_chunk<T, NT_SCAN>(sm.Kt, sm.Qt, sm.Kh, LD, sm.dO, q, k, a.log_alpha, dout, s, L, H, h, j0, tid);
         if (tid < C) sm.beta[tid] = (tid < L) ? a.beta[(size_t)(s + tid) * H + h] : 0.f;
-        {
-            float *dst = a.ck_dS + rec * kBwdStateFloats;
-            for (int idx = tid; idx < DK * DVB; idx += NT_SCAN) {
-                const int c = idx / DVB, j = idx % DVB;
-                dst[(size_t)c * DK + j0 + j] = sm.dS[idx];
-            }
-        }
+        fp32c::store_block32<NT_SCAN>(a.ck_dS + rec * kBwdStateFloats + j0, DK, sm.dS, DK, tid);
         __syncthreads();
 
-        // ---- cumulative log-decay and the decay-scaled operands (one thread per key channel)
-        if (tid < DK) {
-            const int c = tid;
-            float g = 0.f;
-            for (int r = 0; r < C; ++r) { g += sm.Kh[r * LD + c]; sm.Kh[r * LD + c] = g; }
-            const float gl = g;
-            sm.gam[c] = expf(gl);
-            for (int r = 0; r < C; ++r) {
+        // ---- cumulative log-decay (all threads, in row parts), then the decay-scaled operands
+        {
+            const float gl = fp32c::decay_prefix<NT_SCAN>(sm.Kh, LD, tid);
+            constexpr int RP = C / (NT_SCAN / DK);
+            const int c = tid % DK, r0 = (tid / DK) * RP;
+            if (tid < DK) sm.gam[c] = expf(gl);
+#pragma unroll 4
+            for (int r = r0; r < r0 + RP; ++r) {
                 const float gr = sm.Kh[r * LD + c];
                 const float kk = sm.Kt[r * LD + c];
                 const float e = expf(gr);
@@ -181,48 +159,19 @@ chunk_bwd_scan_kernel(BwdArgs a)
             float acc[8];
 #pragma unroll
             for (int x = 0; x < 8; ++x) acc[x] = 0.f;
-            for (int i = r; i < C; ++i) {
-                const float m = sm.M[i * LDC + r];
+            for (int i = r; i < C; ++i) fp32c::axpy<8>(acc, sm.M[i * LDC + r], sm.dO + i * DVB + jg);
+            for (int c = 0; c < DK; ++c) fp32c::axpy<8>(acc, sm.Ke[r * LD + c], sm.dS + c * DVB + jg);
 #pragma unroll
-                for (int x = 0; x < 8; ++x) acc[x] += m * sm.dO[i * DVB + jg + x];
-            }
-            for (int c = 0; c < DK; ++c) {
-                const float ke = sm.Ke[r * LD + c];
-#pragma unroll
-                for (int x = 0; x < 8; ++x) acc[x] += ke * sm.dS[c * DVB + jg + x];
-            }
-#pragma unroll
-            for (int x = 0; x < 8; ++x) sm.dU[r * DVB + jg + x] = acc[x];
+            for (int x = 0; x < 8; ++x) sm.Y[r * DVB + jg + x] = acc[x];
         }
         __syncthreads();
 
-        // ---- Y = (I + A)^{-T} dU by back substitution: Y_r = dU_r - sum_{i>r} A_ir Y_i.
-        //      Warp w owns columns 4w..4w+3; eight lanes per column split the sum.
-        {
-            const int warp = tid >> 5, lane = tid & 31;
-            const int j = warp * 4 + lane / 8, p = lane % 8;
-            for (int r = C - 1; r >= 0; --r) {
-                float part = 0.f;
-                for (int i = r + 1 + p; i < C; i += 8) part += sm.A[i * LDC + r] * sm.Y[i * DVB + j];
-                part += __shfl_xor_sync(0xffffffffu, part, 1);
-                part += __shfl_xor_sync(0xffffffffu, part, 2);
-                part += __shfl_xor_sync(0xffffffffu, part, 4);
-                if (p == 0) sm.Y[r * DVB + j] = sm.dU[r * DVB + j] - part;
-                __syncwarp();
-            }
-        }
-        __syncthreads();
+        // ---- Y = (I + A)^{-T} dU: blocked back substitution in place
+        fp32c::upper_solve_32<NT_SCAN>(sm.A, LDC, sm.Y, tid);
 
         // ---- dV = diag(beta) Y -> dv (rows < L); Y -> record (all rows)
-        {
-            float *ydst = a.ck_Y + rec * kBwdRowsFloats;
-            for (int idx = tid; idx < C * DVB; idx += NT_SCAN) {
-                const int r = idx / DVB, j = idx % DVB;
-                const float y = sm.Y[idx];
-                ydst[(size_t)r * DK + j0 + j] = y;
-                if (r < L) a.dv[((size_t)(s + r) * H + h) * DK + j0 + j] = sm.beta[r] * y;
-            }
-        }
+        fp32c::store_block32<NT_SCAN>(a.ck_Y + rec * kBwdRowsFloats + j0, DK, sm.Y, C, tid);
+        fp32c::store_block32<NT_SCAN>(a.dv + ((size_t)s * H + h) * DK + j0, (size_t)H * DK, sm.Y, L, tid, sm.beta);
 
         // ---- dS <- Diag(gamma) dS' + Qt^T dO - Kt^T diag(beta) Y: thread -> key channel c, 16 columns
         {
@@ -232,10 +181,8 @@ chunk_bwd_scan_kernel(BwdArgs a)
 #pragma unroll
             for (int x = 0; x < 16; ++x) acc[x] = gm * sm.dS[c * DVB + jh + x];
             for (int r = 0; r < C; ++r) {
-                const float qt = sm.Qt[r * LD + c];
-                const float kb = sm.Kt[r * LD + c] * sm.beta[r];
-#pragma unroll
-                for (int x = 0; x < 16; ++x) acc[x] += qt * sm.dO[r * DVB + jh + x] - kb * sm.Y[r * DVB + jh + x];
+                fp32c::axpy<16>(acc, sm.Qt[r * LD + c], sm.dO + r * DVB + jh);
+                fp32c::axpy<16>(acc, -sm.Kt[r * LD + c] * sm.beta[r], sm.Y + r * DVB + jh);
             }
 #pragma unroll
             for (int x = 0; x < 16; ++x) sm.dS[c * DVB + jh + x] = acc[x];
@@ -263,7 +210,7 @@ struct LocalSmem {
     // one 32-column block of the value axis at a time; after the loop: dM and dP (64 x LDC each)
     float S[DK * LDV];
     float dSn[DK * LDV];
-    float dO[C * LDV];
+    float dO[C * LDV];       // after the last products: per-warp column sums (16 x 128)
     float U[C * LDV];
     float Y[C * LDV];
     float R[C * LDV];
@@ -271,9 +218,9 @@ struct LocalSmem {
     float beta[C];
     float gam[DK];
     float dgam[DK];
-    float dgl[DK];
     float ry[C];
 };
+static_assert((NT_LOC / 32) * DK <= C * LDV, "per-warp column sums must fit the dO block");
 
 template <typename T>
 __global__ void __launch_bounds__(NT_LOC, 1)
@@ -292,36 +239,28 @@ chunk_bwd_local_kernel(BwdArgs a)
     const T *k = (const T *)a.k;
     const T *dout = (const T *)a.dout;
 
-    // ---- load q, k, log_alpha (zero past L), beta
-    for (int idx = tid; idx < C * DK; idx += NT_LOC) {
-        const int r = idx / DK, c = idx % DK;
-        float kk = 0.f, qq = 0.f, la = 0.f;
-        if (r < L) {
-            const size_t off = ((size_t)(s + r) * H + h) * DK + c;
-            kk = to_f32(k[off]);
-            qq = to_f32(q[off]);
-            la = a.log_alpha[off];
-        }
-        sm.Kt[r * LD + c] = kk;
-        sm.Qt[r * LD + c] = qq;
-        sm.E[r * LD + c] = la;
-    }
+    // ---- load q, k, log_alpha (zero past L), beta; then g = cumsum(log_alpha) in row parts
+    fp32c::load_rows<T, NT_LOC, DK>(sm.Kt, LD, k, s, L, H, h, 0, tid);
+    fp32c::load_rows<T, NT_LOC, DK>(sm.Qt, LD, q, s, L, H, h, 0, tid);
+    fp32c::load_rows<float, NT_LOC, DK>(sm.E, LD, a.log_alpha, s, L, H, h, 0, tid);
     if (tid < C) sm.beta[tid] = (tid < L) ? a.beta[(size_t)(s + tid) * H + h] : 0.f;
-    if (tid < DK) { sm.dgam[tid] = 0.f; sm.dgl[tid] = 0.f; }
+    if (tid < DK) sm.dgam[tid] = 0.f;
     if (tid < C) sm.ry[tid] = 0.f;
     __syncthreads();
-    if (tid < DK) {
-        const int c = tid;
-        float g = 0.f;
-        for (int r = 0; r < C; ++r) {
-            g += sm.E[r * LD + c];
+    {
+        const float gl = fp32c::decay_prefix<NT_LOC>(sm.E, LD, tid);
+        constexpr int RP = C / (NT_LOC / DK);
+        const int c = tid % DK, r0 = (tid / DK) * RP;
+        if (tid < DK) sm.gam[c] = expf(gl);
+#pragma unroll 4
+        for (int r = r0; r < r0 + RP; ++r) {
+            const float g = sm.E[r * LD + c];
             const float e = expf(g), kk = sm.Kt[r * LD + c];
             sm.E[r * LD + c] = e;
             sm.Kt[r * LD + c] = kk * e;
             sm.Kh[r * LD + c] = kk * expf(-g);
             sm.Qt[r * LD + c] *= e;
         }
-        sm.gam[c] = expf(g);
     }
     __syncthreads();
 
@@ -365,17 +304,33 @@ chunk_bwd_local_kernel(BwdArgs a)
     float dgam_acc = 0.f, ry_acc = 0.f;
     for (int j0 = 0; j0 < DK; j0 += DVB) {
         __syncthreads();
-        for (int idx = tid; idx < DK * DVB; idx += NT_LOC) {
-            const int c = idx / DVB, v = idx % DVB;
-            sm.S[c * LDV + v] = gS[(size_t)c * DK + j0 + v];
-            sm.dSn[c * LDV + v] = gdS[(size_t)c * DK + j0 + v];
-        }
-        for (int idx = tid; idx < C * DVB; idx += NT_LOC) {
-            const int r = idx / DVB, v = idx % DVB;
-            sm.U[r * LDV + v] = gU[(size_t)r * DK + j0 + v];
-            sm.Y[r * LDV + v] = gY[(size_t)r * DK + j0 + v];
-            sm.R[r * LDV + v] = gR[(size_t)r * DK + j0 + v];
-            sm.dO[r * LDV + v] = (r < L) ? to_f32(dout[((size_t)(s + r) * H + h) * DK + j0 + v]) : 0.f;
+        {
+            // 16-byte loads, all in flight before the first store: the state blocks (128 rows of
+            // 8 float4, two per thread) and the row blocks (64 rows of 8 float4, one per thread)
+            float4 xs[2], xd[2], xu, xy, xr;
+#pragma unroll
+            for (int it = 0; it < 2; ++it) {
+                const int idx = tid + it * NT_LOC, c = idx >> 3, q4 = idx & 7;
+                xs[it] = __ldg(reinterpret_cast<const float4 *>(gS + (size_t)c * DK + j0) + q4);
+                xd[it] = __ldg(reinterpret_cast<const float4 *>(gdS + (size_t)c * DK + j0) + q4);
+            }
+            const int r = tid >> 3, q4 = tid & 7;
+            xu = __ldg(reinterpret_cast<const float4 *>(gU + (size_t)r * DK + j0) + q4);
+            xy = __ldg(reinterpret_cast<const float4 *>(gY + (size_t)r * DK + j0) + q4);
+            xr = __ldg(reinterpret_cast<const float4 *>(gR + (size_t)r * DK + j0) + q4);
+            fp32c::load_rows<T, NT_LOC, DVB>(sm.dO, LDV, dout, s, L, H, h, j0, tid);
+#pragma unroll
+            for (int it = 0; it < 2; ++it) {
+                const int idx = tid + it * NT_LOC, c = idx >> 3, v = (idx & 7) * 4;
+                float *ds = sm.S + c * LDV + v, *dd = sm.dSn + c * LDV + v;
+                ds[0] = xs[it].x; ds[1] = xs[it].y; ds[2] = xs[it].z; ds[3] = xs[it].w;
+                dd[0] = xd[it].x; dd[1] = xd[it].y; dd[2] = xd[it].z; dd[3] = xd[it].w;
+            }
+            const int v = q4 * 4;
+            float *du = sm.U + r * LDV + v, *dy = sm.Y + r * LDV + v, *dr = sm.R + r * LDV + v;
+            du[0] = xu.x; du[1] = xu.y; du[2] = xu.z; du[3] = xu.w;
+            dy[0] = xy.x; dy[1] = xy.y; dy[2] = xy.z; dy[3] = xy.w;
+            dr[0] = xr.x; dr[1] = xr.y; dr[2] = xr.z; dr[3] = xr.w;
         }
         __syncthreads();
 #pragma unroll 4
@@ -506,14 +461,17 @@ chunk_bwd_local_kernel(BwdArgs a)
     for (int x = 0; x < 4; ++x)
 #pragma unroll
         for (int z = 0; z < 4; ++z) sm.Kh[(4 * rb + x) * LD + cb + 32 * z] = dg[x][z];
+    // per-warp column sums of dKe * Ke into the (now free) dO block, added in a fixed order below
 #pragma unroll
-    for (int z = 0; z < 4; ++z) atomicAdd(&sm.dgl[cb + 32 * z], colp[z]);
+    for (int z = 0; z < 4; ++z) sm.dO[rb * DK + cb + 32 * z] = colp[z];
     __syncthreads();
     // ---- dlog_alpha: reverse cumulative sum over rows, the last row also carrying the terms of
     //      g_{L-1} (through Ke and gamma)
     if (tid < DK) {
         const int c = tid;
-        float run = sm.dgl[c] + sm.dgam[c] * sm.gam[c];
+        float dgl = 0.f;
+        for (int w = 0; w < NT_LOC / 32; ++w) dgl += sm.dO[w * DK + c];
+        float run = dgl + sm.dgam[c] * sm.gam[c];
         for (int r = C - 1; r >= 0; --r) {
             run += sm.Kh[r * LD + c];
             if (r < L) a.dlog_alpha[((size_t)(s + r) * H + h) * DK + c] = run;

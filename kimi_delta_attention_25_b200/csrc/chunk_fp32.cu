@@ -20,6 +20,7 @@
 //
 // For the backward pass the same kernel also records, per (head, chunk slot), the state entering
 // each chunk and the chunk's R = V - Kt S and U (PrefillArgs::ck_*), and may skip the outputs.
+#include "chunk_fp32_common.cuh"
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -76,43 +77,20 @@ chunk_fp32_kernel(PrefillArgs a)
         const int L = (t1 - s < C) ? (int)(t1 - s) : C;
         __syncthreads();
         // ---- load the chunk: k -> Kt, q -> Qt, log_alpha -> Kh, v block -> R
-        for (int idx = tid; idx < C * DK; idx += NT) {
-            const int r = idx / DK, c = idx % DK;
-            float kk = 0.f, qq = 0.f, la = 0.f;
-            if (r < L) {
-                const size_t off = ((size_t)(s + r) * H + h) * DK + c;
-                kk = to_f32(k[off]);
-                qq = to_f32(q[off]);
-                la = a.log_alpha[off];
-            }
-            sm.Kt[r * LD + c] = kk;
-            sm.Qt[r * LD + c] = qq;
-            sm.Kh[r * LD + c] = la;
-        }
-        for (int idx = tid; idx < C * DVB; idx += NT) {
-            const int r = idx / DVB, j = idx % DVB;
-            sm.R[idx] = (r < L) ? to_f32(v[((size_t)(s + r) * H + h) * DK + j0 + j]) : 0.f;
-        }
+        fp32c::load_chunk<T, NT>(sm.Kt, sm.Qt, sm.Kh, LD, sm.R, q, k, a.log_alpha, v, s, L, H, h, j0, tid);
         if (tid < C) sm.beta[tid] = (tid < L) ? a.beta[(size_t)(s + tid) * H + h] : 0.f;
         // backward records of this chunk: (head, chunk slot) blocks
         const size_t rec = (size_t)h * a.n_slots + (size_t)chunk_slot(s, n);
-        if (a.ck_S) {
-            float *dst = a.ck_S + rec * kBwdStateFloats;
-            for (int idx = tid; idx < DK * DVB; idx += NT) {
-                const int c = idx / DVB, j = idx % DVB;
-                dst[(size_t)c * DK + j0 + j] = sm.S[idx];
-            }
-        }
+        if (a.ck_S) fp32c::store_block32<NT>(a.ck_S + rec * kBwdStateFloats + j0, DK, sm.S, DK, tid);
         __syncthreads();
 
-        // ---- cumulative log-decay and the decay-scaled operands (one thread per key channel)
-        if (tid < DK) {
-            const int c = tid;
-            float g = 0.f;
-            for (int r = 0; r < C; ++r) { g += sm.Kh[r * LD + c]; sm.Kh[r * LD + c] = g; }
-            const float gl = g;
-            sm.gam[c] = expf(gl);
-            for (int r = 0; r < C; ++r) {
+        // ---- cumulative log-decay (all threads, in row parts), then the decay-scaled operands
+        {
+            const float gl = fp32c::decay_prefix<NT>(sm.Kh, LD, tid);
+            const int c = tid % DK, part = tid / DK, r0 = part * (C / (NT / DK));
+            if (part == 0) sm.gam[c] = expf(gl);
+#pragma unroll 4
+            for (int r = r0; r < r0 + C / (NT / DK); ++r) {
                 const float gr = sm.Kh[r * LD + c];
                 const float kk = sm.Kt[r * LD + c];
                 const float e = expf(gr);
@@ -132,7 +110,7 @@ chunk_fp32_kernel(PrefillArgs a)
             for (int x = 0; x < 4; ++x)
 #pragma unroll
                 for (int y = 0; y < 4; ++y) { accA[x][y] = 0.f; accM[x][y] = 0.f; }
-            if (ib <= rb) {
+            if (ib <= rb && out) {
                 for (int c = 0; c < DK; ++c) {
                     float kt[4], qt[4], kh[4];
 #pragma unroll
@@ -148,6 +126,19 @@ chunk_fp32_kernel(PrefillArgs a)
                             accA[x][y] += kt[x] * kh[y];
                             accM[x][y] += qt[x] * kh[y];
                         }
+                }
+            } else if (ib <= rb) {                 // records only: M is not needed
+                for (int c = 0; c < DK; ++c) {
+                    float kt[4], kh[4];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        kt[x] = sm.Kt[(4 * rb + x) * LD + c];
+                        kh[x] = sm.Kh[(4 * ib + x) * LD + c];
+                    }
+#pragma unroll
+                    for (int x = 0; x < 4; ++x)
+#pragma unroll
+                        for (int y = 0; y < 4; ++y) accA[x][y] += kt[x] * kh[y];
                 }
             }
 #pragma unroll
@@ -165,45 +156,24 @@ chunk_fp32_kernel(PrefillArgs a)
             float acc[8];
 #pragma unroll
             for (int x = 0; x < 8; ++x) acc[x] = 0.f;
-            for (int c = 0; c < DK; ++c) {
-                const float kt = sm.Kt[r * LD + c];
-#pragma unroll
-                for (int x = 0; x < 8; ++x) acc[x] += kt * sm.S[c * DVB + jg + x];
-            }
+            for (int c = 0; c < DK; ++c) fp32c::axpy<8>(acc, sm.Kt[r * LD + c], sm.S + c * DVB + jg);
             const float b = sm.beta[r];
             if (a.ck_R) {
-                float *dst = a.ck_R + rec * kBwdRowsFloats + (size_t)r * DK + j0 + jg;
-#pragma unroll
-                for (int x = 0; x < 8; ++x) dst[x] = sm.R[r * DVB + jg + x] - acc[x];
+                float4 *dst = reinterpret_cast<float4 *>(a.ck_R + rec * kBwdRowsFloats + (size_t)r * DK + j0 + jg);
+                const float *rv = sm.R + r * DVB + jg;
+                dst[0] = make_float4(rv[0] - acc[0], rv[1] - acc[1], rv[2] - acc[2], rv[3] - acc[3]);
+                dst[1] = make_float4(rv[4] - acc[4], rv[5] - acc[5], rv[6] - acc[6], rv[7] - acc[7]);
             }
 #pragma unroll
             for (int x = 0; x < 8; ++x) sm.R[r * DVB + jg + x] = b * (sm.R[r * DVB + jg + x] - acc[x]);
         }
         __syncthreads();
 
-        // ---- U = (I + A)^{-1} R by forward substitution; warp w owns columns 4w..4w+3,
-        //      eight lanes per column split the sum over earlier rows.
-        {
-            const int warp = tid >> 5, lane = tid & 31;
-            const int j = warp * 4 + lane / 8, p = lane % 8;
-            for (int r = 0; r < C; ++r) {
-                float part = 0.f;
-                for (int i = p; i < r; i += 8) part += sm.A[r * LDC + i] * sm.U[i * DVB + j];
-                part += __shfl_xor_sync(0xffffffffu, part, 1);
-                part += __shfl_xor_sync(0xffffffffu, part, 2);
-                part += __shfl_xor_sync(0xffffffffu, part, 4);
-                if (p == 0) sm.U[r * DVB + j] = sm.R[r * DVB + j] - part;
-                __syncwarp();
-            }
-        }
+        // ---- U = (I + A)^{-1} R: blocked forward substitution (U starts as a copy of R)
+        for (int idx = tid; idx < C * DVB; idx += NT) sm.U[idx] = sm.R[idx];
         __syncthreads();
-        if (a.ck_U) {
-            float *dst = a.ck_U + rec * kBwdRowsFloats;
-            for (int idx = tid; idx < C * DVB; idx += NT) {
-                const int r = idx / DVB, j = idx % DVB;
-                dst[(size_t)r * DK + j0 + j] = sm.U[idx];
-            }
-        }
+        fp32c::lower_solve_32<NT>(sm.A, LDC, sm.U, tid);
+        if (a.ck_U) fp32c::store_block32<NT>(a.ck_U + rec * kBwdRowsFloats + j0, DK, sm.U, C, tid);
 
         // ---- O = Qt S + M U  -> out (rows < L); skipped when only the records are wanted
         if (out) {
@@ -211,16 +181,8 @@ chunk_fp32_kernel(PrefillArgs a)
             float acc[8];
 #pragma unroll
             for (int x = 0; x < 8; ++x) acc[x] = 0.f;
-            for (int c = 0; c < DK; ++c) {
-                const float qt = sm.Qt[r * LD + c];
-#pragma unroll
-                for (int x = 0; x < 8; ++x) acc[x] += qt * sm.S[c * DVB + jg + x];
-            }
-            for (int i = 0; i <= r; ++i) {
-                const float m = sm.M[r * LDC + i];
-#pragma unroll
-                for (int x = 0; x < 8; ++x) acc[x] += m * sm.U[i * DVB + jg + x];
-            }
+            for (int c = 0; c < DK; ++c) fp32c::axpy<8>(acc, sm.Qt[r * LD + c], sm.S + c * DVB + jg);
+            for (int i = 0; i <= r; ++i) fp32c::axpy<8>(acc, sm.M[r * LDC + i], sm.U + i * DVB + jg);
             if (r < L) {
                 TO *o = out + ((size_t)(s + r) * H + h) * DK + j0 + jg;
 #pragma unroll
@@ -236,11 +198,7 @@ chunk_fp32_kernel(PrefillArgs a)
             const float gm = sm.gam[c];
 #pragma unroll
             for (int x = 0; x < 16; ++x) acc[x] = gm * sm.S[c * DVB + jh + x];
-            for (int r = 0; r < C; ++r) {
-                const float ke = sm.Ke[r * LD + c];
-#pragma unroll
-                for (int x = 0; x < 16; ++x) acc[x] += ke * sm.U[r * DVB + jh + x];
-            }
+            for (int r = 0; r < C; ++r) fp32c::axpy<16>(acc, sm.Ke[r * LD + c], sm.U + r * DVB + jh);
 #pragma unroll
             for (int x = 0; x < 16; ++x) sm.S[c * DVB + jh + x] = acc[x];
         }

@@ -183,3 +183,14 @@ def test_backward_host_checks(lib):
     assert _bwd(lib, B=2, N=2, cu=FAKE) == kda.KDA_ERR_INVALID_ARG
     assert _bwd(lib) == kda.KDA_ERR_INVALID_ARG                           # workspace too small
     assert _bwd(lib, ws=FAKE + 8, wsb=need) == kda.KDA_ERR_INVALID_ARG    # misaligned workspace
+
+
+def test_backward_phase_host_checks(lib):
+    P = ctypes.c_void_p
+    f = lib.kda_chunk_bwd_phase
+    args = [P(FAKE)] * 5 + [None, None, P(FAKE), None] + [P(FAKE)] * 5 + [None] + [1, 64, 2, 1, 128, 128, 1]
+    assert f(3, *args, P(FAKE), 256, None) == kda.KDA_ERR_INVALID_ARG      # no such phase
+    assert f(-1, *args, P(FAKE), 256, None) == kda.KDA_ERR_INVALID_ARG
+    assert f(1, *args, P(FAKE), 256, None) == kda.KDA_ERR_INVALID_ARG      # workspace too small
+    args[19] = 64                                                           # dk
+    assert f(2, *args, P(FAKE), 1 << 30, None) == kda.KDA_ERR_UNSUPPORTED

@@ -122,3 +122,43 @@ def test_bf16_t8k_h16_sampled_heads():
     w = K.WORKLOADS["bf16_t8k_h16"]
     d = _with_output_grads(K.make_prefill(w), seed=8)
     _run(d, TOL[torch.bfloat16], heads=[0, 15])
+
+
+def test_phases_one_by_one_equal_one_call_bitwise():
+    w = K.Workload("bwd_phases", B=1, T=300, H=2, dtype="bf16", s0_std=0.1)
+    d = to_device(_with_output_grads(K.make_prefill(w, seed=37), seed=9), DEV)
+    args = (d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["dout"])
+    kw = dict(S0=d["S0"], dS_final=d["dS_final"])
+    ref = kda.chunk_bwd(*args, **kw)
+    g = None
+    ws = None
+    for phase in range(3):
+        g = kda.chunk_bwd(*args, **kw, grads=g, workspace=ws, phase=phase)
+        ws = kda.chunk_bwd.last_workspace
+    assert kda.workspace_status(ws) == kda.KDA_OK
+    for name in GRADS:
+        assert torch.equal(g[name], ref[name]), name
+
+
+@pytest.mark.slow
+def test_bf16_t128k_h32_sampled_head():
+    """The benchmark workload (128K tokens, 32 heads, bf16) in the benchmark's launch configuration;
+    one head is recomputed by the oracle (heads are independent)."""
+    w = K.WORKLOADS["bf16_t128k_h32"]
+    d = K.make_prefill(w, device=DEV)
+    g = torch.Generator(device=DEV).manual_seed(10)
+    B, T, H, D = d["v"].shape
+    d["dout"] = torch.randn(B, T, H, D, generator=g, device=DEV).to(torch.bfloat16)
+    d["dS_final"] = torch.randn(B, H, D, D, generator=g, device=DEV)
+    gr = kda.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["dout"], S0=d["S0"],
+                       dS_final=d["dS_final"])
+    assert kda.workspace_status(kda.chunk_bwd.last_workspace) == kda.KDA_OK
+    h = 7
+    sub = {x: d[x][:, :, h:h + 1].contiguous() for x in ("q", "k", "v", "log_alpha", "beta", "dout")}
+    sub["S0"] = d["S0"][:, h:h + 1].contiguous()
+    sub["dS_final"] = d["dS_final"][:, h:h + 1].contiguous()
+    sub["cu_seqlens"] = None
+    r = _oracle(sub)
+    for name in GRADS:
+        x = gr[name][:, h:h + 1] if name == "dS0" else gr[name][:, :, h:h + 1]
+        assert_close(np32(x), r[name], TOL[torch.bfloat16], name)
