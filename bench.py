@@ -225,6 +225,26 @@ def cpu_oracle_sample(budget_s=12.0):
             "seconds": dt, "host_cores": cores}
 
 
+def cpu_oracle_backward_sample(tokens=8192):
+    """Times the float64 backward oracle (token-level reverse sweep, numpy, one thread) as it
+    stands on the first `tokens` tokens of one head of the prefill workload; scaled to tokens of
+    the full 32-head workload per second."""
+    from oracle import backward as bw
+    w = K.WORKLOADS[WORKLOAD]
+    d = K.make_prefill(w, T=tokens, H=1)
+    g = torch.Generator().manual_seed(1234)
+    dout = torch.randn(d["v"].shape, generator=g).to(torch.bfloat16)
+    f = lambda t: t.float().numpy()  # noqa: E731
+    t0 = time.perf_counter()
+    bw.backward(f(d["q"]), f(d["k"]), f(d["v"]), f(d["log_alpha"]), f(d["beta"]), f(dout),
+                S0=d["S0"].double().numpy())
+    dt = time.perf_counter() - t0
+    return {"value": tokens / w.H / dt / 1e6, "unit": "Mtok/s", "cores": 1, "kind": "oracle",
+            "sample": "float64 numpy reverse sweep on the first %d tokens of 1 of the %d heads "
+                      "(%.1f s; scaled to tokens of all %d heads)" % (tokens, w.H, dt, w.H),
+            "seconds": dt}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -357,6 +377,7 @@ def run_native(args):
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample()
+        bwd["cpu_baseline"] = cpu_oracle_backward_sample()
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": ws, "steps": args.steps,
