@@ -7,7 +7,9 @@ definition and by calculus, never by the backward code itself.
 * reverse-mode autograd (torch, float64, CPU) of an independent torch statement of the
   definition -- mechanical differentiation instead of the hand-derived chain rule;
 * closed forms: beta = 0 (pure decay, every gradient in closed form) and alpha = 1 with
-  orthonormal keys and S0 = 0 (plain linear attention, whose dv, dq and dbeta are textbook).
+  orthonormal keys and S0 = 0 (plain linear attention, whose dv, dq and dbeta are textbook);
+* exact directional derivatives: dual numbers over rationals stepped through the definition with
+  explicit transition matrices, on the exact inputs of the golden fixture.
 The last test plants slips in a copy of the backward oracle and checks the pins catch them.
 """
 import math
@@ -209,6 +211,8 @@ def test_pins_reject_planted_slips(slip, monkeypatch):
     monkeypatch.setattr(bw, "backward_head", _slipped_head(slip))
     with pytest.raises(AssertionError):
         test_backward_equals_autograd(64)
+    with pytest.raises(AssertionError):
+        test_backward_equals_exact_directional_derivatives_on_the_golden_inputs()
 
 
 @pytest.mark.parametrize("T,d,C,cu", [(1, 8, 64, None), (130, 16, 64, None), (200, 32, 64, [0, 70, 70, 200]),
@@ -224,3 +228,112 @@ def test_chunked_backward_equals_token_backward(T, d, C, cu):
                          cu_seqlens=cu, chunk=C)
     for key in a:
         assert rel_err(b[key], a[key]) < 1e-12, key
+
+
+# --- exact directional derivatives: dual numbers over rationals ------------------------------
+
+class _Dual:
+    """a + b eps with eps^2 = 0, over Fractions: forward-mode derivative in exact arithmetic."""
+    __slots__ = ("a", "b")
+
+    def __init__(self, a, b=0):
+        from fractions import Fraction
+        self.a, self.b = Fraction(a), Fraction(b)
+
+    @staticmethod
+    def lift(x):
+        return x if isinstance(x, _Dual) else _Dual(x)
+
+    def __add__(self, o):
+        o = _Dual.lift(o)
+        return _Dual(self.a + o.a, self.b + o.b)
+
+    __radd__ = __add__
+
+    def __sub__(self, o):
+        o = _Dual.lift(o)
+        return _Dual(self.a - o.a, self.b - o.b)
+
+    def __rsub__(self, o):
+        return _Dual.lift(o) - self
+
+    def __mul__(self, o):
+        o = _Dual.lift(o)
+        return _Dual(self.a * o.a, self.a * o.b + self.b * o.a)
+
+    __rmul__ = __mul__
+
+
+def _exact_jvp(q, k, v, alpha, beta, S0, dout, dSf, direction):
+    """Exact d/d(eps) of L = sum dout * o + sum dSf * S_final for one (sequence, head) when every
+    input x moves to x + eps * direction[x]; log_alpha moving by eps * delta moves alpha by
+    eps * alpha * delta. The recurrence is stepped with explicit transition matrices
+    (I - beta k k^T) Diag(alpha), straight from the definition."""
+    T, dk, dv = len(q), len(q[0]), len(v[0])
+    D = lambda name, *ix: 0 if name not in direction else direction[name][ix]  # noqa: E731
+
+    def dual(x, name, *ix):
+        return _Dual(x, D(name, *ix))
+
+    S = [[dual(S0[i][j], "S0", i, j) for j in range(dv)] for i in range(dk)]
+    L = _Dual(0)
+    for t in range(T):
+        qt = [dual(q[t][i], "q", t, i) for i in range(dk)]
+        kt = [dual(k[t][i], "k", t, i) for i in range(dk)]
+        vt = [dual(v[t][j], "v", t, j) for j in range(dv)]
+        at = [_Dual(alpha[t][i], alpha[t][i] * D("log_alpha", t, i)) for i in range(dk)]
+        bt = dual(beta[t], "beta", t)
+        A = [[((1 if i == c else 0) - bt * kt[i] * kt[c]) * at[c] for c in range(dk)] for i in range(dk)]
+        S = [[sum((A[i][c] * S[c][j] for c in range(dk)), _Dual(0)) + bt * kt[i] * vt[j] for j in range(dv)]
+             for i in range(dk)]
+        for j in range(dv):
+            o = sum((S[i][j] * qt[i] for i in range(dk)), _Dual(0))
+            L = L + o * dout[t][j]
+    for i in range(dk):
+        for j in range(dv):
+            L = L + S[i][j] * dSf[i][j]
+    return L.b
+
+
+def test_backward_equals_exact_directional_derivatives_on_the_golden_inputs():
+    """On the exact rational inputs of tests/golden/brute_tiny.json (two packed sequences, two
+    heads, d_k = 3, d_v = 2), every gradient of the float64 backward oracle, contracted with a
+    rational direction, equals the exact directional derivative of the definition."""
+    import json
+    import os
+    import random
+    from fractions import Fraction as F
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "brute_tiny.json")
+    with open(path) as f:
+        gd = json.load(f)
+    fr = lambda a: np.vectorize(lambda x: F(x), otypes=[object])(np.array(a, dtype=object))  # noqa: E731
+    q, k, v = fr(gd["q"]), fr(gd["k"]), fr(gd["v"])                 # [T][H][d]
+    alpha, beta, S0 = fr(gd["alpha"]), fr(gd["beta"]), fr(gd["S0"])
+    cu = gd["cu_seqlens"]
+    T, H = q.shape[0], q.shape[1]
+    rnd = random.Random(11)
+    rat = lambda *shape: np.vectorize(lambda _: F(rnd.randint(-6, 6), 4), otypes=[object])(  # noqa: E731
+        np.zeros(shape))
+    dout, dSf = rat(T, H, v.shape[2]), rat(len(cu) - 1, H, k.shape[2], v.shape[2])
+    fl = lambda a: np.vectorize(float)(a).astype(np.float64)  # noqa: E731
+    g = bw.backward(fl(q)[None], fl(k)[None], fl(v)[None], np.log(fl(alpha))[None], fl(beta)[None],
+                    fl(dout)[None], S0=fl(S0), dS_final=fl(dSf), cu_seqlens=cu)
+    for n in range(len(cu) - 1):
+        t0, t1 = cu[n], cu[n + 1]
+        for h in range(H):
+            seq = lambda a: [list(a[t, h]) for t in range(t0, t1)]  # noqa: E731
+            args = (seq(q), seq(k), seq(v), seq(alpha), [beta[t, h] for t in range(t0, t1)],
+                    [list(r) for r in S0[n, h]], seq(dout), [list(r) for r in dSf[n, h]])
+            for name, gname in NAMES:
+                if name == "S0":
+                    d = rat(k.shape[2], v.shape[2])
+                    mine = float(np.sum(g["dS0"][n, h] * fl(d)))
+                elif name == "beta":
+                    d = rat(t1 - t0)
+                    mine = float(np.sum(g["dbeta"][0, t0:t1, h] * fl(d)))
+                else:
+                    width = v.shape[2] if name == "v" else k.shape[2]
+                    d = rat(t1 - t0, width)
+                    mine = float(np.sum(g[gname][0, t0:t1, h] * fl(d)))
+                exact = _exact_jvp(*args, direction={name: d})
+                assert abs(mine - float(exact)) <= 1e-12 * max(1.0, abs(float(exact))), (n, h, name, mine, exact)
