@@ -141,10 +141,55 @@ def _chunk_backward(S, dSn, dO, q, k, v, la, be):
     return dq, dk, dv, dla, dbe, dS
 
 
-def backward(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens=None, chunk=64):
+def _chunk_backward_regrouped(S, dSn, dO, q, k, v, la, be):
+    """The same gradients as ``_chunk_backward``, regrouped the way the GPU backward computes them:
+    no inverse is formed -- Y = (I + A)^{-T} dU comes from one triangular solve -- and every sum
+    over the value channels is a dense product:
+      dU = M^T dO + Kend dSn,  Y = (I + A)^{-T} dU,  dV = diag(beta) Y,
+      dS = Diag(gamma) dSn + Qt^T dO - Kt^T dV,
+      dM = tril(dO U^T),  dA = -StrictLower(Y U^T),  dP = diag(beta) dA,
+      dQt = dO S^T + dM Kh,  dKt = -diag(beta) Y S^T + dP Kh,  dKh = dM^T Qt + dP^T Kt,
+      dKend = U dSn^T,  dgamma = rowsum(dSn * S),  dbeta = rowsum(R * Y) + rowsum(dA * Kt Kh^T).
+    (From Tb = Tm diag(beta) and U = Tb R: Tm^T dTm Tm^T = Y U^T and sum_i dTb_ij Tm_ij =
+    sum_v R_jv Y_jv.)"""
+    L = q.shape[0]
+    g = np.cumsum(la, axis=0)
+    E = np.exp(g)
+    Kt, Kh, Qt = k * E, k / E, q * E
+    gam = E[L - 1]
+    Kend = Kh * gam[None, :]
+    P = Kt @ Kh.T
+    A = np.tril(be[:, None] * P, -1)
+    M = np.tril(Qt @ Kh.T)
+    R = v - Kt @ S
+    U = np.linalg.solve(np.eye(L) + A, be[:, None] * R)
+    dU = M.T @ dO + Kend @ dSn
+    Y = np.linalg.solve((np.eye(L) + A).T, dU)
+    dv = be[:, None] * Y
+    dS = gam[:, None] * dSn + Qt.T @ dO - Kt.T @ dv
+    dM = np.tril(dO @ U.T)
+    dA = -np.tril(Y @ U.T, -1)
+    dP = be[:, None] * dA
+    dQt = dO @ S.T + dM @ Kh
+    dKt = -be[:, None] * (Y @ S.T) + dP @ Kh
+    dKh = dM.T @ Qt + dP.T @ Kt
+    dKend = U @ dSn.T
+    dgam = np.sum(dSn * S, axis=1)
+    dbe = np.sum(R * Y, axis=1) + np.sum(dA * P, axis=1)
+    dq = dQt * E
+    dk = dKt * E + (dKh + dKend * gam[None, :]) / E
+    dg = dQt * Qt + dKt * Kt - dKh * Kh - dKend * Kend
+    dg[L - 1] += np.sum(dKend * Kend, axis=0) + dgam * gam
+    dla = np.cumsum(dg[::-1], axis=0)[::-1]
+    return dq, dk, dv, dla, dbe, dS
+
+
+def backward(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens=None, chunk=64,
+             regrouped=False):
     """The gradients of ``backward.backward`` (same arguments and result), computed chunk by
     chunk: a forward sweep keeps the state entering every chunk, then a reverse sweep over the
-    chunks carries the state gradient dS and differentiates each chunk on its own."""
+    chunks carries the state gradient dS and differentiates each chunk on its own (with
+    ``regrouped``, in the regrouped form of ``_chunk_backward_regrouped``)."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -170,8 +215,9 @@ def backward(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens=
                 S = _chunk(S, q[b, s:e, h], k[b, s:e, h], v[b, s:e, h], la[b, s:e, h], be[b, s:e, h])[1]
             dS = np.zeros((dk, dv)) if dS_final is None else np.array(dS_final[n, h], dtype=np.float64)
             for (s, e), Sc in zip(reversed(bounds), reversed(states)):
-                r = _chunk_backward(Sc, dS, dout[b, s:e, h], q[b, s:e, h], k[b, s:e, h], v[b, s:e, h],
-                                    la[b, s:e, h], be[b, s:e, h])
+                f = _chunk_backward_regrouped if regrouped else _chunk_backward
+                r = f(Sc, dS, dout[b, s:e, h], q[b, s:e, h], k[b, s:e, h], v[b, s:e, h],
+                      la[b, s:e, h], be[b, s:e, h])
                 res["dq"][b, s:e, h], res["dk"][b, s:e, h], res["dv"][b, s:e, h] = r[0], r[1], r[2]
                 res["dlog_alpha"][b, s:e, h], res["dbeta"][b, s:e, h] = r[3], r[4]
                 dS = r[5]
