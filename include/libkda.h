@@ -25,6 +25,9 @@
  *    16-byte aligned; beta and cu_seqlens 4-byte aligned. A misaligned or
  *    NULL required pointer returns KDA_ERR_INVALID_ARG before any launch.
  *  - Only d_k = d_v = 128 is implemented; other sizes return KDA_ERR_UNSUPPORTED.
+ *  - The chunked calls (prefill, its passes, its backward) take at most 65535 heads
+ *    and 65535 sequences (one launch-grid dimension each); more return
+ *    KDA_ERR_UNSUPPORTED. The decode step takes any N x H below 2^31.
  *  - q and k are expected to be L2-normalised per head (a precondition of the
  *    layer, not applied here). log_alpha must be finite and <= 0, beta in [0, 1];
  *    neither is checked. The chunked prefill additionally needs the cumulative

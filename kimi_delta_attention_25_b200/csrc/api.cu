@@ -58,6 +58,7 @@ kda_status_t check_prefill(const void *q, const void *k, const void *v, const fl
     if (out_dtype != KDA_F32 && out_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || H <= 0 || N < 0) return KDA_ERR_INVALID_ARG;
     if (dk != kHeadDim || dv != kHeadDim) return KDA_ERR_UNSUPPORTED;
+    if (H > kMaxGridDim || N > kMaxGridDim) return KDA_ERR_UNSUPPORTED;
     if (cu_seqlens) {
         if (B != 1) return KDA_ERR_INVALID_ARG;
         if (!aligned(cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
@@ -179,6 +180,7 @@ kda_status_t chunk_bwd_impl(unsigned phases, const void *q, const void *k, const
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || H <= 0 || N < 0) return KDA_ERR_INVALID_ARG;
     if (dk != kHeadDim || dv != kHeadDim) return KDA_ERR_UNSUPPORTED;
+    if (H > kMaxGridDim || N > kMaxGridDim) return KDA_ERR_UNSUPPORTED;
     if (cu_seqlens) {
         if (B != 1 || !aligned(cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
     } else if (N != B) {

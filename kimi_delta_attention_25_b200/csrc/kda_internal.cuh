@@ -12,6 +12,8 @@ namespace kda {
 constexpr int kHeadDim = 128;   // d_k = d_v supported by every kernel
 constexpr int kChunk = 64;      // chunk length of the prefill (tokens)
 constexpr size_t kStatusBytes = 256;  // workspace prefix holding the device status word
+constexpr int kMaxGridDim = 65535;    // heads and sequences index grid dimensions y and z of the
+                                      // chunked kernels
 
 // Two-pass bf16 prefill: per (chunk slot, head) block of prepared operands in the workspace,
 // laid out as the scan pass wants them in shared memory (see chunk_prep.cu). The first 66048 bytes

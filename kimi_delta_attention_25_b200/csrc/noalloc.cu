@@ -64,6 +64,7 @@ extern "C" kda_status_t kda_chunk_fwd_noalloc(const void *q, const void *k, cons
     if (out_dtype != KDA_F32 && out_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || H <= 0 || N < 0) return KDA_ERR_INVALID_ARG;
     if (dk != kHeadDim || dv != kHeadDim) return KDA_ERR_UNSUPPORTED;
+    if (H > kMaxGridDim || N > kMaxGridDim) return KDA_ERR_UNSUPPORTED;
     if (cu_seqlens) {
         if (B != 1 || !aligned_to(cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
     } else if (N != B) {

@@ -194,3 +194,21 @@ def test_backward_phase_host_checks(lib):
     assert f(1, *args, P(FAKE), 256, None) == kda.KDA_ERR_INVALID_ARG      # workspace too small
     args[19] = 64                                                           # dk
     assert f(2, *args, P(FAKE), 1 << 30, None) == kda.KDA_ERR_UNSUPPORTED
+
+
+def test_chunked_calls_refuse_more_heads_or_sequences_than_a_grid_dimension(lib):
+    """Heads and sequences index launch-grid dimensions (at most 65535 each): more is refused on
+    the host, before any launch."""
+    assert _chunk(lib, H=65536) == kda.KDA_ERR_UNSUPPORTED
+    assert _chunk(lib, B=65536, N=65536) == kda.KDA_ERR_UNSUPPORTED
+    assert _chunk(lib, B=1, N=70000, cu=FAKE) == kda.KDA_ERR_UNSUPPORTED
+    assert _prep(lib, H=70000) == kda.KDA_ERR_UNSUPPORTED
+    assert _scan(lib, H=70000) == kda.KDA_ERR_UNSUPPORTED
+    assert _bwd(lib, H=65536) == kda.KDA_ERR_UNSUPPORTED
+    assert _bwd(lib, B=1, N=65536, cu=FAKE) == kda.KDA_ERR_UNSUPPORTED
+    P = ctypes.c_void_p
+    f = lib.kda_chunk_fwd_noalloc
+    assert f(*[P(FAKE)] * 5, None, None, P(FAKE), None, 1, 64, 65536, 1, 128, 128, 1, 0, None) == \
+        kda.KDA_ERR_UNSUPPORTED
+    # the limit itself is accepted by the host checks (this call then stops at its workspace)
+    assert _chunk(lib, H=65535) == kda.KDA_ERR_INVALID_ARG
