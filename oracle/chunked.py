@@ -184,12 +184,59 @@ def _chunk_backward_regrouped(S, dSn, dO, q, k, v, la, be):
     return dq, dk, dv, dla, dbe, dS
 
 
+def _chunk_backward_scan_form(S, dSn, dO, q, k, v, la, be):
+    """The regrouped gradients with the serial part in the shape of the forward's state scan: every
+    state-independent product is formed ahead (Tm = (I + A)^{-1} explicitly), so that only two
+    products per chunk involve the carried state gradient dSn --
+      seeds (no dSn):  Y0 = Tm^T M^T dO,   G0 = Qt^T dO
+      operands:        Kp = Tm^T Kend,     Bk = diag(beta) Kt
+      chain:           Y = Y0 + Kp dSn,    dS = Diag(gamma) dSn + G0 - Bk^T Y
+    (from dU = M^T dO + Kend dSn and Y = Tm^T dU) -- mirroring U = Tb V - W S and
+    S' = Diag(gamma) S + Kend^T U forward. The rest is as ``_chunk_backward_regrouped``."""
+    L = q.shape[0]
+    g = np.cumsum(la, axis=0)
+    E = np.exp(g)
+    Kt, Kh, Qt = k * E, k / E, q * E
+    gam = E[L - 1]
+    Kend = Kh * gam[None, :]
+    P = Kt @ Kh.T
+    Tm = np.linalg.inv(np.eye(L) + np.tril(be[:, None] * P, -1))
+    M = np.tril(Qt @ Kh.T)
+    Kp, Bk = Tm.T @ Kend, be[:, None] * Kt
+    Y0, G0 = Tm.T @ (M.T @ dO), Qt.T @ dO
+    Y = Y0 + Kp @ dSn
+    dS = gam[:, None] * dSn + G0 - Bk.T @ Y
+    R = v - Kt @ S
+    U = Tm @ (be[:, None] * R)
+    dv = be[:, None] * Y
+    dM = np.tril(dO @ U.T)
+    dA = -np.tril(Y @ U.T, -1)
+    dP = be[:, None] * dA
+    dQt = dO @ S.T + dM @ Kh
+    dKt = -be[:, None] * (Y @ S.T) + dP @ Kh
+    dKh = dM.T @ Qt + dP.T @ Kt
+    dKend = U @ dSn.T
+    dgam = np.sum(dSn * S, axis=1)
+    dbe = np.sum(R * Y, axis=1) + np.sum(dA * P, axis=1)
+    dq = dQt * E
+    dk = dKt * E + (dKh + dKend * gam[None, :]) / E
+    dg = dQt * Qt + dKt * Kt - dKh * Kh - dKend * Kend
+    dg[L - 1] += np.sum(dKend * Kend, axis=0) + dgam * gam
+    dla = np.cumsum(dg[::-1], axis=0)[::-1]
+    return dq, dk, dv, dla, dbe, dS
+
+
+_BACKWARD_FORMS = {"plain": "_chunk_backward", "regrouped": "_chunk_backward_regrouped",
+                   "scan": "_chunk_backward_scan_form"}
+
+
 def backward(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens=None, chunk=64,
-             regrouped=False):
+             form="plain"):
     """The gradients of ``backward.backward`` (same arguments and result), computed chunk by
     chunk: a forward sweep keeps the state entering every chunk, then a reverse sweep over the
-    chunks carries the state gradient dS and differentiates each chunk on its own (with
-    ``regrouped``, in the regrouped form of ``_chunk_backward_regrouped``)."""
+    chunks carries the state gradient dS and differentiates each chunk on its own. ``form`` picks
+    the per-chunk algebra: "plain" (chain rule line by line), "regrouped" (the current GPU
+    backward's) or "scan" (the state-gradient scan in the forward scan's shape)."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -215,7 +262,7 @@ def backward(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens=
                 S = _chunk(S, q[b, s:e, h], k[b, s:e, h], v[b, s:e, h], la[b, s:e, h], be[b, s:e, h])[1]
             dS = np.zeros((dk, dv)) if dS_final is None else np.array(dS_final[n, h], dtype=np.float64)
             for (s, e), Sc in zip(reversed(bounds), reversed(states)):
-                f = _chunk_backward_regrouped if regrouped else _chunk_backward
+                f = globals()[_BACKWARD_FORMS[form]]
                 r = f(Sc, dS, dout[b, s:e, h], q[b, s:e, h], k[b, s:e, h], v[b, s:e, h],
                       la[b, s:e, h], be[b, s:e, h])
                 res["dq"][b, s:e, h], res["dk"][b, s:e, h], res["dv"][b, s:e, h] = r[0], r[1], r[2]

@@ -215,19 +215,19 @@ def test_pins_reject_planted_slips(slip, monkeypatch):
         test_backward_equals_exact_directional_derivatives_on_the_golden_inputs()
 
 
-@pytest.mark.parametrize("regrouped", [False, True])
+@pytest.mark.parametrize("form", ["plain", "regrouped", "scan"])
 @pytest.mark.parametrize("T,d,C,cu", [(1, 8, 64, None), (130, 16, 64, None), (200, 32, 64, [0, 70, 70, 200]),
                                       (37, 8, 8, None)])
-def test_chunked_backward_equals_token_backward(T, d, C, cu, regrouped):
-    """The chunk-form gradients, plain and regrouped (the regrouped form is the algebra the GPU
-    backward follows), equal the token-level reverse sweep, across chunk boundaries, a ragged
-    tail and an empty sequence."""
+def test_chunked_backward_equals_token_backward(T, d, C, cu, form):
+    """The chunk-form gradients -- plain, regrouped (the algebra the GPU backward follows) and in
+    the scan shape (two state products per chunk) -- equal the token-level reverse sweep, across
+    chunk boundaries, a ragged tail and an empty sequence."""
     from oracle import chunked
     x, dout, dSf = _inputs(1, T, 2, d, d - 3, seed=T, n_seqs=cu)
     a = bw.backward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], dout, S0=x["S0"], dS_final=dSf,
                     cu_seqlens=cu)
     b = chunked.backward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], dout, S0=x["S0"], dS_final=dSf,
-                         cu_seqlens=cu, chunk=C, regrouped=regrouped)
+                         cu_seqlens=cu, chunk=C, form=form)
     for key in a:
         assert rel_err(b[key], a[key]) < 1e-12, key
 
