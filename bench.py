@@ -196,27 +196,27 @@ def time_loop(fn, steps, warmup, ws):
 
 # ---------------------------------------------------------------------------------------------
 
-def cpu_oracle_sample(budget_s=12.0):
-    """Times the float64 oracle (as it stands) on a bounded sample of the prefill workload:
+def cpu_oracle_sample(budget_s=12.0, workload=WORKLOAD):
+    """Times the float64 oracle (as it stands) on a bounded sample of a prefill workload:
     the first T' tokens of H' heads, with T' sized from a short calibration run so that the
     whole sample takes about `budget_s` seconds on all host cores. Returns a dict in Mtok/s."""
     from oracle import ref
     cores = ref.online_cores()
-    w = K.WORKLOADS[WORKLOAD]
+    w = K.WORKLOADS[workload]
     Hs = w.H
     cal_T = 1024
-    d = K.make_prefill(w, T=cal_T, H=1)
-    args = [d[x].float().numpy() for x in ("q", "k", "v", "log_alpha", "beta")]
-    t0 = time.perf_counter()
-    ref.forward(*args, S0=d["S0"].double().numpy(), nthreads=1)
-    per_tok_head = (time.perf_counter() - t0) / cal_T
+    def run(d, nthreads):
+        args = [d[x].float().numpy() for x in ("q", "k", "v", "log_alpha", "beta")]
+        S0 = None if d["S0"] is None else d["S0"].double().numpy()
+        cu = None if d["cu_seqlens"] is None else d["cu_seqlens"].numpy()
+        t0 = time.perf_counter()
+        ref.forward(*args, S0=S0, cu_seqlens=cu, nthreads=nthreads)
+        return time.perf_counter() - t0
+
+    per_tok_head = run(K.make_prefill(w, T=cal_T, H=1), 1) / cal_T
     Ts = int(max(1024, min(w.T, budget_s / per_tok_head * min(Hs, cores) / Hs)))
     Ts -= Ts % C
-    d = K.make_prefill(w, T=Ts, H=Hs)
-    args = [d[x].float().numpy() for x in ("q", "k", "v", "log_alpha", "beta")]
-    t0 = time.perf_counter()
-    ref.forward(*args, S0=d["S0"].double().numpy(), nthreads=min(Hs, cores))
-    dt = time.perf_counter() - t0
+    dt = run(K.make_prefill(w, T=Ts, H=Hs), min(Hs, cores))
     tok_equiv = Ts * Hs / w.H                 # tokens of the full 32-head workload
     return {"value": tok_equiv / dt / 1e6, "unit": "Mtok/s", "cores": min(Hs, cores),
             "kind": "oracle",
@@ -364,12 +364,16 @@ def run_native(args):
     e2e_val = ws * tokens / (ms_e2e * 1e-3) / 1e6
     del host, dbuf, h_out, h_sf
 
+    # ---- the other prefill workloads: 8K tokens x 16 heads, and 8 packed sequences (262K tokens)
+    del work
+    torch.cuda.empty_cache()
+    other = {name: run_prefill_config(kda, dev, pk, ws, rank, args, name, 6.0)
+             for name in ("bf16_t8k_h16", "bf16_varlen8_262k_h32")}
+
     # ---- decode step
     dec = run_decode(kda, dev, pk, ws, local, args)
 
     # ---- backward of the same prefill
-    del work
-    torch.cuda.empty_cache()
     bwd = run_backward(kda, dev, pk, ws, local, args, d)
 
     del d, out
@@ -400,6 +404,7 @@ def run_native(args):
                     "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
             "gpu_launches": args.steps * PREFILL_KERNELS_PER_STEP,
             "clocks": clk.summary(),
+            "configs": other,
             "decode": dec,
             "backward": bwd,
             "cpu_baseline": cpu,
@@ -407,6 +412,73 @@ def run_native(args):
         print(json.dumps(line), flush=True)
     if ws > 1:
         torch.distributed.destroy_process_group()
+
+
+def run_prefill_config(kda, dev, pk, ws, rank, args, name, cpu_budget_s):
+    """One more prefill workload (two passes, bf16 outputs), timed like the headline step: Mtok/s,
+    the roofline of each pass and of the step, and the oracle on a bounded sample of it."""
+    from kimi_delta_attention_25_b200 import shard
+    w = K.WORKLOADS[name]
+    d = K.make_prefill(w, device=dev, seed=shard.rank_seed(w.seed, rank))
+    B, T, H = w.B, w.T, w.H
+    cu = d.get("cu_seqlens")
+    N = B if cu is None else cu.shape[0] - 1
+    if cu is not None:
+        cu = cu.to(dev)
+    out = torch.empty(B, T, H, D, dtype=torch.bfloat16, device=dev)
+    Sf = torch.empty(N, H, D, D, dtype=torch.float32, device=dev)
+    work = torch.empty(max(256, kda.chunk_fwd_workspace_size(B, T, H, N)), dtype=torch.uint8, device=dev)
+    steps = max(3, args.steps)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+
+    def passes(ev=None):
+        if ev is not None:
+            ev[0].record()
+        kda.chunk_prep(d["q"], d["k"], d["log_alpha"], d["beta"], work, cu_seqlens=cu)
+        if ev is not None:
+            ev[1].record()
+        kda.chunk_scan(d["v"], work, S0=d["S0"], cu_seqlens=cu, out=out, S_final=Sf)
+        if ev is not None:
+            ev[2].record()
+
+    with Clocks(int(os.environ.get("LOCAL_RANK", "0"))) as clk:
+        for _ in range(args.warmup):
+            passes()
+        torch.cuda.synchronize()
+        barrier(ws)
+        torch.cuda.synchronize()
+        t_s, t_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t_s.record()
+        for i in range(steps):
+            passes(evs[i])
+        t_e.record()
+        torch.cuda.synchronize()
+        barrier(ws)
+    assert kda.workspace_status(work) == kda.KDA_OK
+    ms = max_over_ranks(t_s.elapsed_time(t_e) / steps, ws)
+    th = B * T * H
+    kern = {}
+    for i, (kname, per) in enumerate((("chunk_prep", PREP_BYTES_PER_TOKEN_HEAD),
+                                      ("chunk_scan", SCAN_BYTES_PER_TOKEN_HEAD))):
+        t_ms = statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+        a = th * per / (t_ms * 1e-3) / 1e9
+        kern[kname] = {"ms": t_ms, "achieved": a, "frac": a / pk["hbm"]}
+    gbs = th * PREFILL_BYTES_PER_TOKEN_HEAD / (ms * 1e-3) / 1e9
+    tfs = th * PREFILL_FLOPS_PER_TOKEN_HEAD / (ms * 1e-3) / 1e12
+    res = {"workload": name, "tokens": B * T, "heads": H, "sequences": N, "ms_per_step": ms,
+           "Mtok_s": ws * B * T / (ms * 1e-3) / 1e6, "steps": steps, "out": "bf16",
+           "l2": "inputs %.2f GB per step (%s L2)" % (th * PREFILL_BYTES_PER_TOKEN_HEAD / 1e9,
+                                                      "larger than" if th * 1540 > 126e6 else "within"),
+           "roofline": {"bound": "hbm", "peak": pk["hbm"], "unit": "GB/s", "peak_source": "of %s" % pk["src"],
+                        "kernels": kern,
+                        "step": {"achieved": gbs, "frac": gbs / pk["hbm"], "tensor_tflops_useful": tfs,
+                                 "tensor_frac_useful": tfs / pk["bf16"]}},
+           "gpu_launches": 2 * steps, "clocks": clk.summary()}
+    del d, out, Sf, work
+    torch.cuda.empty_cache()
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_oracle_sample(budget_s=cpu_budget_s, workload=name)
+    return res
 
 
 def run_decode(kda, dev, pk, ws, local, args):
@@ -470,8 +542,7 @@ def run_backward(kda, dev, pk, ws, local, args, d):
     dSf = torch.randn(B, H, D, D, generator=g, device=dev)
     args_ = (d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], dout)
     kw = dict(S0=d["S0"], dS_final=dSf)
-    grads = kda.chunk_bwd(*args_, **kw)
-    work = kda.chunk_bwd.last_workspace
+    grads, work = kda.chunk_bwd(*args_, **kw, return_workspace=True)
     torch.cuda.synchronize()
     assert kda.workspace_status(work) == kda.KDA_OK
     steps = max(1, min(args.steps, 3))
@@ -537,19 +608,20 @@ def run_profile_case(args):
         w = K.WORKLOADS[WORKLOAD]
         d = K.make_prefill(w, device=dev, T=args.tokens)
         for _ in range(2):
-            kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"],
-                          out_dtype=torch.bfloat16)
+            ws = kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"],
+                               out_dtype=torch.bfloat16, return_workspace=True)[2]
         torch.cuda.synchronize()
-        assert kda.workspace_status(kda.chunk_fwd.last_workspace) == kda.KDA_OK
+        assert kda.workspace_status(ws) == kda.KDA_OK
     elif args.profile == "backward":
         w = K.WORKLOADS[WORKLOAD]
         d = K.make_prefill(w, device=dev, T=args.tokens)
         g = torch.Generator(device=dev).manual_seed(1234)
         dout = torch.randn(d["v"].shape, generator=g, device=dev).to(torch.bfloat16)
         for _ in range(2):
-            kda.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], dout, S0=d["S0"])
+            _, ws = kda.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], dout, S0=d["S0"],
+                                  return_workspace=True)
         torch.cuda.synchronize()
-        assert kda.workspace_status(kda.chunk_bwd.last_workspace) == kda.KDA_OK
+        assert kda.workspace_status(ws) == kda.KDA_OK
     else:
         w = K.WORKLOADS[DECODE]
         S = K.make_decode_state(w, device=dev)

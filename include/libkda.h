@@ -30,9 +30,14 @@
  *    KDA_ERR_UNSUPPORTED. The decode step takes any N x H below 2^31.
  *  - q and k are expected to be L2-normalised per head (a precondition of the
  *    layer, not applied here). log_alpha must be finite and <= 0, beta in [0, 1];
- *    neither is checked. The chunked prefill additionally needs the cumulative
- *    log-decay inside one 64-token chunk to stay above -80 per channel
- *    (exp of its negation must be finite in fp32); the decode step has no such limit.
+ *    neither is checked. The chunked prefill (kda_chunk_fwd, its passes and its
+ *    backward, for either input dtype) additionally needs the cumulative log-decay
+ *    inside one 64-token chunk to stay at or above -80 per channel (exp of its
+ *    negation must be finite in fp32). That check needs device data, so the call
+ *    returns KDA_OK and a chunk outside the range writes KDA_ERR_UNSUPPORTED to the
+ *    workspace status word (read it with kda_workspace_status); the outputs of such a
+ *    call are not usable. kda_chunk_fwd_noalloc with bf16 inputs has a narrower range
+ *    (see there). The decode step has no such limit.
  *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
  *    legacy default stream). A KDA_ERR_CUDA return means a launch failed.
  *  - Calls are thread-safe; concurrent calls must not share output buffers
@@ -52,9 +57,13 @@ extern "C" {
 typedef enum {
     KDA_OK = 0,
     KDA_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or cu_seqlens content */
-    KDA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (d_k, d_v != 128) */
+    KDA_ERR_UNSUPPORTED = 2,   /* valid but not implemented: d_k, d_v != 128, more heads or
+                                * sequences than a launch grid holds, or (in a status word)
+                                * a chunk whose decay is outside the supported range */
     KDA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
-    KDA_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up */
+    KDA_ERR_TIMEOUT = 4,       /* a bounded device-side wait gave up */
+    KDA_ERR_BOUNDS = 5         /* debug builds only (libkda_debug.so): a kernel computed a global
+                                * index outside its buffer and skipped that access */
 } kda_status_t;
 
 typedef enum {
@@ -219,18 +228,29 @@ kda_status_t kda_decode_step(const void *q, const void *k, const void *v,
  * current) and caches it; make that first call before any stream capture begins. bf16 inputs run
  * the single-kernel prefill, whose only scratch is the 256-byte status header (a scratch need
  * beyond the array would be refused with KDA_ERR_UNSUPPORTED); it is slower than the two-pass
- * prefill kda_chunk_fwd runs with its workspace. The function calls no cudaMalloc, cudaFree or
- * other allocating routine.
+ * prefill kda_chunk_fwd runs with its workspace, and its f16 tensor-core operands narrow the
+ * decay range: the cumulative log-decay inside one 64-token chunk must stay at or above -9.0 per
+ * channel (fp32 inputs keep the -80 of kda_chunk_fwd). The function calls no cudaMalloc, cudaFree
+ * or other allocating routine.
  * The array is shared by every call and keeps the last call's contents; each call clears its
  * status header first. Calls whose work overlaps on the GPU (for example on two streams) race
  * on that shared array: serialise them. Device-side check results (cu_seqlens contents, the
- * tensor-core decay range) are written to that shared status header and are not returned. */
+ * decay range) are written to that shared status header; read them back with
+ * kda_chunk_fwd_noalloc_status. */
 kda_status_t kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
                                    const float *log_alpha, const float *beta,
                                    const float *S0, const int32_t *cu_seqlens,
                                    void *out, float *S_final,
                                    int B, int T, int H, int N, int dk, int dv,
                                    kda_dtype_t dtype, kda_dtype_t out_dtype, void *stream);
+
+/* Waits for `stream`, then copies the status word of the shared scratch array of
+ * kda_chunk_fwd_noalloc on the current device to *status: KDA_OK when every device-side check
+ * of the last kda_chunk_fwd_noalloc call on this device passed, else the first failure
+ * (KDA_ERR_INVALID_ARG for inconsistent cu_seqlens contents, KDA_ERR_UNSUPPORTED for a decay
+ * outside the range, KDA_ERR_TIMEOUT for a device wait that gave up). The pages have no
+ * counterpart. Allocates nothing. Errors: KDA_ERR_INVALID_ARG (status NULL), KDA_ERR_CUDA. */
+kda_status_t kda_chunk_fwd_noalloc_status(void *stream, int32_t *status);
 
 /* Self-test of the library's failure detection (the pages have no counterpart): every device-side
  * wait of the kernels (on an mbarrier or a copy) is bounded and, when it runs out, records

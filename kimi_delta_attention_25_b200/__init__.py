@@ -22,21 +22,25 @@ from typing import Optional
 import torch
 
 __all__ = ["chunk_fwd", "chunk_prep", "chunk_scan", "decode_step", "chunk_fwd_workspace_size", "workspace_status",
-           "status_string", "library_path", "load", "KDAError",
+           "status_string", "library_path", "load", "KDAError", "cu_seqlens_from_mask", "unpad", "pad",
+           "chunk_fwd_noalloc", "noalloc_status",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA", "KDA_ERR_TIMEOUT"]
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
 KDA_F32, KDA_BF16 = 0, 1
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-library_path = os.path.join(_PKG, "libkda.so")
+# KDA_LIBRARY selects another build of the same ABI (the debug build libkda_debug.so, which checks
+# every global index); by default the release build next to this file.
+library_path = os.environ.get("KDA_LIBRARY") or os.path.join(_PKG, "libkda.so")
 _lib = None
 
 # Every entry point declared in include/libkda.h.
 EXPORTS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
            "kda_workspace_status", "kda_status_string", "kda_version", "kda_chunk_fwd_noalloc",
            "kda_chunk_prep", "kda_chunk_scan", "kda_selftest_wait_timeout",
-           "kda_chunk_bwd_workspace_size", "kda_chunk_bwd", "kda_chunk_bwd_phase")
+           "kda_chunk_bwd_workspace_size", "kda_chunk_bwd", "kda_chunk_bwd_phase",
+           "kda_chunk_fwd_noalloc_status")
 
 
 class KDAError(RuntimeError):
@@ -68,6 +72,8 @@ def load():
     lib.kda_version.restype = I
     lib.kda_chunk_fwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P]
     lib.kda_chunk_fwd_noalloc.restype = I
+    lib.kda_chunk_fwd_noalloc_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
+    lib.kda_chunk_fwd_noalloc_status.restype = I
     lib.kda_chunk_prep.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, Z, P]
     lib.kda_chunk_prep.restype = I
     lib.kda_chunk_scan.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, Z, P]
@@ -118,11 +124,14 @@ def chunk_fwd_workspace_size(B, T, H, N, dk=128, dv=128, dtype=torch.bfloat16) -
 
 
 def chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, S_final=None,
-              workspace=None, want_state=True, out_dtype=torch.float32):
+              workspace=None, want_state=True, out_dtype=torch.float32, return_workspace=False):
     """Chunkwise KDA prefill. Shapes: q, k, log_alpha [B,T,H,dk]; v [B,T,H,dv];
     beta [B,T,H]; S0 [N,H,dk,dv] fp32 or None; cu_seqlens int32 [N+1] or None.
     Returns (out [B,T,H,dv] in out_dtype (or the dtype of a given ``out``),
-    S_final [N,H,dk,dv] fp32 or None)."""
+    S_final [N,H,dk,dv] fp32 or None), and the workspace as a third element when
+    ``return_workspace`` (its status word holds the device-side checks: ``workspace_status``).
+    Without a ``workspace`` argument each call takes a fresh one from torch's caching allocator
+    (about 1 KiB per token and head for bf16 inputs); a caller that runs many calls passes its own."""
     lib = load()
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -143,8 +152,7 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, S_fi
                            _dtype_code(out), _ptr(workspace), workspace.numel(), _stream(q.device))
     if st != KDA_OK:
         raise KDAError(st, "kda_chunk_fwd")
-    chunk_fwd.last_workspace = workspace
-    return out, S_final
+    return (out, S_final, workspace) if return_workspace else (out, S_final)
 
 
 def chunk_prep(q, k, log_alpha, beta, workspace, cu_seqlens=None):
@@ -190,13 +198,14 @@ def chunk_bwd_workspace_size(B, T, H, N, dk=128, dv=128) -> int:
 
 
 def chunk_bwd(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens=None,
-              want_dS0=True, grads=None, workspace=None, phase=None):
+              want_dS0=True, grads=None, workspace=None, phase=None, return_workspace=False):
     """``kda_chunk_bwd``: gradients of a loss with gradients ``dout`` (w.r.t. every output, dtype of
     q) and ``dS_final`` (w.r.t. the final states, fp32 or None) through ``chunk_fwd`` with the same
     inputs. Returns a dict of fp32 tensors dq, dk, dv, dlog_alpha, dbeta and dS0 (None unless
     ``want_dS0``). ``grads`` may supply those tensors (same keys) to be written in place.
     ``phase`` (0, 1 or 2) runs one of the three kernels only (``kda_chunk_bwd_phase``); the phases
-    must then run in order on the same ``grads`` and ``workspace``."""
+    must then run in order on the same ``grads`` and ``workspace``. With ``return_workspace`` the
+    result is ``(grads, workspace)``."""
     lib = load()
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -234,8 +243,7 @@ def chunk_bwd(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens
         st = lib.kda_chunk_bwd_phase(int(phase), *args)
     if st != KDA_OK:
         raise KDAError(st, "kda_chunk_bwd")
-    chunk_bwd.last_workspace = workspace
-    return g
+    return (g, workspace) if return_workspace else g
 
 
 def selftest_wait_timeout(workspace: torch.Tensor, budget_cycles: int) -> None:
@@ -289,3 +297,48 @@ def chunk_fwd_noalloc(q, k, v, log_alpha, beta, out, S_final=None, S0=None, cu_s
     if st != KDA_OK:
         raise KDAError(st, "kda_chunk_fwd_noalloc")
     return out, S_final
+
+
+def noalloc_status(device=None) -> int:
+    """``kda_chunk_fwd_noalloc_status``: the device-side check result of the last
+    ``chunk_fwd_noalloc`` call on the current device (syncs the current stream)."""
+    v = ctypes.c_int32(0)
+    st = load().kda_chunk_fwd_noalloc_status(_stream(device), ctypes.byref(v))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_fwd_noalloc_status")
+    return int(v.value)
+
+
+# ---- padding-mask form -> packed sequences -------------------------------------------------------
+# The layer can receive a batch as a [batch, seq_len] 0/1 attention mask (1 = real token, 0 =
+# padding; the lpnh.cn Kimi Linear article, sec. 5, gives this form). libkda takes packed sequences
+# instead: the real tokens of every row one after another (B = 1) with cu_seqlens offsets. These
+# helpers only move data (index selects); every step of the computation runs in libkda.
+
+def cu_seqlens_from_mask(mask: torch.Tensor):
+    """``mask`` [B, T] of 0/1 (bool or integer). Returns ``(cu_seqlens, indices)``: int32 [B+1]
+    offsets of each row's real tokens in the packed order, and int64 [total] flat indices
+    (row * T + t) of those tokens, in row order and, within a row, in token order. Padding may sit
+    anywhere in a row (left, right or between tokens); its positions are dropped."""
+    if mask.dim() != 2:
+        raise ValueError("mask must be [batch, seq_len]")
+    m = mask.to(torch.bool)
+    lens = m.sum(dim=1, dtype=torch.int64)
+    cu = torch.zeros(m.shape[0] + 1, dtype=torch.int64, device=m.device)
+    cu[1:] = torch.cumsum(lens, 0)
+    indices = torch.nonzero(m.reshape(-1), as_tuple=False).reshape(-1)
+    return cu.to(torch.int32), indices
+
+
+def unpad(x: torch.Tensor, indices: torch.Tensor) -> torch.Tensor:
+    """[B, T, ...] -> [1, total, ...]: the real tokens (``indices`` from ``cu_seqlens_from_mask``)
+    packed in order, contiguous, ready for ``chunk_fwd(..., cu_seqlens=...)``."""
+    B, T = x.shape[:2]
+    return x.reshape(B * T, *x.shape[2:]).index_select(0, indices).unsqueeze(0).contiguous()
+
+
+def pad(y: torch.Tensor, indices: torch.Tensor, B: int, T: int, fill: float = 0.0) -> torch.Tensor:
+    """Inverse of ``unpad``: [1, total, ...] -> [B, T, ...] with ``fill`` at the padding positions."""
+    flat = torch.full((B * T, *y.shape[2:]), fill, dtype=y.dtype, device=y.device)
+    flat.index_copy_(0, indices, y.reshape(-1, *y.shape[2:]))
+    return flat.reshape(B, T, *y.shape[2:])

@@ -3,7 +3,11 @@
 Usage: ``python -m kimi_delta_attention_25_b200.build [--force] [--debug]``.
 Each translation unit is compiled in parallel to ``_build/*.o`` and linked into
 ``kimi_delta_attention_25_b200/libkda.so`` (CUDA runtime linked statically, so
-the library needs only the driver at run time).
+the library needs only the driver at run time). ``--debug`` builds
+``libkda_debug.so`` instead (objects in ``_build/debug``): the same kernels with
+``KDA_DEBUG=1``, which checks every global index against its buffer and records
+KDA_ERR_BOUNDS in the status word instead of making the access. Select it at run
+time with the environment variable ``KDA_LIBRARY``.
 """
 from __future__ import annotations
 
@@ -20,6 +24,7 @@ CSRC = os.path.join(PKG, "csrc")
 INC = os.path.join(ROOT, "include")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libkda.so")
+LIB_DEBUG = os.path.join(PKG, "libkda_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
@@ -40,15 +45,17 @@ def _deps_mtime() -> float:
 
 def build(force: bool = False, debug: bool = False, verbose: bool = False) -> str:
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _deps_mtime():
-        return LIB
-    os.makedirs(OBJ, exist_ok=True)
+    lib = LIB_DEBUG if debug else LIB
+    obj_dir = os.path.join(OBJ, "debug") if debug else OBJ
+    if not force and os.path.exists(lib) and os.path.getmtime(lib) >= _deps_mtime():
+        return lib
+    os.makedirs(obj_dir, exist_ok=True)
     extra = ["-DKDA_DEBUG=1"] if debug else []
     if verbose:
         extra += ["-Xptxas", "-v"]
 
     def compile_one(src):
-        obj = os.path.join(OBJ, os.path.basename(src) + ".o")
+        obj = os.path.join(obj_dir, os.path.basename(src) + ".o")
         cmd = [nvcc()] + ARCH + FLAGS + extra + ["-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
@@ -61,13 +68,13 @@ def build(force: bool = False, debug: bool = False, verbose: bool = False) -> st
         for _, log in results:
             print(log)
     objs = [o for o, _ in results]
-    tmp = LIB + ".tmp%d" % os.getpid()
+    tmp = lib + ".tmp%d" % os.getpid()
     cmd = [nvcc()] + ARCH + ["-shared", "-o", tmp] + objs + ["-lpthread"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("link failed:\n%s%s" % (r.stdout, r.stderr))
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 def main():

@@ -26,9 +26,10 @@ const char *kda_status_string(kda_status_t s)
     switch (s) {
     case KDA_OK: return "ok";
     case KDA_ERR_INVALID_ARG: return "invalid argument";
-    case KDA_ERR_UNSUPPORTED: return "unsupported size (only d_k = d_v = 128)";
+    case KDA_ERR_UNSUPPORTED: return "unsupported (size, or a decay outside the range)";
     case KDA_ERR_CUDA: return "CUDA error";
     case KDA_ERR_TIMEOUT: return "device wait timed out";
+    case KDA_ERR_BOUNDS: return "global index out of bounds (debug build)";
     }
     return "unknown status";
 }

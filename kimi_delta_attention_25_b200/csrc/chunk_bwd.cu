@@ -80,6 +80,7 @@ chunk_bwd_scan_kernel(BwdArgs a)
     if (!sequence_span(a.cu_seqlens, n, a.N, a.T, &t0, &t1, a.status)) return;
 
     const size_t sbase = ((size_t)n * H + h) * DK * DK;
+    if (!in_bounds(a.status, (long long)sbase, DK * DK, (long long)a.N * H * DK * DK)) return;
     for (int idx = tid; idx < DK * DVB; idx += NT_SCAN) {
         const int c = idx / DVB, j = idx % DVB;
         sm.dS[idx] = a.dS_final ? a.dS_final[sbase + (size_t)c * DK + j0 + j] : 0.f;
@@ -90,6 +91,9 @@ chunk_bwd_scan_kernel(BwdArgs a)
         const int64_t s = t0 + ci * C;
         const int L = (t1 - s < C) ? (int)(t1 - s) : C;
         const size_t rec = (size_t)h * a.n_slots + (size_t)chunk_slot(s, n);
+        if (!in_bounds(a.status, s, L, (long long)a.B * a.T) ||
+            !in_bounds(a.status, (long long)rec, 1, (long long)H * a.n_slots))
+            break;
         __syncthreads();
         // ---- load the chunk (k -> Kt, q -> Qt, log_alpha -> Kh, dO block) and record dS'
         fp32c::load_chunk<T, NT_SCAN>(sm.Kt, sm.Qt, sm.Kh, LD, sm.dO, q, k, a.log_alpha, dout, s, L, H, h, j0, tid);
@@ -103,6 +107,7 @@ chunk_bwd_scan_kernel(BwdArgs a)
             constexpr int RP = C / (NT_SCAN / DK);
             const int c = tid % DK, r0 = (tid / DK) * RP;
             if (tid < DK) sm.gam[c] = expf(gl);
+            if (tid < DK && !(gl >= kMinChunkLogDecay)) set_status(a.status, KDA_ERR_UNSUPPORTED);
 #pragma unroll 4
             for (int r = r0; r < r0 + RP; ++r) {
                 const float gr = sm.Kh[r * LD + c];
@@ -235,6 +240,10 @@ chunk_bwd_local_kernel(BwdArgs a)
     int64_t s;
     if (!slot_to_chunk(a.cu_seqlens, a.N, a.T, slot, &n, &s, &L)) return;
     const size_t rec = (size_t)h * a.n_slots + (size_t)slot;
+    // every global access below lies in the token rows [s, s + L) and the (head, slot) records
+    if (!in_bounds(a.status, s, L, (long long)a.B * a.T) ||
+        !in_bounds(a.status, (long long)rec, 1, (long long)H * a.n_slots))
+        return;
     const T *q = (const T *)a.q;
     const T *k = (const T *)a.k;
     const T *dout = (const T *)a.dout;
@@ -252,6 +261,7 @@ chunk_bwd_local_kernel(BwdArgs a)
         constexpr int RP = C / (NT_LOC / DK);
         const int c = tid % DK, r0 = (tid / DK) * RP;
         if (tid < DK) sm.gam[c] = expf(gl);
+        if (tid < DK && !(gl >= kMinChunkLogDecay)) set_status(a.status, KDA_ERR_UNSUPPORTED);
 #pragma unroll 4
         for (int r = r0; r < r0 + RP; ++r) {
             const float g = sm.E[r * LD + c];

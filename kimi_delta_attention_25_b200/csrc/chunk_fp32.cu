@@ -66,8 +66,9 @@ chunk_fp32_kernel(PrefillArgs a)
     int64_t t0, t1;
     if (!sequence_span(a.cu_seqlens, n, a.N, a.T, &t0, &t1, a.status)) return;
 
-    // initial state block
+    // initial state block (every state access below stays inside this head's DK x DK block)
     const size_t sbase = ((size_t)n * H + h) * DK * DK;
+    if (!in_bounds(a.status, (long long)sbase, DK * DK, (long long)a.N * H * DK * DK)) return;
     for (int idx = tid; idx < DK * DVB; idx += NT) {
         const int c = idx / DVB, j = idx % DVB;
         sm.S[idx] = a.S0 ? a.S0[sbase + (size_t)c * DK + j0 + j] : 0.f;
@@ -75,6 +76,12 @@ chunk_fp32_kernel(PrefillArgs a)
 
     for (int64_t s = t0; s < t1; s += C) {
         const int L = (t1 - s < C) ? (int)(t1 - s) : C;
+        // every global access of this chunk lies in its token rows [s, s + L) and, for the records,
+        // in its (head, chunk slot) block
+        if (!in_bounds(a.status, s, L, (long long)a.B * a.T) ||
+            ((a.ck_S || a.ck_U) && !in_bounds(a.status, (long long)h * a.n_slots + chunk_slot(s, n), 1,
+                                                   (long long)H * a.n_slots)))
+            break;
         __syncthreads();
         // ---- load the chunk: k -> Kt, q -> Qt, log_alpha -> Kh, v block -> R
         fp32c::load_chunk<T, NT>(sm.Kt, sm.Qt, sm.Kh, LD, sm.R, q, k, a.log_alpha, v, s, L, H, h, j0, tid);
@@ -89,6 +96,8 @@ chunk_fp32_kernel(PrefillArgs a)
             const float gl = fp32c::decay_prefix<NT>(sm.Kh, LD, tid);
             const int c = tid % DK, part = tid / DK, r0 = part * (C / (NT / DK));
             if (part == 0) sm.gam[c] = expf(gl);
+            // e^{-g} must stay finite in fp32: outside the range the outputs are not usable
+            if (part == 0 && !(gl >= kMinChunkLogDecay)) set_status(a.status, KDA_ERR_UNSUPPORTED);
 #pragma unroll 4
             for (int r = r0; r < r0 + C / (NT / DK); ++r) {
                 const float gr = sm.Kh[r * LD + c];

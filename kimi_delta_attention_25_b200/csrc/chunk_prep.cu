@@ -39,9 +39,12 @@ constexpr int C = kChunk;
 constexpr int DK = kHeadDim;
 constexpr int NT = 256;
 
-// Operands are rounded to f16 for the tensor cores: Kh = K e^{-g} must stay finite, so the decay
-// accumulated over one chunk must keep e^{g} above 2^-15 per channel; beyond that UNSUPPORTED.
-constexpr float kMinChunkDecay = 3.0517578125e-05f;
+// The intra-chunk product P1 pairs Kt = K e^{g} with Kh = K e^{-g}: for a channel that forgets fast
+// within the chunk, e^{-g} exceeds the f16 range long before the product loses meaning. P1 therefore
+// runs on tf32 operands (fp32 range, the 10-bit significand of f16); every later product takes f16
+// operands, which only shrink toward zero there. e^{-g} must stay finite in fp32: the decay
+// accumulated over one chunk must keep e^{g} above e^{-80} per channel; beyond that UNSUPPORTED.
+constexpr float kMinChunkDecay = 1.80485139e-35f;   // e^{-80}
 
 // shared memory (1024-aligned base)
 constexpr uint32_t OFF_QK = 0;               // [Qt; Kt] (f16): per 64-channel half (16 KB apart),
@@ -49,7 +52,7 @@ constexpr uint32_t OFF_QK = 0;               // [Qt; Kt] (f16): per 64-channel h
 constexpr uint32_t QK_HALF = 16384;
 constexpr uint32_t OFF_KT = OFF_QK + 8192;   // Kt rows of half 0 (half 1 at + QK_HALF)
 constexpr uint32_t OFF_TB = 32768;           // Tb (f16), 64 x 128 B; N-block 0 of [Tb | W]
-constexpr uint32_t OFF_KH = 40960;           // Kh; after P1: A^T (fp32, column-major);
+constexpr uint32_t OFF_KH = 40960;           // after P1: A^T (fp32, column-major);
                                              // after P3: W (f16), N-blocks 1-2 of [Tb | W]
 constexpr uint32_t OFF_M = 57344;            // M (f16), 64 x 128 B
 // input staging of the chunk (bulk copies), dead once the rows are in registers: aliases the
@@ -57,13 +60,20 @@ constexpr uint32_t OFF_M = 57344;            // M (f16), 64 x 128 B
 constexpr uint32_t STG_Q = 0;                // q rows, 64 x 256 B
 constexpr uint32_t STG_K = 16384;            // k rows
 constexpr uint32_t STG_LA = 32768;           // log_alpha rows, 64 x 512 B
+// tf32 operands of P1, dead once P1 has completed (alias everything above and T): [Qt; Kt] as four
+// 32-channel quarters of 128 rows x 128 B (rows 0-63 Qt, 64-127 Kt), then Kh as four quarters of
+// 64 rows x 128 B; the f16 tiles above are written after P1 from registers
+constexpr uint32_t OFF_QK32 = 0;
+constexpr uint32_t OFF_KH32 = 65536;
 constexpr int LDT = 68;
 constexpr uint32_t OFF_TF = 65536;           // T (fp32, stride LDT) = 17408 B
-constexpr uint32_t OFF_PS = OFF_TF + 17408;  // 4 KB: row-block products, then inverse scratch
+constexpr uint32_t OFF_PS = 98304;           // 4 KB: row-block products, then inverse scratch
 constexpr uint32_t OFF_BET = OFF_PS + 4096;  // 64 fp32
 constexpr uint32_t OFF_BAR = OFF_BET + 256;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
+static_assert(OFF_KH32 + 4 * 8192 <= OFF_PS && OFF_TF + 17408 <= OFF_PS, "P1 operands and T end below Ps");
+static_assert(2 * (SMEM_ALLOC + 1024) <= 233472, "two CTAs per SM");
 
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t TM_D1A = 0;               // [Qt; Kt] Kh^T (M=128, 64 cols), later W (cols 0-127),
@@ -89,6 +99,7 @@ struct PrepParams {
     const int32_t *cu_seqlens;
     unsigned char *ws;              // chunk blocks, [H][n_slots][kPrepBlockBytes]
     int T, H, N, n_slots;
+    long long tokens;               // B * T (rows of q, k, log_alpha; beta has tokens * H entries)
     int prefetch_wave;              // CTAs resident at once; > 0: prefetch that many units ahead
     int32_t *status;
 };
@@ -230,6 +241,8 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
     int64_t tok0;
     int L;
     if (!slot_chunk(p, slot, &tok0, &L)) return;  // unused slot
+    // every workspace store below is at a constant offset below kPrepBlockBytes inside this block
+    if (!in_bounds(p.status, (long long)h * p.n_slots + slot, 1, (long long)H * p.n_slots)) return;
     unsigned char *blk = p.ws + ((size_t)h * p.n_slots + slot) * kPrepBlockBytes;
 
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
@@ -287,7 +300,10 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
             qr[x] = kr[x];
         }
     }
-    if (tid < C) bet[tid] = (tid < L) ? p.beta[(size_t)(tok0 + tid) * H + h] : 0.f;
+    if (tid < C) {
+        const long long bi = (long long)(tok0 + tid) * H + h;
+        bet[tid] = (tid < L && in_bounds(p.status, bi, 1, p.tokens * H)) ? p.beta[bi] : 0.f;
+    }
 
     // ---- decay scaling: per-thread products over its 8 rows, then over the 8 warps via smem
     float a[8][4], pre[8][4];
@@ -322,16 +338,18 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
     }
     // Workspace (global) stores of each phase are issued after that phase's proxy fence and MMA
     // issue: a fence.proxy.async would otherwise also wait for them to complete.
-    uint2 kend[8];
+    uint2 kend[8], okt8[8], oqt8[8];   // f16 Kend (to the workspace), Kt and Qt (tiles after P1)
     {
         float suf[4] = {1.f, 1.f, 1.f, 1.f};
+        const uint32_t qj = (uint32_t)(lane >> 3), ch16 = (uint32_t)(lane & 7);   // tf32 quarter, chunk
 #pragma unroll
         for (int x = 7; x >= 0; --x) {
             const int r = 8 * warp + x;
-            const uint32_t off = r * 128 + ((((lc4 >> 1) ^ (r & 7)) & 7) << 4) + ((lc4 & 1) << 3);
+            const uint32_t off32 = r * 128 + (((ch16 ^ (r & 7)) & 7) << 4);
             const uint32_t kw[2] = {kr[x].x, kr[x].y};
             const uint32_t qw[2] = {qr[x].x, qr[x].y};
-            uint32_t okt[2], oqt[2], oke[2], okh[2];
+            uint32_t okt[2], oqt[2], oke[2];
+            float kt4[4], qt4[4], kh4[4];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const int e = 2 * u;
@@ -340,17 +358,24 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
                 const float k0 = bf_lo(kw[u]), k1 = bf_hi(kw[u]);
                 const float q0 = bf_lo(qw[u]), q1 = bf_hi(qw[u]);
                 const float e0 = k0 * b0, e1 = k1 * b1;
-                okt[u] = pack_f16x2(k0 * f0, k1 * f1);
-                oqt[u] = pack_f16x2(q0 * f0, q1 * f1);
+                kt4[e] = k0 * f0; kt4[e + 1] = k1 * f1;
+                qt4[e] = q0 * f0; qt4[e + 1] = q1 * f1;
+                kh4[e] = e0 * rg[e]; kh4[e + 1] = e1 * rg[e + 1];
+                okt[u] = pack_f16x2(kt4[e], kt4[e + 1]);
+                oqt[u] = pack_f16x2(qt4[e], qt4[e + 1]);
                 oke[u] = pack_f16x2(e0, e1);
-                okh[u] = pack_f16x2(e0 * rg[e], e1 * rg[e + 1]);
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) suf[e] *= a[x][e];
-            *reinterpret_cast<uint2 *>(sm + OFF_KT + kh * QK_HALF + off) = make_uint2(okt[0], okt[1]);
-            *reinterpret_cast<uint2 *>(sm + OFF_QK + kh * QK_HALF + off) = make_uint2(oqt[0], oqt[1]);
-            *reinterpret_cast<uint2 *>(sm + OFF_KH + kh * 8192 + off) = make_uint2(okh[0], okh[1]);
+            *reinterpret_cast<float4 *>(sm + OFF_QK32 + qj * 16384 + off32) =
+                make_float4(to_tf32(qt4[0]), to_tf32(qt4[1]), to_tf32(qt4[2]), to_tf32(qt4[3]));
+            *reinterpret_cast<float4 *>(sm + OFF_QK32 + qj * 16384 + 8192 + off32) =
+                make_float4(to_tf32(kt4[0]), to_tf32(kt4[1]), to_tf32(kt4[2]), to_tf32(kt4[3]));
+            *reinterpret_cast<float4 *>(sm + OFF_KH32 + qj * 8192 + off32) =
+                make_float4(to_tf32(kh4[0]), to_tf32(kh4[1]), to_tf32(kh4[2]), to_tf32(kh4[3]));
             kend[x] = make_uint2(oke[0], oke[1]);
+            okt8[x] = make_uint2(okt[0], okt[1]);
+            oqt8[x] = make_uint2(oqt[0], oqt[1]);
         }
     }
     fence_proxy_async_smem();
@@ -359,14 +384,14 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // ---- P1: D1A = [Qt; Kt] Kh^T (M=128, N=64, K=128): rows 0-63 Qt Kh^T, rows 64-127 Kt Kh^T
+    // ---- P1: D1A = [Qt; Kt] Kh^T (M=128, N=64, K=128, tf32): rows 0-63 Qt Kh^T, rows 64-127 Kt Kh^T
     if (tid == 0) {
-        const uint32_t id = idesc_f16(128, 64, 0, 0);
+        const uint32_t id = idesc_tf32(128, 64, 0, 0);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t k2 = ks >> 2, ko = (ks & 3) * 32;
-            umma_ss(tmem + TM_D1A, smem_desc(sbase + OFF_QK + k2 * QK_HALF + ko, 16, 1024, SW_128B),
-                    smem_desc(sbase + OFF_KH + k2 * 8192 + ko, 16, 1024, SW_128B), id, ks > 0);
+        for (int ks = 0; ks < 16; ++ks) {
+            const uint32_t qj = ks >> 2, ko = (ks & 3) * 32;
+            umma_ss_tf32(tmem + TM_D1A, smem_desc(sbase + OFF_QK32 + qj * 16384 + ko, 16, 1024, SW_128B),
+                         smem_desc(sbase + OFF_KH32 + qj * 8192 + ko, 16, 1024, SW_128B), id, ks > 0);
         }
         umma_commit(bar);
     }
@@ -386,6 +411,14 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
     if (tid == 0 && !mbar_wait(bar, 0)) failed = 1;
     __syncthreads();
     tc_fence_after();
+    // ---- the tf32 operands are dead: f16 Kt and Qt tiles (B of P3; read by the last epilogue)
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+        const int r = 8 * warp + x;
+        const uint32_t off = r * 128 + ((((lc4 >> 1) ^ (r & 7)) & 7) << 4) + ((lc4 & 1) << 3);
+        *reinterpret_cast<uint2 *>(sm + OFF_KT + kh * QK_HALF + off) = okt8[x];
+        *reinterpret_cast<uint2 *>(sm + OFF_QK + kh * QK_HALF + off) = oqt8[x];
+    }
     // ---- P1 epilogue (M=128: lane = row): rows 0-63 -> M (f16, smem), rows 64-127 -> A^T (fp32,
     //      smem); warp w takes columns 32 (w / 4) .. +31 of its rows
     {
@@ -595,6 +628,7 @@ cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slo
     p.q = (const __nv_bfloat16 *)a.q; p.k = (const __nv_bfloat16 *)a.k;
     p.log_alpha = a.log_alpha; p.beta = a.beta; p.cu_seqlens = a.cu_seqlens;
     p.ws = ws; p.T = a.T; p.H = a.H; p.N = a.N; p.n_slots = n_slots; p.status = a.status;
+    p.tokens = (long long)a.B * a.T;
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)

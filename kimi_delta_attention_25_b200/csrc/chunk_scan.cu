@@ -78,6 +78,7 @@ struct ScanParams {
     void *out;
     float *S_final;
     int T, H, N, n_slots;
+    long long tokens;               // B * T (rows of v and out)
     int32_t *status;
 };
 
@@ -196,9 +197,11 @@ chunk_scan_kernel(ScanParams p)
             for (int rr = 0; rr < 2; ++rr) {
                 const int r = 2 * lane + rr;
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    vr[rr][u] = (r < L) ? ldg_nc(p.v + ((size_t)(tok0 + r) * H + h) * DK + j0 + 8 * u)
-                                        : make_uint4(0, 0, 0, 0);
+                for (int u = 0; u < 4; ++u) {
+                    const long long vi = ((long long)(tok0 + r) * H + h) * DK + j0 + 8 * u;
+                    vr[rr][u] = (r < L && in_bounds(p.status, vi, 8, p.tokens * H * DK)) ? ldg_nc(p.v + vi)
+                                                                                        : make_uint4(0, 0, 0, 0);
+                }
             }
         };
         if (nchunks > 0) load_v(0);
@@ -218,6 +221,11 @@ chunk_scan_kernel(ScanParams p)
             int ok = 1;
             if (c >= NSTAGE && lane == 0) ok = mbar_wait(&bars[B_EMPTY + s], ((c / NSTAGE) - 1) & 1);
             if (!__shfl_sync(0xffffffffu, ok, 0)) { if (lane == 0) fail(); break; }
+            if (!__shfl_sync(0xffffffffu, (int)in_bounds(p.status, (long long)h * p.n_slots + first_slot + c, 1,
+                                                         (long long)H * p.n_slots), 0)) {
+                if (lane == 0) *abort_flag = 1;        // KDA_ERR_BOUNDS recorded; every role stops
+                break;
+            }
             if (lane == 0) {
                 const unsigned char *blk = block_of(c);
                 mbar_arrive_expect_tx(&bars[B_FULL + s], (uint32_t)kPrepBlockBytes);
@@ -251,7 +259,8 @@ chunk_scan_kernel(ScanParams p)
             const size_t sidx = (((size_t)n * H + h) * DK + st) * DK + j0;
 #pragma unroll
             for (int j = 0; j < DVB; j += 4) {
-                const float4 v = p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + sidx + j) : make_float4(0, 0, 0, 0);
+                const float4 v = (p.S0 && in_bounds(p.status, (long long)(sidx + j), 4, (long long)p.N * H * DK * DK))
+                                     ? *reinterpret_cast<const float4 *>(p.S0 + sidx + j) : make_float4(0, 0, 0, 0);
                 S[j] = v.x; S[j + 1] = v.y; S[j + 2] = v.z; S[j + 3] = v.w;
             }
         }
@@ -309,7 +318,8 @@ chunk_scan_kernel(ScanParams p)
             mbar_arrive(&bars[B_SREADY]);
             mbar_arrive(&bars[B_EMPTY + s]);          // gamma of stage s has been read
             // outputs of this chunk (kept off the chain: global stores here overlap the next S1)
-            if (warp >= 2 && st - 64 < L) {
+            if (warp >= 2 && st - 64 < L &&
+                in_bounds(p.status, ((long long)(tok0 + st - 64) * H + h) * DK + j0, DVB, p.tokens * H * DK)) {
                 TO *dst = reinterpret_cast<TO *>(p.out) + ((size_t)(tok0 + st - 64) * H + h) * DK + j0;
                 if constexpr (sizeof(TO) == 4) {
 #pragma unroll
@@ -327,7 +337,8 @@ chunk_scan_kernel(ScanParams p)
                 }
             }
         }
-        if (p.S_final && !*abort_flag) {
+        if (p.S_final && !*abort_flag &&
+            in_bounds(p.status, (long long)((((size_t)n * H + h) * DK + st) * DK + j0), DVB, (long long)p.N * H * DK * DK)) {
             const size_t sidx = (((size_t)n * H + h) * DK + st) * DK + j0;
 #pragma unroll
             for (int j = 0; j < DVB; j += 4)
@@ -346,6 +357,7 @@ cudaError_t launch_typed(const PrefillArgs &a, const unsigned char *ws, int n_sl
     p.v = (const __nv_bfloat16 *)a.v; p.S0 = a.S0; p.cu_seqlens = a.cu_seqlens; p.ws = ws;
     p.out = a.out; p.S_final = a.S_final; p.T = a.T; p.H = a.H; p.N = a.N; p.n_slots = n_slots;
     p.status = a.status;
+    p.tokens = (long long)a.B * a.T;
     auto kern = chunk_scan_kernel<TO>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;

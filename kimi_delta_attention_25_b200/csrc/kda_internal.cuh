@@ -12,6 +12,9 @@ namespace kda {
 constexpr int kHeadDim = 128;   // d_k = d_v supported by every kernel
 constexpr int kChunk = 64;      // chunk length of the prefill (tokens)
 constexpr size_t kStatusBytes = 256;  // workspace prefix holding the device status word
+// Lowest cumulative log-decay within one chunk (per channel) that the chunked kernels take: they
+// factor e^{g_r - g_i} = e^{g_r} e^{-g_i}, and e^{-g} must stay finite in fp32.
+constexpr float kMinChunkLogDecay = -80.f;
 constexpr int kMaxGridDim = 65535;    // heads and sequences index grid dimensions y and z of the
                                       // chunked kernels
 
@@ -41,6 +44,25 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // Records the first device-side error in the workspace status word.
 __device__ __forceinline__ void set_status(int32_t *status, int32_t code) {
     if (status) atomicCAS(status, 0, code);
+}
+
+#ifndef KDA_DEBUG
+#define KDA_DEBUG 0
+#endif
+// Bounds check of a global access of `n` consecutive elements starting at element `idx` of a
+// buffer of `extent` elements. Debug builds (-DKDA_DEBUG=1, the library's stand-in for a memory
+// checker) record KDA_ERR_BOUNDS in the status word and return false, and the caller skips the
+// access (a skipped load reads zero); release builds compile the check away.
+__device__ __forceinline__ bool in_bounds(int32_t *status, long long idx, long long n, long long extent) {
+#if KDA_DEBUG
+    if (idx < 0 || n < 0 || idx + n > extent) {
+        set_status(status, KDA_ERR_BOUNDS);
+        return false;
+    }
+#else
+    (void)status; (void)idx; (void)n; (void)extent;
+#endif
+    return true;
 }
 
 // Resolves the token span [t0, t1) of sequence n (flat token index = b * T + t)
@@ -128,7 +150,6 @@ cudaError_t launch_chunk_fp32(const PrefillArgs &a, kda_dtype_t dtype, kda_dtype
                               cudaStream_t stream);
 
 // Tensor-core (tcgen05) chunk path for bf16 q/k/v in one kernel (no workspace beyond the status).
-bool chunk_tc_supported(const PrefillArgs &a);
 cudaError_t launch_chunk_tc(const PrefillArgs &a, kda_dtype_t out_dtype, cudaStream_t stream);
 
 // Two-pass tensor-core chunk path for bf16 q/k/v: prepared operands go through the workspace.

@@ -98,10 +98,24 @@ extern "C" kda_status_t kda_chunk_fwd_noalloc(const void *q, const void *k, cons
     a.status = (int32_t *)scratch;
     a.scratch = (unsigned char *)scratch + kStatusBytes;
     a.scratch_bytes = kNoAllocScratchBytes - kStatusBytes;
-    cudaError_t e;
-    if (dtype == KDA_BF16 && chunk_tc_supported(a))
-        e = launch_chunk_tc(a, out_dtype, s);
-    else
-        e = launch_chunk_fp32(a, dtype, out_dtype, s);
+    // bf16 inputs: the single-kernel tensor-core prefill (its decay-range check and the cu_seqlens
+    // check land in the status header); fp32 inputs: the CUDA-core prefill
+    const cudaError_t e = (dtype == KDA_BF16) ? launch_chunk_tc(a, out_dtype, s)
+                                              : launch_chunk_fp32(a, dtype, out_dtype, s);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+extern "C" kda_status_t kda_chunk_fwd_noalloc_status(void *stream, int32_t *status)
+{
+    if (!status) return KDA_ERR_INVALID_ARG;
+    void *scratch = nullptr;
+    kda_status_t st = scratch_address(&scratch);
+    if (st != KDA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    int32_t v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, scratch, sizeof(v), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    *status = v;
+    return KDA_OK;
 }

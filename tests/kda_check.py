@@ -27,8 +27,21 @@ def rel_err(x, r):
     return float(np.max(np.abs(x - r))) / (rms if rms > 0 else 1.0)
 
 
+# Every comparison made through the helpers below, as (test, what, max|err|/RMS(ref), tol); the
+# test session prints them and, when KDA_MARGINS_FILE is set, writes them there as JSON lines.
+MARGINS = []
+
+
+def _record(what, e, tol):
+    import os
+    test = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]
+    MARGINS.append({"test": test, "what": what, "err_over_rms": e, "tol": tol})
+    print("margin %-60s %-28s max|err|/RMS = %.3e (tol %.0e)" % (test[-60:], what, e, tol))
+
+
 def assert_close(x, r, tol, what):
     e = rel_err(x, r)
+    _record(what, e, tol)
     assert np.all(np.isfinite(np.asarray(x, dtype=np.float64))), "%s: non-finite values" % what
     assert e <= tol, "%s: max|err|/RMS(ref) = %.3e > %.1e" % (what, e, tol)
     return e
@@ -43,9 +56,11 @@ def assert_close_bf16_out(x, r, tol, what):
     rms = math.sqrt(float(np.mean(r * r))) if r.size else 0.0
     slack = np.abs(x - r) - (tol * rms * (1 + 2.0 ** -8) + 2.0 ** -8 * np.abs(r))
     worst = float(np.max(slack)) if r.size else -1.0
+    e = rel_err(x, r)
+    _record(what, e, tol)
     assert np.all(np.isfinite(x)), "%s: non-finite values" % what
     assert worst <= 0, "%s: exceeds tol*RMS + bf16 rounding by %.3e (RMS %.3e)" % (what, worst, rms)
-    return rel_err(x, r)
+    return e
 
 
 def oracle_prefill(d, heads=None, nthreads=0):

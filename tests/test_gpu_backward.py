@@ -46,9 +46,10 @@ def _oracle(d, heads=None):
 
 def _run(d, tol, heads=None, want_dS0=True):
     gd = to_device(d, DEV)
-    g = kda.chunk_bwd(gd["q"], gd["k"], gd["v"], gd["log_alpha"], gd["beta"], gd["dout"], S0=gd["S0"],
-                      dS_final=gd["dS_final"], cu_seqlens=gd["cu_seqlens"], want_dS0=want_dS0)
-    assert kda.workspace_status(kda.chunk_bwd.last_workspace) == kda.KDA_OK
+    g, ws = kda.chunk_bwd(gd["q"], gd["k"], gd["v"], gd["log_alpha"], gd["beta"], gd["dout"], S0=gd["S0"],
+                          dS_final=gd["dS_final"], cu_seqlens=gd["cu_seqlens"], want_dS0=want_dS0,
+                          return_workspace=True)
+    assert kda.workspace_status(ws) == kda.KDA_OK
     r = _oracle(d, heads=heads)
     errs = {}
     for name in GRADS:
@@ -113,8 +114,19 @@ def test_invalid_cu_seqlens_flagged_on_device():
     w = K.Workload("bwd_bad", B=1, T=128, H=2, dtype="bf16")
     d = to_device(_with_output_grads(K.make_prefill(w, seed=36), seed=7), DEV)
     cu = torch.tensor([0, 100, 50, 128], dtype=torch.int32, device=DEV)
-    kda.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["dout"], cu_seqlens=cu)
-    assert kda.workspace_status(kda.chunk_bwd.last_workspace) == kda.KDA_ERR_INVALID_ARG
+    _, ws = kda.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["dout"], cu_seqlens=cu,
+                          return_workspace=True)
+    assert kda.workspace_status(ws) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_decay_outside_range_is_reported():
+    """A chunk whose cumulative log-decay falls below -80 in some channel cannot be factored in
+    fp32 (e^{-g} overflows): the backward reports KDA_ERR_UNSUPPORTED in its status word instead
+    of returning non-finite gradients silently."""
+    w = K.Workload("bwd_too_strong", B=1, T=128, H=2, dtype="bf16", alpha_lo=0.2, alpha_hi=0.25)
+    d = to_device(_with_output_grads(K.make_prefill(w, seed=38), seed=11), DEV)
+    _, ws = kda.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["dout"], return_workspace=True)
+    assert kda.workspace_status(ws) == kda.KDA_ERR_UNSUPPORTED
 
 
 @pytest.mark.slow
@@ -133,8 +145,7 @@ def test_phases_one_by_one_equal_one_call_bitwise():
     g = None
     ws = None
     for phase in range(3):
-        g = kda.chunk_bwd(*args, **kw, grads=g, workspace=ws, phase=phase)
-        ws = kda.chunk_bwd.last_workspace
+        g, ws = kda.chunk_bwd(*args, **kw, grads=g, workspace=ws, phase=phase, return_workspace=True)
     assert kda.workspace_status(ws) == kda.KDA_OK
     for name in GRADS:
         assert torch.equal(g[name], ref[name]), name
@@ -150,9 +161,9 @@ def test_bf16_t128k_h32_sampled_head():
     B, T, H, D = d["v"].shape
     d["dout"] = torch.randn(B, T, H, D, generator=g, device=DEV).to(torch.bfloat16)
     d["dS_final"] = torch.randn(B, H, D, D, generator=g, device=DEV)
-    gr = kda.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["dout"], S0=d["S0"],
-                       dS_final=d["dS_final"])
-    assert kda.workspace_status(kda.chunk_bwd.last_workspace) == kda.KDA_OK
+    gr, ws = kda.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["dout"], S0=d["S0"],
+                           dS_final=d["dS_final"], return_workspace=True)
+    assert kda.workspace_status(ws) == kda.KDA_OK
     h = 7
     sub = {x: d[x][:, :, h:h + 1].contiguous() for x in ("q", "k", "v", "log_alpha", "beta", "dout")}
     sub["S0"] = d["S0"][:, h:h + 1].contiguous()
