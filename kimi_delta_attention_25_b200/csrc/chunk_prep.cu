@@ -40,11 +40,14 @@ constexpr int DK = kHeadDim;
 constexpr int NT = 256;
 
 // The intra-chunk product P1 pairs Kt = K e^{g} with Kh = K e^{-g}: for a channel that forgets fast
-// within the chunk, e^{-g} exceeds the f16 range long before the product loses meaning. P1 therefore
-// runs on tf32 operands (fp32 range, the 10-bit significand of f16); every later product takes f16
-// operands, which only shrink toward zero there. e^{-g} must stay finite in fp32: the decay
-// accumulated over one chunk must keep e^{g} above e^{-80} per channel; beyond that UNSUPPORTED.
+// within the chunk, e^{-g} leaves the f16 range (and Kt its normal range) long before the product
+// loses meaning. A chunk whose decay stays above kF16MinDecay in every channel runs P1 on f16
+// operands; any other chunk runs it on tf32 operands (fp32 range, the 10-bit significand of f16).
+// Every later product takes f16 operands, which only shrink toward zero there. e^{-g} must stay
+// finite in fp32: the decay over one chunk must keep e^{g} above e^{-80} per channel; beyond that
+// the chunk is reported UNSUPPORTED.
 constexpr float kMinChunkDecay = 1.80485139e-35f;   // e^{-80}
+constexpr float kF16MinDecay = 3.35462628e-04f;     // e^{-8}: Kh <= 2981 |k|, Kt >= 3.4e-4 |k|
 
 // shared memory (1024-aligned base)
 constexpr uint32_t OFF_QK = 0;               // [Qt; Kt] (f16): per 64-channel half (16 KB apart),
@@ -321,6 +324,7 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
     *reinterpret_cast<float4 *>(Ps + warp * 128 + 4 * cq) = make_float4(pre[7][0], pre[7][1], pre[7][2], pre[7][3]);
     __syncthreads();
     float before[4] = {1.f, 1.f, 1.f, 1.f}, after[4] = {1.f, 1.f, 1.f, 1.f}, g[4], rg[4];
+    float gall[4] = {1.f, 1.f, 1.f, 1.f};      // the same product in one fixed order in every warp
 #pragma unroll
     for (int y = 0; y < 8; ++y) {
         const float4 t = *reinterpret_cast<const float4 *>(Ps + y * 128 + 4 * cq);
@@ -329,8 +333,13 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
         for (int e = 0; e < 4; ++e) {
             if (y < warp) before[e] *= tv[e];
             if (y > warp) after[e] *= tv[e];
+            gall[e] *= tv[e];
         }
     }
+    // tf32 operands for P1 when any channel decays below e^-8 over the chunk (bitwise the same
+    // decision in every warp: each lane holds 4 channels, the lanes of a warp all 128)
+    const bool wide = __any_sync(0xffffffffu, gall[0] < kF16MinDecay || gall[1] < kF16MinDecay ||
+                                               gall[2] < kF16MinDecay || gall[3] < kF16MinDecay) != 0;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
         g[e] = before[e] * pre[7][e] * after[e];
@@ -367,12 +376,20 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) suf[e] *= a[x][e];
-            *reinterpret_cast<float4 *>(sm + OFF_QK32 + qj * 16384 + off32) =
-                make_float4(to_tf32(qt4[0]), to_tf32(qt4[1]), to_tf32(qt4[2]), to_tf32(qt4[3]));
-            *reinterpret_cast<float4 *>(sm + OFF_QK32 + qj * 16384 + 8192 + off32) =
-                make_float4(to_tf32(kt4[0]), to_tf32(kt4[1]), to_tf32(kt4[2]), to_tf32(kt4[3]));
-            *reinterpret_cast<float4 *>(sm + OFF_KH32 + qj * 8192 + off32) =
-                make_float4(to_tf32(kh4[0]), to_tf32(kh4[1]), to_tf32(kh4[2]), to_tf32(kh4[3]));
+            if (wide) {
+                *reinterpret_cast<float4 *>(sm + OFF_QK32 + qj * 16384 + off32) =
+                    make_float4(to_tf32(qt4[0]), to_tf32(qt4[1]), to_tf32(qt4[2]), to_tf32(qt4[3]));
+                *reinterpret_cast<float4 *>(sm + OFF_QK32 + qj * 16384 + 8192 + off32) =
+                    make_float4(to_tf32(kt4[0]), to_tf32(kt4[1]), to_tf32(kt4[2]), to_tf32(kt4[3]));
+                *reinterpret_cast<float4 *>(sm + OFF_KH32 + qj * 8192 + off32) =
+                    make_float4(to_tf32(kh4[0]), to_tf32(kh4[1]), to_tf32(kh4[2]), to_tf32(kh4[3]));
+            } else {
+                const uint32_t off = r * 128 + ((((lc4 >> 1) ^ (r & 7)) & 7) << 4) + ((lc4 & 1) << 3);
+                *reinterpret_cast<uint2 *>(sm + OFF_KT + kh * QK_HALF + off) = make_uint2(okt[0], okt[1]);
+                *reinterpret_cast<uint2 *>(sm + OFF_QK + kh * QK_HALF + off) = make_uint2(oqt[0], oqt[1]);
+                *reinterpret_cast<uint2 *>(sm + OFF_KH + kh * 8192 + off) =
+                    make_uint2(pack_f16x2(kh4[0], kh4[1]), pack_f16x2(kh4[2], kh4[3]));
+            }
             kend[x] = make_uint2(oke[0], oke[1]);
             okt8[x] = make_uint2(okt[0], okt[1]);
             oqt8[x] = make_uint2(oqt[0], oqt[1]);
@@ -384,14 +401,25 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // ---- P1: D1A = [Qt; Kt] Kh^T (M=128, N=64, K=128, tf32): rows 0-63 Qt Kh^T, rows 64-127 Kt Kh^T
+    // ---- P1: D1A = [Qt; Kt] Kh^T (M=128, N=64, K=128; f16, or tf32 for a wide decay range):
+    //      rows 0-63 Qt Kh^T, rows 64-127 Kt Kh^T
     if (tid == 0) {
-        const uint32_t id = idesc_tf32(128, 64, 0, 0);
+        if (wide) {
+            const uint32_t id = idesc_tf32(128, 64, 0, 0);
 #pragma unroll
-        for (int ks = 0; ks < 16; ++ks) {
-            const uint32_t qj = ks >> 2, ko = (ks & 3) * 32;
-            umma_ss_tf32(tmem + TM_D1A, smem_desc(sbase + OFF_QK32 + qj * 16384 + ko, 16, 1024, SW_128B),
-                         smem_desc(sbase + OFF_KH32 + qj * 8192 + ko, 16, 1024, SW_128B), id, ks > 0);
+            for (int ks = 0; ks < 16; ++ks) {
+                const uint32_t qj = ks >> 2, ko = (ks & 3) * 32;
+                umma_ss_tf32(tmem + TM_D1A, smem_desc(sbase + OFF_QK32 + qj * 16384 + ko, 16, 1024, SW_128B),
+                             smem_desc(sbase + OFF_KH32 + qj * 8192 + ko, 16, 1024, SW_128B), id, ks > 0);
+            }
+        } else {
+            const uint32_t id = idesc_f16(128, 64, 0, 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t k2 = ks >> 2, ko = (ks & 3) * 32;
+                umma_ss(tmem + TM_D1A, smem_desc(sbase + OFF_QK + k2 * QK_HALF + ko, 16, 1024, SW_128B),
+                        smem_desc(sbase + OFF_KH + k2 * 8192 + ko, 16, 1024, SW_128B), id, ks > 0);
+            }
         }
         umma_commit(bar);
     }
@@ -411,13 +439,16 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
     if (tid == 0 && !mbar_wait(bar, 0)) failed = 1;
     __syncthreads();
     tc_fence_after();
-    // ---- the tf32 operands are dead: f16 Kt and Qt tiles (B of P3; read by the last epilogue)
+    // ---- tf32 path: its operands are dead; the f16 Kt and Qt tiles (B of P3; read by the last
+    //      epilogue) take their place
+    if (wide) {
 #pragma unroll
-    for (int x = 0; x < 8; ++x) {
-        const int r = 8 * warp + x;
-        const uint32_t off = r * 128 + ((((lc4 >> 1) ^ (r & 7)) & 7) << 4) + ((lc4 & 1) << 3);
-        *reinterpret_cast<uint2 *>(sm + OFF_KT + kh * QK_HALF + off) = okt8[x];
-        *reinterpret_cast<uint2 *>(sm + OFF_QK + kh * QK_HALF + off) = oqt8[x];
+        for (int x = 0; x < 8; ++x) {
+            const int r = 8 * warp + x;
+            const uint32_t off = r * 128 + ((((lc4 >> 1) ^ (r & 7)) & 7) << 4) + ((lc4 & 1) << 3);
+            *reinterpret_cast<uint2 *>(sm + OFF_KT + kh * QK_HALF + off) = okt8[x];
+            *reinterpret_cast<uint2 *>(sm + OFF_QK + kh * QK_HALF + off) = oqt8[x];
+        }
     }
     // ---- P1 epilogue (M=128: lane = row): rows 0-63 -> M (f16, smem), rows 64-127 -> A^T (fp32,
     //      smem); warp w takes columns 32 (w / 4) .. +31 of its rows

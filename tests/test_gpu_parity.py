@@ -264,7 +264,7 @@ def test_decode_n256_h32_1000_steps_sampled():
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("lo,hi", [(0.3, 0.7), (0.8, 0.9)])
+@pytest.mark.parametrize("lo,hi", [(0.3, 0.7), (0.8, 0.9), (0.85, 0.95)])
 def test_fast_forgetting_channels(dtype, lo, hi):
     """Channel gates that forget fast within a chunk (alpha ~ U(0.3, 0.7): the cumulative
     log-decay of one 64-token chunk reaches about -47; U(0.8, 0.9): about -11): the gate is
