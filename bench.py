@@ -364,9 +364,12 @@ def run_native(args):
     e2e_val = ws * tokens / (ms_e2e * 1e-3) / 1e6
     del host, dbuf, h_out, h_sf
 
-    # ---- the other prefill workloads: 8K tokens x 16 heads, and 8 packed sequences (262K tokens)
+    # ---- the same workload as a full layer step (gate producers and output norm fused)
     del work
     torch.cuda.empty_cache()
+    layer_step = run_layer_step(kda, dev, pk, ws, rank, args, d)
+
+    # ---- the other prefill workloads: 8K tokens x 16 heads, and 8 packed sequences (262K tokens)
     other = {name: run_prefill_config(kda, dev, pk, ws, rank, args, name, 6.0)
              for name in ("bf16_t8k_h16", "bf16_varlen8_262k_h32")}
 
@@ -404,6 +407,7 @@ def run_native(args):
                     "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
             "gpu_launches": args.steps * PREFILL_KERNELS_PER_STEP,
             "clocks": clk.summary(),
+            "layer_step": layer_step,
             "configs": other,
             "decode": dec,
             "backward": bwd,
@@ -479,6 +483,64 @@ def run_prefill_config(kda, dev, pk, ws, rank, args, name, cpu_budget_s):
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_oracle_sample(budget_s=cpu_budget_s, workload=name)
     return res
+
+
+# the layer step: q, k, v, out bf16 (4 x 256 B), the decay-gate input f bf16 (256 B) in place of
+# fp32 log_alpha, the write-gate logits bf16 (2 B) in place of fp32 beta, the output gate g bf16 (256 B)
+LAYER_BYTES_PER_TOKEN_HEAD = 4 * D * 2 + D * 2 + 2 + D * 2
+
+
+def run_layer_step(kda, dev, pk, ws, rank, args, d):
+    """The same 128K x 32 prefill as a full KDA layer step: gates produced inside the preparation
+    pass from f, A_log, dt_bias and the beta logits, and the gated RMSNorm applied in the scan's
+    output epilogue (4-CTA clusters); bf16 outputs. Timed per pass like the headline step."""
+    B, T, H = d["v"].shape[:3]
+    lay = K.make_layer_inputs(B, T, H, dtype="bf16", device=dev, seed=5)
+    opts = dict(lay, norm_eps=1e-5)
+    out = torch.empty(B, T, H, D, dtype=torch.bfloat16, device=dev)
+    Sf = torch.empty(B, H, D, D, dtype=torch.float32, device=dev)
+    work = torch.empty(max(256, kda.chunk_fwd_workspace_size(B, T, H, B)), dtype=torch.uint8, device=dev)
+    steps = max(3, args.steps)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+
+    def passes(ev=None):
+        if ev is not None:
+            ev[0].record()
+        kda.chunk_prep(d["q"], d["k"], None, None, work, layer=opts)
+        if ev is not None:
+            ev[1].record()
+        kda.chunk_scan(d["v"], work, S0=d["S0"], out=out, S_final=Sf, layer=opts)
+        if ev is not None:
+            ev[2].record()
+
+    with Clocks(int(os.environ.get("LOCAL_RANK", "0"))) as clk:
+        for _ in range(args.warmup):
+            passes()
+        torch.cuda.synchronize()
+        barrier(ws)
+        torch.cuda.synchronize()
+        t_s, t_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t_s.record()
+        for i in range(steps):
+            passes(evs[i])
+        t_e.record()
+        torch.cuda.synchronize()
+        barrier(ws)
+    assert kda.workspace_status(work) == kda.KDA_OK
+    ms = max_over_ranks(t_s.elapsed_time(t_e) / steps, ws)
+    th = B * T * H
+    gbs = th * LAYER_BYTES_PER_TOKEN_HEAD / (ms * 1e-3) / 1e9
+    kern = {"chunk_prep_gates": {"ms": statistics.mean(e[0].elapsed_time(e[1]) for e in evs)},
+            "chunk_scan_norm": {"ms": statistics.mean(e[1].elapsed_time(e[2]) for e in evs)}}
+    del out, Sf, work, lay, opts
+    torch.cuda.empty_cache()
+    return {"workload": WORKLOAD, "ms_per_step": ms, "Mtok_s": ws * B * T / (ms * 1e-3) / 1e6, "steps": steps,
+            "fused": "decay gate from f, A_log, dt_bias and beta from logits in the preparation pass; "
+                     "gated RMSNorm (sigmoid gate) in the scan's output epilogue",
+            "algorithmic_bytes_per_token_head": LAYER_BYTES_PER_TOKEN_HEAD,
+            "roofline_step": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                              "frac": gbs / pk["hbm"], "peak_source": "of %s" % pk["src"]},
+            "kernels": kern, "gpu_launches": 2 * steps, "clocks": clk.summary()}
 
 
 def run_decode(kda, dev, pk, ws, local, args):

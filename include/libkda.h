@@ -212,6 +212,79 @@ kda_status_t kda_decode_step(const void *q, const void *k, const void *v,
                              int N, int H, int dk, int dv, kda_dtype_t dtype,
                              kda_dtype_t out_dtype, void *stream);
 
+/* ---------------------------------------------------------------------------------------------
+ * The KDA layer's element-wise neighbours of the recurrence, fused into its kernels.
+ *
+ * The pages name these parts of the Kimi Linear KDA module without printing a formula
+ * (lpnh.cn Kimi Linear KDA/NoPE article, sec. 3: A_log, dt_bias and the low-rank f_a/f_b
+ * projection feed the channel-wise decay through fused_kda_gate; b_proj feeds the write gate
+ * beta; the output goes through o_norm = FusedRMSNormGated with the activation fixed to
+ * sigmoid; sec. 4 names the decay and beta gating). The readings used here:
+ *   log_alpha[t,h,c] = -exp(A_log[h]) * softplus(gate_f[t,h,c] + dt_bias[h*dk + c])
+ *   beta[t,h]        = sigmoid(beta_logits[t,h])
+ *   y[t,h,:]         = o[t,h,:] / sqrt(mean_c o[t,h,c]^2 + norm_eps) * norm_weight[:]
+ *                      * sigmoid(out_gate[t,h,:])
+ * Each group is optional: a NULL gate_f means log_alpha is passed directly, a NULL beta_logits
+ * means beta is passed directly, a NULL out_gate means the raw outputs o are written.
+ *   gate_f      [B,T,H,dk] (decode: [N,H,dk]) in dtype; A_log [H] and dt_bias [H*dk] float32
+ *   beta_logits [B,T,H]    (decode: [N,H])    in dtype
+ *   out_gate    [B,T,H,dv] (decode: [N,H,dv]) in dtype; norm_weight [dv] float32 (shared by
+ *               the heads); norm_eps >= 0
+ * Alignment: gate_f, out_gate, dt_bias 16 bytes; A_log, norm_weight, beta_logits 4 bytes.
+ * --------------------------------------------------------------------------------------------- */
+typedef struct {
+    const void *gate_f;
+    const float *A_log;
+    const float *dt_bias;
+    const void *beta_logits;
+    const void *out_gate;
+    const float *norm_weight;
+    float norm_eps;
+} kda_layer_opts_t;
+
+/* Workspace bytes of kda_chunk_fwd_layer: that of kda_chunk_fwd, plus (fp32 inputs only) fp32
+ * scratch for the produced gates and for the outputs before the norm. 0 for rejected sizes. */
+size_t kda_chunk_fwd_layer_workspace_size(int B, int T, int H, int N, int dk, int dv,
+                                          kda_dtype_t dtype, const kda_layer_opts_t *opts);
+
+/* kda_chunk_fwd with the layer options above (opts NULL or all-NULL: exactly kda_chunk_fwd).
+ * log_alpha / beta may be NULL when their producer inputs are given. For bf16 inputs every part
+ * is fused: the decay and write gates are produced inside the preparation pass (the fp32
+ * log_alpha stream is never written or read), and the output norm runs in the scan's output
+ * epilogue, with the four 32-channel CTAs of a head exchanging per-token sums of squares through
+ * distributed shared memory (a 4-CTA cluster). fp32 inputs run separate gate and norm passes
+ * around the CUDA-core prefill. Errors as for kda_chunk_fwd; a NULL A_log/dt_bias with gate_f, or
+ * a NULL norm_weight with out_gate, or norm_eps < 0 is KDA_ERR_INVALID_ARG. */
+kda_status_t kda_chunk_fwd_layer(const void *q, const void *k, const void *v,
+                                 const float *log_alpha, const float *beta,
+                                 const float *S0, const int32_t *cu_seqlens,
+                                 void *out, float *S_final,
+                                 int B, int T, int H, int N, int dk, int dv,
+                                 kda_dtype_t dtype, kda_dtype_t out_dtype,
+                                 const kda_layer_opts_t *opts,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/* The two passes of kda_chunk_fwd_layer for bf16 inputs, one by one (see kda_chunk_prep and
+ * kda_chunk_scan): the preparation pass with the gate producers, the scan with the output norm. */
+kda_status_t kda_chunk_prep_layer(const void *q, const void *k,
+                                  const float *log_alpha, const float *beta,
+                                  const int32_t *cu_seqlens,
+                                  int B, int T, int H, int N, int dk, int dv,
+                                  const kda_layer_opts_t *opts,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+kda_status_t kda_chunk_scan_layer(const void *v, const float *S0, const int32_t *cu_seqlens,
+                                  void *out, float *S_final,
+                                  int B, int T, int H, int N, int dk, int dv, kda_dtype_t out_dtype,
+                                  const kda_layer_opts_t *opts,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/* kda_decode_step with the layer options (all fused into the decode kernel). */
+kda_status_t kda_decode_step_layer(const void *q, const void *k, const void *v,
+                                   const float *log_alpha, const float *beta,
+                                   float *S_inout, void *out,
+                                   int N, int H, int dk, int dv, kda_dtype_t dtype,
+                                   kda_dtype_t out_dtype, const kda_layer_opts_t *opts, void *stream);
+
 /* Capacity of the library-owned scratch array used by kda_chunk_fwd_noalloc (bytes). */
 #define KDA_NOALLOC_SCRATCH_BYTES 4096
 

@@ -31,7 +31,7 @@ from typing import List, Optional
 import torch
 
 __all__ = ["Workload", "WORKLOADS", "make_prefill", "make_decode_state",
-           "make_decode_step", "varlen_lengths", "to_dtype"]
+           "make_decode_step", "varlen_lengths", "to_dtype", "make_layer_inputs"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -173,3 +173,23 @@ def make_decode_step(w: Workload, step: int, device="cpu", N: Optional[int] = No
     log_alpha = torch.log(w.alpha_lo + (w.alpha_hi - w.alpha_lo) * u)
     beta = torch.sigmoid(torch.randn(N, H, generator=g, device=device))
     return dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta)
+
+
+def make_layer_inputs(B: int, T: int, H: int, dtype: str = "bf16", device="cpu", seed: int = 0,
+                      dk: int = 128, dv: int = 128):
+    """Inputs of the layer's gate producers and output norm (synthetic, seeded; draw order f,
+    A_log, dt_bias, b, g, w): the decay-gate projection output f ~ N(0, 0.5^2) [B,T,H,dk], the
+    per-head A_log ~ U(0, 2) [H], the per-channel dt_bias ~ U(-6, -3) [H*dk], the write-gate logits
+    b ~ N(0, 1) [B,T,H], the output gate g ~ N(0, 1) [B,T,H,dv] and the norm weight
+    w ~ U(0.5, 1.5) [dv]. f, b and g take the input dtype (rounded from fp32); A_log, dt_bias and w
+    stay fp32. (With these ranges the decay per token lies between about e^-0.4 and e^-0.0003.)"""
+    dt = to_dtype(dtype)
+    g = _gen(device, seed)
+    f = (0.5 * torch.randn(B, T, H, dk, generator=g, device=device)).to(dt)
+    A_log = 2.0 * torch.rand(H, generator=g, device=device)
+    dt_bias = -6.0 + 3.0 * torch.rand(H * dk, generator=g, device=device)
+    b = torch.randn(B, T, H, generator=g, device=device).to(dt)
+    og = torch.randn(B, T, H, dv, generator=g, device=device).to(dt)
+    w = 0.5 + torch.rand(dv, generator=g, device=device)
+    return dict(gate_f=f, A_log=A_log, dt_bias=dt_bias, beta_logits=b, out_gate=og, norm_weight=w)
+

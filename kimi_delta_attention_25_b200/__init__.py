@@ -37,10 +37,36 @@ _lib = None
 
 # Every entry point declared in include/libkda.h.
 EXPORTS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
+           "kda_chunk_fwd_layer_workspace_size", "kda_chunk_fwd_layer", "kda_chunk_prep_layer",
+           "kda_chunk_scan_layer", "kda_decode_step_layer",
            "kda_workspace_status", "kda_status_string", "kda_version", "kda_chunk_fwd_noalloc",
            "kda_chunk_prep", "kda_chunk_scan", "kda_selftest_wait_timeout",
            "kda_chunk_bwd_workspace_size", "kda_chunk_bwd", "kda_chunk_bwd_phase",
            "kda_chunk_fwd_noalloc_status")
+
+
+class LayerOpts(ctypes.Structure):
+    """``kda_layer_opts_t``: the layer's gate producers and output norm (device pointers)."""
+    _fields_ = [("gate_f", ctypes.c_void_p), ("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
+                ("beta_logits", ctypes.c_void_p), ("out_gate", ctypes.c_void_p),
+                ("norm_weight", ctypes.c_void_p), ("norm_eps", ctypes.c_float)]
+
+
+_LAYER_KEYS = ("gate_f", "A_log", "dt_bias", "beta_logits", "out_gate", "norm_weight")
+
+
+def _layer_opts(layer):
+    """A ``LayerOpts`` from a dict of tensors (keys of ``_LAYER_KEYS`` plus ``norm_eps``), or None."""
+    if not layer or not any(layer.get(k) is not None for k in ("gate_f", "beta_logits", "out_gate")):
+        return None
+    o = LayerOpts()
+    for key in _LAYER_KEYS:
+        t = layer.get(key)
+        if t is not None:
+            _need_cuda(t)
+            setattr(o, key, t.data_ptr())
+    o.norm_eps = float(layer.get("norm_eps", 1e-5))
+    return o
 
 
 class KDAError(RuntimeError):
@@ -86,6 +112,17 @@ def load():
     lib.kda_chunk_bwd.restype = I
     lib.kda_chunk_bwd_phase.argtypes = [I] + [P] * 15 + [I] * 7 + [P, Z, P]
     lib.kda_chunk_bwd_phase.restype = I
+    LP = ctypes.POINTER(LayerOpts)
+    lib.kda_chunk_fwd_layer_workspace_size.argtypes = [I, I, I, I, I, I, I, LP]
+    lib.kda_chunk_fwd_layer_workspace_size.restype = Z
+    lib.kda_chunk_fwd_layer.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, LP, P, Z, P]
+    lib.kda_chunk_fwd_layer.restype = I
+    lib.kda_chunk_prep_layer.argtypes = [P, P, P, P, P, I, I, I, I, I, I, LP, P, Z, P]
+    lib.kda_chunk_prep_layer.restype = I
+    lib.kda_chunk_scan_layer.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, LP, P, Z, P]
+    lib.kda_chunk_scan_layer.restype = I
+    lib.kda_decode_step_layer.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, LP, P]
+    lib.kda_decode_step_layer.restype = I
     _lib = lib
     return lib
 
@@ -124,14 +161,17 @@ def chunk_fwd_workspace_size(B, T, H, N, dk=128, dv=128, dtype=torch.bfloat16) -
 
 
 def chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, S_final=None,
-              workspace=None, want_state=True, out_dtype=torch.float32, return_workspace=False):
+              workspace=None, want_state=True, out_dtype=torch.float32, return_workspace=False, layer=None):
     """Chunkwise KDA prefill. Shapes: q, k, log_alpha [B,T,H,dk]; v [B,T,H,dv];
     beta [B,T,H]; S0 [N,H,dk,dv] fp32 or None; cu_seqlens int32 [N+1] or None.
     Returns (out [B,T,H,dv] in out_dtype (or the dtype of a given ``out``),
     S_final [N,H,dk,dv] fp32 or None), and the workspace as a third element when
     ``return_workspace`` (its status word holds the device-side checks: ``workspace_status``).
     Without a ``workspace`` argument each call takes a fresh one from torch's caching allocator
-    (about 1 KiB per token and head for bf16 inputs); a caller that runs many calls passes its own."""
+    (about 1 KiB per token and head for bf16 inputs); a caller that runs many calls passes its own.
+    ``layer`` (a dict with any of gate_f, A_log, dt_bias, beta_logits, out_gate, norm_weight,
+    norm_eps) selects ``kda_chunk_fwd_layer``: the gate producers (log_alpha and/or beta may then be
+    None) and the gated output norm, fused into the kernels."""
     lib = load()
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -144,18 +184,26 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, S_fi
     if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
         raise TypeError("cu_seqlens must be int32")
     code = _dtype_code(q)
-    ws_bytes = lib.kda_chunk_fwd_workspace_size(B, T, H, N, dk, dv, code)
+    opts = _layer_opts(layer)
+    if opts is None:
+        ws_bytes = lib.kda_chunk_fwd_workspace_size(B, T, H, N, dk, dv, code)
+    else:
+        ws_bytes = lib.kda_chunk_fwd_layer_workspace_size(B, T, H, N, dk, dv, code, ctypes.byref(opts))
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=q.device)
-    st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
-                           _ptr(cu_seqlens), _ptr(out), _ptr(S_final), B, T, H, N, dk, dv, code,
-                           _dtype_code(out), _ptr(workspace), workspace.numel(), _stream(q.device))
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(cu_seqlens), _ptr(out),
+            _ptr(S_final), B, T, H, N, dk, dv, code, _dtype_code(out))
+    if opts is None:
+        st = lib.kda_chunk_fwd(*args, _ptr(workspace), workspace.numel(), _stream(q.device))
+    else:
+        st = lib.kda_chunk_fwd_layer(*args, ctypes.byref(opts), _ptr(workspace), workspace.numel(),
+                                     _stream(q.device))
     if st != KDA_OK:
-        raise KDAError(st, "kda_chunk_fwd")
+        raise KDAError(st, "kda_chunk_fwd" if opts is None else "kda_chunk_fwd_layer")
     return (out, S_final, workspace) if return_workspace else (out, S_final)
 
 
-def chunk_prep(q, k, log_alpha, beta, workspace, cu_seqlens=None):
+def chunk_prep(q, k, log_alpha, beta, workspace, cu_seqlens=None, layer=None):
     """``kda_chunk_prep``: first pass of the bf16 prefill (everything that does not depend on the
     state), written into ``workspace`` (uint8, ``chunk_fwd_workspace_size(...)`` bytes)."""
     lib = load()
@@ -164,15 +212,20 @@ def chunk_prep(q, k, log_alpha, beta, workspace, cu_seqlens=None):
     _need_cuda(q, k, log_alpha, beta, cu_seqlens, workspace)
     if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16:
         raise TypeError("chunk_prep takes bfloat16 q and k")
-    st = lib.kda_chunk_prep(_ptr(q), _ptr(k), _ptr(log_alpha), _ptr(beta), _ptr(cu_seqlens),
-                            B, T, H, N, dk, dk, _ptr(workspace), workspace.numel(), _stream(q.device))
+    opts = _layer_opts(layer)
+    args = (_ptr(q), _ptr(k), _ptr(log_alpha), _ptr(beta), _ptr(cu_seqlens), B, T, H, N, dk, dk)
+    if opts is None:
+        st = lib.kda_chunk_prep(*args, _ptr(workspace), workspace.numel(), _stream(q.device))
+    else:
+        st = lib.kda_chunk_prep_layer(*args, ctypes.byref(opts), _ptr(workspace), workspace.numel(),
+                                      _stream(q.device))
     if st != KDA_OK:
         raise KDAError(st, "kda_chunk_prep")
     return workspace
 
 
 def chunk_scan(v, workspace, S0=None, cu_seqlens=None, out=None, S_final=None, want_state=True,
-               out_dtype=torch.float32):
+               out_dtype=torch.float32, layer=None):
     """``kda_chunk_scan``: second pass of the bf16 prefill, after ``chunk_prep`` on the same
     workspace and sizes. Returns (out, S_final) like ``chunk_fwd``."""
     lib = load()
@@ -185,9 +238,13 @@ def chunk_scan(v, workspace, S0=None, cu_seqlens=None, out=None, S_final=None, w
     _need_cuda(v, S0, cu_seqlens, out, S_final, workspace)
     if v.dtype != torch.bfloat16:
         raise TypeError("chunk_scan takes bfloat16 v")
-    st = lib.kda_chunk_scan(_ptr(v), _ptr(S0), _ptr(cu_seqlens), _ptr(out), _ptr(S_final),
-                            B, T, H, N, dv, dv, _dtype_code(out), _ptr(workspace), workspace.numel(),
-                            _stream(v.device))
+    opts = _layer_opts(layer)
+    args = (_ptr(v), _ptr(S0), _ptr(cu_seqlens), _ptr(out), _ptr(S_final), B, T, H, N, dv, dv, _dtype_code(out))
+    if opts is None:
+        st = lib.kda_chunk_scan(*args, _ptr(workspace), workspace.numel(), _stream(v.device))
+    else:
+        st = lib.kda_chunk_scan_layer(*args, ctypes.byref(opts), _ptr(workspace), workspace.numel(),
+                                      _stream(v.device))
     if st != KDA_OK:
         raise KDAError(st, "kda_chunk_scan")
     return out, S_final
@@ -265,18 +322,23 @@ def workspace_status(workspace: torch.Tensor) -> int:
     return int(v.value)
 
 
-def decode_step(q, k, v, log_alpha, beta, S, out=None, out_dtype=torch.float32):
+def decode_step(q, k, v, log_alpha, beta, S, out=None, out_dtype=torch.float32, layer=None):
     """One decode step: q, k, log_alpha [N,H,dk]; v [N,H,dv]; beta [N,H]; S [N,H,dk,dv] fp32
-    (updated in place). Returns out [N,H,dv] in out_dtype (or the dtype of a given ``out``)."""
+    (updated in place). Returns out [N,H,dv] in out_dtype (or the dtype of a given ``out``).
+    ``layer`` as for ``chunk_fwd`` (tensors shaped [N,H,...]) selects ``kda_decode_step_layer``."""
     lib = load()
     N, H, dk = q.shape
     dv = v.shape[-1]
     if out is None:
         out = torch.empty(N, H, dv, dtype=out_dtype, device=q.device)
     _need_cuda(q, k, v, log_alpha, beta, S, out)
-    st = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S),
-                             _ptr(out), N, H, dk, dv, _dtype_code(q), _dtype_code(out),
-                             _stream(q.device))
+    opts = _layer_opts(layer)
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), _ptr(out), N, H, dk, dv,
+            _dtype_code(q), _dtype_code(out))
+    if opts is None:
+        st = lib.kda_decode_step(*args, _stream(q.device))
+    else:
+        st = lib.kda_decode_step_layer(*args, ctypes.byref(opts), _stream(q.device))
     if st != KDA_OK:
         raise KDAError(st, "kda_decode_step")
     return out

@@ -45,7 +45,7 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int N, int dk, int dv, 
 
 }  // extern "C"
 
-namespace {
+namespace kda {
 
 // Host-side checks shared by the prefill entry points. `need_*` selects which tensors the caller
 // passes (the two passes of the bf16 path each take a subset).
@@ -97,7 +97,7 @@ PrefillArgs prefill_args(const void *q, const void *k, const void *v, const floa
     return a;
 }
 
-}  // namespace
+}  // namespace kda
 
 extern "C" {
 

@@ -99,6 +99,11 @@ __device__ __forceinline__ float4 ldg_nc_f4(const float *p) {
 struct PrepParams {
     const __nv_bfloat16 *q, *k;
     const float *log_alpha, *beta;
+    // gate producers (the layer's fused_kda_gate and b_proj gate): with GATE the third tensor copy
+    // brings the bf16 gate input f instead of log_alpha, and log_alpha = -exp(A_log[h]) *
+    // softplus(f + dt_bias[h, c]) is formed here; beta_logits (bf16) gives beta = sigmoid(b)
+    const float *A_log, *dt_bias;
+    const __nv_bfloat16 *beta_logits;
     const int32_t *cu_seqlens;
     unsigned char *ws;              // chunk blocks, [H][n_slots][kPrepBlockBytes]
     int T, H, N, n_slots;
@@ -227,6 +232,11 @@ __device__ __forceinline__ void inverse64(int pt, const float *AT, float *Tf, fl
     __syncthreads();
 }
 
+// softplus on the bf16 path: two fast special-function ops; its absolute error (~1e-7, which is
+// also all that is left of softplus(x) below x = -16) is far inside what bf16 inputs carry
+__device__ __forceinline__ float softplus_f(float x) { return x > 16.f ? x : __logf(1.f + __expf(x)); }
+
+template <bool GATE>
 __global__ void __launch_bounds__(NT, 2)
 chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_la)
@@ -264,7 +274,7 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
         mbar_init(bar, 1);
         mbar_init(bar_in, 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(bar_in, (uint32_t)C * (2 * DK * 2 + DK * 4));
+        mbar_arrive_expect_tx(bar_in, (uint32_t)C * (2 * DK * 2 + DK * (GATE ? 2 : 4)));
         tma_load_3d(sm + STG_Q, &tm_q, bar_in, 0, h, (int)tok0);
         tma_load_3d(sm + STG_K, &tm_k, bar_in, 0, h, (int)tok0);
         tma_load_3d(sm + STG_LA, &tm_la, bar_in, 0, h, (int)tok0);
@@ -290,11 +300,23 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
     const int cq = lane, kh = cq >> 4, lc4 = cq & 15;
     float4 la[8];
     uint2 kr[8], qr[8];
+    float rate = 0.f, bias[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (GATE) {
+        rate = expf(p.A_log[h]);
+        const float4 b4 = *reinterpret_cast<const float4 *>(p.dt_bias + (size_t)h * DK + 4 * cq);
+        bias[0] = b4.x; bias[1] = b4.y; bias[2] = b4.z; bias[3] = b4.w;
+    }
 #pragma unroll
     for (int x = 0; x < 8; ++x) {
         const int r = 8 * warp + x;
         if (r < L) {
-            la[x] = *reinterpret_cast<const float4 *>(sm + STG_LA + r * 512 + 16 * cq);
+            if constexpr (GATE) {         // log_alpha = -exp(A_log) softplus(f + dt_bias)
+                const uint2 fr = *reinterpret_cast<const uint2 *>(sm + STG_LA + r * 256 + 8 * cq);
+                la[x] = make_float4(-rate * softplus_f(bf_lo(fr.x) + bias[0]), -rate * softplus_f(bf_hi(fr.x) + bias[1]),
+                                    -rate * softplus_f(bf_lo(fr.y) + bias[2]), -rate * softplus_f(bf_hi(fr.y) + bias[3]));
+            } else {
+                la[x] = *reinterpret_cast<const float4 *>(sm + STG_LA + r * 512 + 16 * cq);
+            }
             kr[x] = *reinterpret_cast<const uint2 *>(sm + STG_K + r * 256 + 8 * cq);
             qr[x] = *reinterpret_cast<const uint2 *>(sm + STG_Q + r * 256 + 8 * cq);
         } else {
@@ -305,7 +327,10 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
     }
     if (tid < C) {
         const long long bi = (long long)(tok0 + tid) * H + h;
-        bet[tid] = (tid < L && in_bounds(p.status, bi, 1, p.tokens * H)) ? p.beta[bi] : 0.f;
+        float b = 0.f;
+        if (tid < L && in_bounds(p.status, bi, 1, p.tokens * H))
+            b = p.beta_logits ? 1.f / (1.f + __expf(-__bfloat162float(p.beta_logits[bi]))) : p.beta[bi];
+        bet[tid] = b;
     }
 
     // ---- decay scaling: per-thread products over its 8 rows, then over the 8 warps via smem
@@ -653,11 +678,16 @@ bool token_rows_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, ui
 
 }  // namespace
 
-cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slots, cudaStream_t stream)
+cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slots, cudaStream_t stream,
+                              const GateArgs *gate)
 {
     PrepParams p;
     p.q = (const __nv_bfloat16 *)a.q; p.k = (const __nv_bfloat16 *)a.k;
     p.log_alpha = a.log_alpha; p.beta = a.beta; p.cu_seqlens = a.cu_seqlens;
+    const bool fgate = gate && gate->f;
+    p.A_log = fgate ? gate->A_log : nullptr;
+    p.dt_bias = fgate ? gate->dt_bias : nullptr;
+    p.beta_logits = gate ? (const __nv_bfloat16 *)gate->beta_logits : nullptr;
     p.ws = ws; p.T = a.T; p.H = a.H; p.N = a.N; p.n_slots = n_slots; p.status = a.status;
     p.tokens = (long long)a.B * a.T;
     int dev = 0, sms = 0;
@@ -670,14 +700,15 @@ cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slo
     CUtensorMap tq, tk, tla;
     if (!token_rows_map(&tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, tokens) ||
         !token_rows_map(&tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, tokens) ||
-        !token_rows_map(&tla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.H, tokens))
+        !(fgate ? token_rows_map(&tla, gate->f, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, tokens)
+                : token_rows_map(&tla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.H, tokens)))
         return cudaErrorNotSupported;
 
-    cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_ALLOC);
+    auto kern = fgate ? chunk_prep_kernel<true> : chunk_prep_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)n_slots * (unsigned)a.H);
-    chunk_prep_kernel<<<grid, NT, SMEM_ALLOC, stream>>>(p, tq, tk, tla);
+    kern<<<grid, NT, SMEM_ALLOC, stream>>>(p, tq, tk, tla);
     return cudaGetLastError();
 }
 

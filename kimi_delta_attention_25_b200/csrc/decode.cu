@@ -16,6 +16,12 @@
 // state row (fully coalesced, 128-bit per thread). The reductions over rows for w and p are done
 // in registers, then across the 8 warps through shared memory. The state is touched exactly once
 // in each direction, with streaming (evict-first) cache hints since it is far larger than L2.
+//
+// With the layer options (GATE, NORM; the gate producers and the output norm of the KDA module,
+// lpnh.cn Kimi Linear article, sec. 3): alpha = exp(-exp(A_log[h]) softplus(f + dt_bias)) and
+// beta = sigmoid(b) are formed from their inputs as they are loaded, and the output becomes
+// o / sqrt(mean(o^2) + eps) * w * sigmoid(g), its sum of squares reduced across the four warps that
+// hold o at the barrier the state update already waits on.
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -24,11 +30,27 @@ namespace {
 constexpr int kDecThreads = 256;
 constexpr int kRowsPerWarp = kHeadDim / (kDecThreads / 32);   // 16
 
-template <typename T, typename TO>
+// Layer options of the decode step (pointers NULL when unused; f, b, g in the inputs' dtype).
+template <typename T>
+struct DecodeLayer {
+    const T *f;                 // decay gate input [N, H, dk]
+    const float *A_log;         // [H]
+    const float *dt_bias;       // [H * dk]
+    const T *b;                 // write gate logits [N, H]
+    const T *g;                 // output gate [N, H, dv]
+    const float *w;             // norm weight [dv]
+    float eps;
+    int H;
+};
+
+__device__ __forceinline__ float softplus_d(float x) { return x > 20.f ? x : log1pf(__expf(x)); }
+__device__ __forceinline__ float sigmoid_d(float x) { return 1.f / (1.f + __expf(-x)); }
+
+template <typename T, typename TO, bool GATE, bool NORM>
 __global__ void __launch_bounds__(kDecThreads, 2)
 decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
               const float *__restrict__ log_alpha, const float *__restrict__ beta,
-              float *__restrict__ S, TO *__restrict__ out)
+              float *__restrict__ S, TO *__restrict__ out, DecodeLayer<T> lay)
 {
     const int nh = blockIdx.x;                      // flat (sequence, head)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -36,6 +58,7 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
     __shared__ __align__(16) float s_u[kHeadDim];
     __shared__ __align__(16) float s_red[2][kDecThreads / 32][kHeadDim];
     __shared__ float s_qk;
+    __shared__ float s_ss[kHeadDim / 32];
 
     float *Sh = S + (size_t)nh * kHeadDim * kHeadDim;
     const int row0 = warp * kRowsPerWarp;
@@ -48,7 +71,12 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
 
     const size_t vec = (size_t)nh * kHeadDim;
     if (tid < kHeadDim) {
-        s_a[tid] = expf(log_alpha[vec + tid]);
+        if constexpr (GATE) {
+            const int h = nh % lay.H;
+            s_a[tid] = expf(-expf(lay.A_log[h]) * softplus_d(to_f32(lay.f[vec + tid]) + lay.dt_bias[(size_t)h * kHeadDim + tid]));
+        } else {
+            s_a[tid] = expf(log_alpha[vec + tid]);
+        }
         s_k[tid] = to_f32(k[vec + tid]);
         s_q[tid] = to_f32(q[vec + tid]);
     }
@@ -75,15 +103,31 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
     reinterpret_cast<float4 *>(s_red[1][warp])[lane] = wq;
     __syncthreads();
 
+    float o = 0.f;
     if (tid < kHeadDim) {
         float w = 0.f, p = 0.f;
 #pragma unroll
         for (int x = 0; x < kDecThreads / 32; ++x) { w += s_red[0][x][tid]; p += s_red[1][x][tid]; }
-        const float u = beta[nh] * (to_f32(v[vec + tid]) - w);
+        const float bt = lay.b ? sigmoid_d(to_f32(lay.b[nh])) : beta[nh];
+        const float u = bt * (to_f32(v[vec + tid]) - w);
         s_u[tid] = u;
-        out[vec + tid] = from_f32<TO>(p + s_qk * u);
+        o = p + s_qk * u;
+        if constexpr (NORM) {
+            float ss = o * o;
+#pragma unroll
+            for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+            if (lane == 0) s_ss[warp] = ss;
+        } else {
+            out[vec + tid] = from_f32<TO>(o);
+        }
     }
     __syncthreads();
+    if constexpr (NORM) {
+        if (tid < kHeadDim) {
+            const float rinv = rsqrtf((s_ss[0] + s_ss[1] + s_ss[2] + s_ss[3]) * (1.f / kHeadDim) + lay.eps);
+            out[vec + tid] = from_f32<TO>(o * rinv * lay.w[tid] * sigmoid_d(to_f32(lay.g[vec + tid])));
+        }
+    }
 
     const float4 u4 = reinterpret_cast<const float4 *>(s_u)[lane];
 #pragma unroll
@@ -99,15 +143,31 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
 
 template <typename T, typename TO>
 static void launch_typed(const void *q, const void *k, const void *v, const float *log_alpha,
-                         const float *beta, float *S, void *out, unsigned blocks, cudaStream_t stream)
+                         const float *beta, float *S, void *out, unsigned blocks, int H,
+                         const GateArgs *gate, const NormArgs *norm, cudaStream_t stream)
 {
-    decode_kernel<T, TO><<<blocks, kDecThreads, 0, stream>>>(
-        (const T *)q, (const T *)k, (const T *)v, log_alpha, beta, S, (TO *)out);
+    DecodeLayer<T> lay = {};
+    lay.H = H;
+    if (gate) {
+        lay.f = (const T *)gate->f; lay.A_log = gate->A_log; lay.dt_bias = gate->dt_bias;
+        lay.b = (const T *)gate->beta_logits;
+    }
+    if (norm) { lay.g = (const T *)norm->gate; lay.w = norm->weight; lay.eps = norm->eps; }
+    const bool fg = lay.f != nullptr, nm = norm != nullptr;
+    auto args = [&](auto kern) {
+        kern<<<blocks, kDecThreads, 0, stream>>>((const T *)q, (const T *)k, (const T *)v, log_alpha, beta, S,
+                                                 (TO *)out, lay);
+    };
+    if (fg && nm) args(decode_kernel<T, TO, true, true>);
+    else if (fg) args(decode_kernel<T, TO, true, false>);
+    else if (nm) args(decode_kernel<T, TO, false, true>);
+    else args(decode_kernel<T, TO, false, false>);
 }
 
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,
                           const float *beta, float *S, void *out, int N, int H,
-                          kda_dtype_t dtype, kda_dtype_t out_dtype, cudaStream_t stream)
+                          kda_dtype_t dtype, kda_dtype_t out_dtype, cudaStream_t stream,
+                          const GateArgs *gate, const NormArgs *norm)
 {
     const long long blocks = (long long)N * H;
     if (blocks == 0) return cudaSuccess;
@@ -115,13 +175,13 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const flo
     const unsigned nb = (unsigned)blocks;
     using bf = __nv_bfloat16;
     if (dtype == KDA_BF16 && out_dtype == KDA_BF16)
-        launch_typed<bf, bf>(q, k, v, log_alpha, beta, S, out, nb, stream);
+        launch_typed<bf, bf>(q, k, v, log_alpha, beta, S, out, nb, H, gate, norm, stream);
     else if (dtype == KDA_BF16)
-        launch_typed<bf, float>(q, k, v, log_alpha, beta, S, out, nb, stream);
+        launch_typed<bf, float>(q, k, v, log_alpha, beta, S, out, nb, H, gate, norm, stream);
     else if (out_dtype == KDA_BF16)
-        launch_typed<float, bf>(q, k, v, log_alpha, beta, S, out, nb, stream);
+        launch_typed<float, bf>(q, k, v, log_alpha, beta, S, out, nb, H, gate, norm, stream);
     else
-        launch_typed<float, float>(q, k, v, log_alpha, beta, S, out, nb, stream);
+        launch_typed<float, float>(q, k, v, log_alpha, beta, S, out, nb, H, gate, norm, stream);
     return cudaGetLastError();
 }
 

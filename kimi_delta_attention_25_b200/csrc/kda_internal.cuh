@@ -152,10 +152,28 @@ cudaError_t launch_chunk_fp32(const PrefillArgs &a, kda_dtype_t dtype, kda_dtype
 // Tensor-core (tcgen05) chunk path for bf16 q/k/v in one kernel (no workspace beyond the status).
 cudaError_t launch_chunk_tc(const PrefillArgs &a, kda_dtype_t out_dtype, cudaStream_t stream);
 
+// The layer's output norm, fused into the output epilogue when given: y = o / sqrt(mean(o^2) + eps)
+// * weight * sigmoid(gate), over the d_v channels of each head (gate in the inputs' dtype).
+struct NormArgs {
+    const void *gate;
+    const float *weight;
+    float eps;
+};
+
+// The layer's gate producers: log_alpha = -exp(A_log[h]) * softplus(f + dt_bias[h, c]) (f NULL:
+// log_alpha given), beta = sigmoid(beta_logits) (NULL: beta given); f and beta_logits in the inputs'
+// dtype.
+struct GateArgs {
+    const void *f;
+    const float *A_log, *dt_bias;
+    const void *beta_logits;
+};
+
 // Two-pass tensor-core chunk path for bf16 q/k/v: prepared operands go through the workspace.
-cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slots, cudaStream_t stream);
+cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slots, cudaStream_t stream,
+                              const GateArgs *gate = nullptr);
 cudaError_t launch_chunk_scan(const PrefillArgs &a, const unsigned char *ws, int n_slots,
-                              kda_dtype_t out_dtype, cudaStream_t stream);
+                              kda_dtype_t out_dtype, cudaStream_t stream, const NormArgs *norm = nullptr);
 
 // Backward pass (chunk_bwd.cu). Gradient pointers and the records of the forward kernel.
 struct BwdArgs {
@@ -171,9 +189,28 @@ struct BwdArgs {
 cudaError_t launch_chunk_bwd_scan(const BwdArgs &a, kda_dtype_t dtype, cudaStream_t stream);
 cudaError_t launch_chunk_bwd_local(const BwdArgs &a, kda_dtype_t dtype, cudaStream_t stream);
 
-// Decode step (memory-bound state update in place).
+// Decode step (memory-bound state update in place), optionally with the layer's gate producers
+// and output norm.
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,
                           const float *beta, float *S, void *out, int N, int H,
-                          kda_dtype_t dtype, kda_dtype_t out_dtype, cudaStream_t stream);
+                          kda_dtype_t dtype, kda_dtype_t out_dtype, cudaStream_t stream,
+                          const GateArgs *gate = nullptr, const NormArgs *norm = nullptr);
+
+// Stand-alone layer passes (layer.cu), used around the fp32 CUDA-core prefill: the gate producers
+// into fp32 log_alpha / beta, and the gated output norm of fp32 outputs o into out.
+cudaError_t launch_gates(const GateArgs &gate, float *log_alpha, float *beta, long long tokens, int H,
+                         kda_dtype_t dtype, cudaStream_t stream);
+cudaError_t launch_gated_norm(const float *o, const NormArgs &norm, void *out, long long rows,
+                              kda_dtype_t dtype, kda_dtype_t out_dtype, cudaStream_t stream);
+
+// Host-side argument checks of the prefill entry points (api.cu) and the launch arguments they build.
+kda_status_t check_prefill(const void *q, const void *k, const void *v, const float *log_alpha,
+                           const float *beta, const float *S0, const int32_t *cu_seqlens, const void *out,
+                           const float *S_final, int B, int T, int H, int N, int dk, int dv,
+                           kda_dtype_t dtype, kda_dtype_t out_dtype, const void *workspace,
+                           size_t workspace_bytes, bool need_qk, bool need_vout);
+PrefillArgs prefill_args(const void *q, const void *k, const void *v, const float *log_alpha,
+                         const float *beta, const float *S0, const int32_t *cu_seqlens, void *out,
+                         float *S_final, int B, int T, int H, int N, void *workspace, size_t workspace_bytes);
 
 }  // namespace kda

@@ -48,6 +48,83 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
     return true;
 }
 
+// Bounded wait for a role that is off the critical path: each try_wait asks the hardware to suspend
+// the thread until the phase completes (or up to `hint_ns`), so the waiting warp does not take issue
+// slots from the warps it shares a scheduler with.
+__device__ __forceinline__ bool mbar_wait_sleepy(uint64_t *bar, uint32_t parity, uint32_t hint_ns = 20000,
+                                                 long long budget = 4000000000LL) {
+    const long long t0 = clock64();
+    while (true) {
+        uint32_t ok;
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns) : "memory");
+        if (ok) return true;
+        if (clock64() - t0 > budget) return false;
+    }
+}
+
+// ------------------------------------------------------------------------------ clusters
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Address of the same shared-memory location in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t caddr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(caddr), "f"(v) : "memory");
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t caddr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(caddr) : "memory");
+    return v;
+}
+// Asynchronous 4-byte store into another CTA's shared memory that completes 4 transaction bytes on
+// an mbarrier in that CTA (both addresses through mapa_shared): the waiter on that mbarrier sees
+// the data once the phase completes, with no fence on the storing side.
+__device__ __forceinline__ void st_async_remote_f32(uint32_t caddr, float v, uint32_t cbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+                 ::"r"(caddr), "r"(__float_as_uint(v)), "r"(cbar) : "memory");
+}
+// The same with 16 bytes (address 16-byte aligned), completing 16 transaction bytes.
+__device__ __forceinline__ void st_async_remote_v4(uint32_t caddr, float a, float b, float c, float d, uint32_t cbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+                 ::"r"(caddr), "r"(__float_as_uint(a)), "r"(__float_as_uint(b)), "r"(__float_as_uint(c)),
+                   "r"(__float_as_uint(d)), "r"(cbar) : "memory");
+}
+// Arrive without ordering (relaxed) on an mbarrier in another CTA of the cluster.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t caddr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
+}
+// Arrive (release at cluster scope: this thread's earlier writes become visible to the waiter)
+// on an mbarrier in another CTA of the cluster, addressed through mapa_shared.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
+}
+// Bounded wait with acquire at cluster scope (sees writes released by remote arrivals).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, long long budget = 4000000000LL) {
+    const long long t0 = clock64();
+    while (true) {
+        uint32_t ok;
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+        if (ok) return true;
+        if (clock64() - t0 > budget) return false;
+    }
+}
+// Every thread of every CTA in the cluster (warp-uniform call sites only).
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // ------------------------------------------------------------------------------ fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
