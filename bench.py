@@ -666,7 +666,19 @@ def run_profile_case(args):
     import kimi_delta_attention_25_b200 as kda
     kda.load()
     dev = torch.device("cuda", 0)
-    if args.profile == "prefill":
+    if args.profile == "step":
+        # the headline step as timed (two passes, bf16 outputs), full size, `--steps` times
+        w = K.WORKLOADS[WORKLOAD]
+        d = K.make_prefill(w, device=dev)
+        out = torch.empty(w.B, w.T, w.H, D, dtype=torch.bfloat16, device=dev)
+        Sf = torch.empty(w.B, w.H, D, D, dtype=torch.float32, device=dev)
+        ws = torch.empty(kda.chunk_fwd_workspace_size(w.B, w.T, w.H, w.B), dtype=torch.uint8, device=dev)
+        for _ in range(args.steps):
+            kda.chunk_prep(d["q"], d["k"], d["log_alpha"], d["beta"], ws)
+            kda.chunk_scan(d["v"], ws, S0=d["S0"], out=out, S_final=Sf)
+        torch.cuda.synchronize()
+        assert kda.workspace_status(ws) == kda.KDA_OK
+    elif args.profile == "prefill":
         w = K.WORKLOADS[WORKLOAD]
         d = K.make_prefill(w, device=dev, T=args.tokens)
         for _ in range(2):
@@ -701,7 +713,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["prefill", "decode", "backward"], default=None,
+    ap.add_argument("--profile", choices=["step", "prefill", "decode", "backward"], default=None,
                     help="run one small case for an Nsight Compute capture instead of the benchmark")
     ap.add_argument("--tokens", type=int, default=32768, help="tokens of the --profile prefill case")
     args = ap.parse_args()

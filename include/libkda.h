@@ -285,6 +285,45 @@ kda_status_t kda_decode_step_layer(const void *q, const void *k, const void *v,
                                    int N, int H, int dk, int dv, kda_dtype_t dtype,
                                    kda_dtype_t out_dtype, const kda_layer_opts_t *opts, void *stream);
 
+/* ---------------------------------------------------------------------------------------------
+ * Short causal convolution in front of q, k and v, and its decode step. The layer config sets
+ * short_conv_kernel_size 4 and the cache keeps conv_states beside the recurrent states (lpnh.cn
+ * Kimi Linear KDA/NoPE article, sec. 3 and 6); no formula is printed. Reading used: a depthwise
+ * convolution over tokens, per channel c,
+ *     y[t,c] = act(bias[c] + sum_{j=0}^{K-1} weight[c,j] * x[t-K+1+j, c])   (taps oldest first)
+ * with the inputs before a sequence's first token taken from its conv state, act = SiLU when
+ * activation_silu is 1 (identity when 0), then, when normalize_head_dim = 128, each consecutive
+ * 128-channel head vector divided by sqrt(|y|^2 + 1e-6) (the unit-norm q and k of the recurrence).
+ *
+ *   x, y        [B,T,D] (packed: B = 1 and cu_seqlens as for kda_chunk_fwd) in dtype; D a multiple
+ *               of 128 (for example H * 128 channels of q); 16-byte aligned
+ *   weight      [D,K] float32; bias [D] float32 or NULL; 1 <= K <= 8
+ *   conv_state  [N,D,K-1] float32, the last K-1 inputs before each sequence, oldest first, or NULL
+ *               (zeros); conv_state_out [N,D,K-1] float32 or NULL: written with the last K-1 inputs
+ *               of each sequence (the old state shifted in for sequences shorter than K-1); it may
+ *               be the same buffer as conv_state.
+ * kda_short_conv_step: one token per sequence, x and y [N,D], conv_state [N,D,K-1] read and
+ * updated in place.
+ * Errors: KDA_ERR_INVALID_ARG (sizes, pointers, alignment), KDA_ERR_UNSUPPORTED (D not a multiple
+ * of 128, K > 8, normalize_head_dim other than 0 or 128), KDA_ERR_CUDA. */
+kda_status_t kda_short_conv(const void *x, const float *weight, const float *bias,
+                            const float *conv_state, float *conv_state_out, const int32_t *cu_seqlens,
+                            void *y, int B, int T, int N, int D, int K, int activation_silu,
+                            int normalize_head_dim, kda_dtype_t dtype, void *stream);
+kda_status_t kda_short_conv_step(const void *x, const float *weight, const float *bias,
+                                 float *conv_state, void *y, int N, int D, int K, int activation_silu,
+                                 int normalize_head_dim, kda_dtype_t dtype, void *stream);
+
+/* S_out[h] = Phi[h] S_in[h] + Psi[h] for every head (float32, [H,dk,dv], Phi [H,dk,dk]; Psi may be
+ * NULL for zero). A segment of the recurrence maps the state entering it to the state leaving it
+ * affinely, S -> Phi S + Psi: Phi is S_final of the segment run from S0 = I with v = 0, and Psi is
+ * S_final run from S0 = 0. Composing the maps of consecutive segments gives each segment's entering
+ * state without running the earlier segments again: the exchange step of a sequence split across
+ * devices (context-parallel prefill). The pages do not describe this split; it follows from the
+ * recurrence being linear in the state. S_out must not alias S_in or Phi (KDA_ERR_INVALID_ARG). */
+kda_status_t kda_state_affine(const float *Phi, const float *S_in, const float *Psi, float *S_out,
+                              int H, int dk, int dv, void *stream);
+
 /* Capacity of the library-owned scratch array used by kda_chunk_fwd_noalloc (bytes). */
 #define KDA_NOALLOC_SCRATCH_BYTES 4096
 

@@ -38,7 +38,8 @@ _lib = None
 # Every entry point declared in include/libkda.h.
 EXPORTS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
            "kda_chunk_fwd_layer_workspace_size", "kda_chunk_fwd_layer", "kda_chunk_prep_layer",
-           "kda_chunk_scan_layer", "kda_decode_step_layer",
+           "kda_chunk_scan_layer", "kda_decode_step_layer", "kda_short_conv", "kda_short_conv_step",
+           "kda_state_affine",
            "kda_workspace_status", "kda_status_string", "kda_version", "kda_chunk_fwd_noalloc",
            "kda_chunk_prep", "kda_chunk_scan", "kda_selftest_wait_timeout",
            "kda_chunk_bwd_workspace_size", "kda_chunk_bwd", "kda_chunk_bwd_phase",
@@ -123,6 +124,12 @@ def load():
     lib.kda_chunk_scan_layer.restype = I
     lib.kda_decode_step_layer.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, LP, P]
     lib.kda_decode_step_layer.restype = I
+    lib.kda_short_conv.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P]
+    lib.kda_short_conv.restype = I
+    lib.kda_short_conv_step.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P]
+    lib.kda_short_conv_step.restype = I
+    lib.kda_state_affine.argtypes = [P, P, P, P, I, I, I, P]
+    lib.kda_state_affine.restype = I
     _lib = lib
     return lib
 
@@ -404,3 +411,59 @@ def pad(y: torch.Tensor, indices: torch.Tensor, B: int, T: int, fill: float = 0.
     flat = torch.full((B * T, *y.shape[2:]), fill, dtype=y.dtype, device=y.device)
     flat.index_copy_(0, indices, y.reshape(-1, *y.shape[2:]))
     return flat.reshape(B, T, *y.shape[2:])
+
+
+# ---- short causal convolution and state composition --------------------------------------------
+
+def short_conv(x, weight, bias=None, conv_state=None, cu_seqlens=None, out=None, conv_state_out=None,
+               activation="silu", normalize_head_dim=0):
+    """``kda_short_conv``: x [B,T,D] (float32 or bfloat16, D a multiple of 128), weight [D,K] fp32,
+    bias [D] fp32 or None, conv_state [N,D,K-1] fp32 or None (zeros). Returns (y [B,T,D] in x's
+    dtype, conv_state_out [N,D,K-1] or None); pass ``conv_state_out=conv_state`` to update in place,
+    or ``conv_state_out=True`` for a new tensor. ``normalize_head_dim=128`` L2-normalises each head."""
+    lib = load()
+    B, T, D = x.shape
+    K = weight.shape[1]
+    N = B if cu_seqlens is None else cu_seqlens.shape[0] - 1
+    if out is None:
+        out = torch.empty_like(x)
+    if conv_state_out is True:
+        conv_state_out = torch.empty(N, D, K - 1, dtype=torch.float32, device=x.device)
+    _need_cuda(x, weight, bias, conv_state, cu_seqlens, out, conv_state_out)
+    st = lib.kda_short_conv(_ptr(x), _ptr(weight), _ptr(bias), _ptr(conv_state), _ptr(conv_state_out),
+                            _ptr(cu_seqlens), _ptr(out), B, T, N, D, K, 1 if activation == "silu" else 0,
+                            int(normalize_head_dim), _dtype_code(x), _stream(x.device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_short_conv")
+    return out, conv_state_out
+
+
+def short_conv_step(x, weight, conv_state, bias=None, out=None, activation="silu", normalize_head_dim=0):
+    """``kda_short_conv_step``: one token per sequence, x [N,D]; conv_state [N,D,K-1] fp32 is
+    updated in place. Returns y [N,D]."""
+    lib = load()
+    N, D = x.shape
+    K = weight.shape[1]
+    if out is None:
+        out = torch.empty_like(x)
+    _need_cuda(x, weight, bias, conv_state, out)
+    st = lib.kda_short_conv_step(_ptr(x), _ptr(weight), _ptr(bias), _ptr(conv_state), _ptr(out), N, D, K,
+                                 1 if activation == "silu" else 0, int(normalize_head_dim), _dtype_code(x),
+                                 _stream(x.device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_short_conv_step")
+    return out
+
+
+def state_affine(Phi, S_in, Psi=None, out=None):
+    """``kda_state_affine``: Phi [H,dk,dk] @ S_in [H,dk,dv] + Psi per head (fp32)."""
+    lib = load()
+    H, dk, dv = S_in.shape
+    if out is None:
+        out = torch.empty_like(S_in)
+    _need_cuda(Phi, S_in, Psi, out)
+    st = lib.kda_state_affine(_ptr(Phi), _ptr(S_in), _ptr(Psi), _ptr(out), H, dk, dv, _stream(S_in.device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_state_affine")
+    return out
+
