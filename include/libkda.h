@@ -328,16 +328,15 @@ kda_status_t kda_state_affine(const float *Phi, const float *S_in, const float *
 #define KDA_NOALLOC_SCRATCH_BYTES 4096
 
 /* kda_chunk_fwd without a workspace argument, for callers that cannot allocate device memory:
- * code running while a CUDA graph is being captured (allocating there is not allowed and would
- * break the capture), plug-ins whose host runtime owns all device memory and passes in only the
- * input and output buffers, and memory-capped servers that may not grow their footprint per call.
+ * plug-ins whose host runtime owns all device memory and passes in only the input and output
+ * buffers, and memory-capped servers that may not grow their footprint per call.
  * The pages describe no such entry point; it has no counterpart there.
  *
  * Arguments, layouts and results are those of kda_chunk_fwd; the caller still passes (and owns)
  * every input and output. Instead of a workspace, the library uses a static device array of
  * KDA_NOALLOC_SCRATCH_BYTES that every GPU on which the library is loaded holds until the process
  * exits. The first call on a device looks up that array's device address (with the device
- * current) and caches it; make that first call before any stream capture begins. bf16 inputs run
+ * current) and caches it. bf16 inputs run
  * the single-kernel prefill, whose only scratch is the 256-byte status header (a scratch need
  * beyond the array would be refused with KDA_ERR_UNSUPPORTED); it is slower than the two-pass
  * prefill kda_chunk_fwd runs with its workspace, and its f16 tensor-core operands narrow the

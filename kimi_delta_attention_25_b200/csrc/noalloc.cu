@@ -1,10 +1,9 @@
 // noalloc.cu -- kda_chunk_fwd_noalloc: the chunked prefill for callers that cannot allocate
 // device memory.
 //
-// Who needs it: code that runs while a CUDA graph is being captured (allocation calls are not
-// allowed inside a capture and would break it), plug-ins hosted by a runtime that owns all device
-// memory and hands out only fixed input/output buffers, and memory-capped serving processes that
-// must not grow their footprint per request. kda_chunk_fwd asks such callers for a workspace they
+// Who needs it: plug-ins hosted by a runtime that owns all device memory and hands out only fixed
+// input/output buffers, and memory-capped serving processes that must not grow their footprint
+// per request. kda_chunk_fwd asks such callers for a workspace they
 // cannot provide; this entry point instead uses a small scratch array that is part of the library
 // image itself.
 //

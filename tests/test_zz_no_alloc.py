@@ -1,5 +1,5 @@
 """kda_chunk_fwd_noalloc, the prefill entry point for callers that cannot allocate device memory
-(code running inside a CUDA-graph capture, or hosted by a runtime that owns all device memory).
+(code hosted by a runtime that owns all device memory, or a process whose footprint is capped).
 
 Called through the C ABI twice in a row on each case, every result is checked against the float64
 oracle within the tolerance the parity tests use (2e-2 of RMS for bf16 inputs, 1e-4 for fp32), and
