@@ -41,7 +41,6 @@ D = 128
 # (256 B; the output takes the inputs' dtype), log_alpha fp32 (512 B), beta fp32 (4 B)
 PREFILL_BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 2 + D * 4 + 4
 # kernels one prefill step launches: the chunk-preparation pass and the state scan
-PREFILL_KERNELS_PER_STEP = 2
 # the same algorithmic bytes, split by the pass that moves them: the preparation pass reads q, k,
 # log_alpha and beta; the scan reads v and writes out (its other traffic is the workspace)
 PREP_BYTES_PER_TOKEN_HEAD = 2 * D * 2 + D * 4 + 4
@@ -291,41 +290,19 @@ def run_native(args):
         kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"],
                       out=out, S_final=Sf, workspace=work)
 
+    def prep():
+        kda.chunk_prep(d["q"], d["k"], d["log_alpha"], d["beta"], work)
+
+    def scan():
+        kda.chunk_scan(d["v"], work, S0=d["S0"], out=out, S_final=Sf)
+
     step()
     torch.cuda.synchronize()
     assert kda.workspace_status(work) == kda.KDA_OK
-
-    # One timed step = the two passes through their own entry points (exactly what chunk_fwd
-    # runs), with CUDA events on the launching stream around each pass.
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-
-    def step_passes(ev=None):
-        if ev is not None:
-            ev[0].record()
-        kda.chunk_prep(d["q"], d["k"], d["log_alpha"], d["beta"], work)
-        if ev is not None:
-            ev[1].record()
-        kda.chunk_scan(d["v"], work, S0=d["S0"], out=out, S_final=Sf)
-        if ev is not None:
-            ev[2].record()
-
-    with Clocks(local) as clk:
-        for _ in range(args.warmup):
-            step_passes()
-        torch.cuda.synchronize()
-        barrier(ws)
-        torch.cuda.synchronize()
-        t_s, t_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        t_s.record()
-        for i in range(args.steps):
-            step_passes(evs[i])
-        t_e.record()
-        torch.cuda.synchronize()
-        barrier(ws)
+    # the step is the public call (one timed step = one chunk_fwd); each pass is also timed alone
+    ms, ms_prep, ms_scan, clk = time_prefill(kda, ws, args, step, prep, scan, args.steps, local)
     assert kda.workspace_status(work) == kda.KDA_OK
-    ms = max_over_ranks(t_s.elapsed_time(t_e) / args.steps, ws)
-    ms_prep = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    ms_scan = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    launches = kda.chunk_fwd_kernel_launches(B, T, H, B)
     tokens = B * T
     value = ws * tokens / (ms * 1e-3) / 1e6                   # Mtok/s, whole job
     th = B * T * H
@@ -405,7 +382,7 @@ def run_native(args):
                                   "tensor_tflops_useful": tfs, "tensor_frac_useful": tfs / pk["bf16"]}},
             "e2e": {"value": e2e_val, "unit": "Mtok/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
-            "gpu_launches": args.steps * PREFILL_KERNELS_PER_STEP,
+            "gpu_launches": args.steps * launches,
             "clocks": clk.summary(),
             "layer_step": layer_step,
             "configs": other,
@@ -416,6 +393,41 @@ def run_native(args):
         print(json.dumps(line), flush=True)
     if ws > 1:
         torch.distributed.destroy_process_group()
+
+
+def time_prefill(kda, ws, args, fwd, prep, scan, steps, local):
+    """Times `steps` calls of the public prefill call fwd() between a barrier + synchronize on both
+    sides (the step; with few (sequence, head) chains the library runs its two passes as a
+    pipeline over token ranges, so they overlap inside the call), then the two passes alone, each
+    between CUDA events on the launching stream, for the per-kernel rooflines. Returns the step time
+    (max over ranks), the mean time of each pass and the clock record of the step's timed region."""
+    with Clocks(local) as clk:
+        for _ in range(args.warmup):
+            fwd()
+        torch.cuda.synchronize()
+        barrier(ws)
+        torch.cuda.synchronize()
+        t_s, t_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t_s.record()
+        for _ in range(steps):
+            fwd()
+        t_e.record()
+        torch.cuda.synchronize()
+        barrier(ws)
+    ms = max_over_ranks(t_s.elapsed_time(t_e) / steps, ws)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    prep()
+    scan()
+    for ev in evs:
+        ev[0].record()
+        prep()
+        ev[1].record()
+        scan()
+        ev[2].record()
+    torch.cuda.synchronize()
+    ms_prep = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    ms_scan = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    return ms, ms_prep, ms_scan, clk
 
 
 def run_prefill_config(kda, dev, pk, ws, rank, args, name, cpu_budget_s):
@@ -433,38 +445,24 @@ def run_prefill_config(kda, dev, pk, ws, rank, args, name, cpu_budget_s):
     Sf = torch.empty(N, H, D, D, dtype=torch.float32, device=dev)
     work = torch.empty(max(256, kda.chunk_fwd_workspace_size(B, T, H, N)), dtype=torch.uint8, device=dev)
     steps = max(3, args.steps)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
 
-    def passes(ev=None):
-        if ev is not None:
-            ev[0].record()
+    def fwd():
+        kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"], cu_seqlens=cu,
+                      out=out, S_final=Sf, workspace=work)
+
+    def prep():
         kda.chunk_prep(d["q"], d["k"], d["log_alpha"], d["beta"], work, cu_seqlens=cu)
-        if ev is not None:
-            ev[1].record()
-        kda.chunk_scan(d["v"], work, S0=d["S0"], cu_seqlens=cu, out=out, S_final=Sf)
-        if ev is not None:
-            ev[2].record()
 
-    with Clocks(int(os.environ.get("LOCAL_RANK", "0"))) as clk:
-        for _ in range(args.warmup):
-            passes()
-        torch.cuda.synchronize()
-        barrier(ws)
-        torch.cuda.synchronize()
-        t_s, t_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        t_s.record()
-        for i in range(steps):
-            passes(evs[i])
-        t_e.record()
-        torch.cuda.synchronize()
-        barrier(ws)
+    def scan():
+        kda.chunk_scan(d["v"], work, S0=d["S0"], cu_seqlens=cu, out=out, S_final=Sf)
+
+    ms, ms_prep, ms_scan, clk = time_prefill(kda, ws, args, fwd, prep, scan, steps,
+                                             int(os.environ.get("LOCAL_RANK", "0")))
     assert kda.workspace_status(work) == kda.KDA_OK
-    ms = max_over_ranks(t_s.elapsed_time(t_e) / steps, ws)
     th = B * T * H
     kern = {}
-    for i, (kname, per) in enumerate((("chunk_prep", PREP_BYTES_PER_TOKEN_HEAD),
-                                      ("chunk_scan", SCAN_BYTES_PER_TOKEN_HEAD))):
-        t_ms = statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+    for kname, t_ms, per in (("chunk_prep", ms_prep, PREP_BYTES_PER_TOKEN_HEAD),
+                             ("chunk_scan", ms_scan, SCAN_BYTES_PER_TOKEN_HEAD)):
         a = th * per / (t_ms * 1e-3) / 1e9
         kern[kname] = {"ms": t_ms, "achieved": a, "frac": a / pk["hbm"]}
     gbs = th * PREFILL_BYTES_PER_TOKEN_HEAD / (ms * 1e-3) / 1e9
@@ -477,7 +475,7 @@ def run_prefill_config(kda, dev, pk, ws, rank, args, name, cpu_budget_s):
                         "kernels": kern,
                         "step": {"achieved": gbs, "frac": gbs / pk["hbm"], "tensor_tflops_useful": tfs,
                                  "tensor_frac_useful": tfs / pk["bf16"]}},
-           "gpu_launches": 2 * steps, "clocks": clk.summary()}
+           "gpu_launches": steps * kda.chunk_fwd_kernel_launches(B, T, H, N), "clocks": clk.summary()}
     del d, out, Sf, work
     torch.cuda.empty_cache()
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -501,37 +499,23 @@ def run_layer_step(kda, dev, pk, ws, rank, args, d):
     Sf = torch.empty(B, H, D, D, dtype=torch.float32, device=dev)
     work = torch.empty(max(256, kda.chunk_fwd_workspace_size(B, T, H, B)), dtype=torch.uint8, device=dev)
     steps = max(3, args.steps)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
 
-    def passes(ev=None):
-        if ev is not None:
-            ev[0].record()
+    def fwd():
+        kda.chunk_fwd(d["q"], d["k"], d["v"], None, None, S0=d["S0"], out=out, S_final=Sf, workspace=work,
+                      layer=opts)
+
+    def prep():
         kda.chunk_prep(d["q"], d["k"], None, None, work, layer=opts)
-        if ev is not None:
-            ev[1].record()
-        kda.chunk_scan(d["v"], work, S0=d["S0"], out=out, S_final=Sf, layer=opts)
-        if ev is not None:
-            ev[2].record()
 
-    with Clocks(int(os.environ.get("LOCAL_RANK", "0"))) as clk:
-        for _ in range(args.warmup):
-            passes()
-        torch.cuda.synchronize()
-        barrier(ws)
-        torch.cuda.synchronize()
-        t_s, t_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        t_s.record()
-        for i in range(steps):
-            passes(evs[i])
-        t_e.record()
-        torch.cuda.synchronize()
-        barrier(ws)
+    def scan():
+        kda.chunk_scan(d["v"], work, S0=d["S0"], out=out, S_final=Sf, layer=opts)
+
+    ms, ms_prep, ms_scan, clk = time_prefill(kda, ws, args, fwd, prep, scan, steps,
+                                             int(os.environ.get("LOCAL_RANK", "0")))
     assert kda.workspace_status(work) == kda.KDA_OK
-    ms = max_over_ranks(t_s.elapsed_time(t_e) / steps, ws)
     th = B * T * H
     gbs = th * LAYER_BYTES_PER_TOKEN_HEAD / (ms * 1e-3) / 1e9
-    kern = {"chunk_prep_gates": {"ms": statistics.mean(e[0].elapsed_time(e[1]) for e in evs)},
-            "chunk_scan_norm": {"ms": statistics.mean(e[1].elapsed_time(e[2]) for e in evs)}}
+    kern = {"chunk_prep_gates": {"ms": ms_prep}, "chunk_scan_norm": {"ms": ms_scan}}
     del out, Sf, work, lay, opts
     torch.cuda.empty_cache()
     return {"workload": WORKLOAD, "ms_per_step": ms, "Mtok_s": ws * B * T / (ms * 1e-3) / 1e6, "steps": steps,
@@ -540,7 +524,8 @@ def run_layer_step(kda, dev, pk, ws, rank, args, d):
             "algorithmic_bytes_per_token_head": LAYER_BYTES_PER_TOKEN_HEAD,
             "roofline_step": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
                               "frac": gbs / pk["hbm"], "peak_source": "of %s" % pk["src"]},
-            "kernels": kern, "gpu_launches": 2 * steps, "clocks": clk.summary()}
+            "kernels": kern, "gpu_launches": steps * kda.chunk_fwd_kernel_launches(B, T, H, B),
+            "clocks": clk.summary()}
 
 
 def run_decode(kda, dev, pk, ws, local, args):

@@ -75,10 +75,17 @@ typedef enum {
  * the first 256 bytes hold the device status word read by kda_workspace_status).
  * For bf16 inputs the workspace also holds the per-chunk operands that the first of the
  * two prefill passes prepares for the second: 66048 bytes per (chunk slot, head), with
- * floor(B*T/64) + N + 1 chunk slots per head (about 1 KiB per token and head).
+ * floor(B*T/64) + N + 1 chunk slots per head (about 1 KiB per token and head), and, when
+ * kda_chunk_fwd pipelines its two passes (see there), N*H*dk*dv*4 bytes that carry the state
+ * between token ranges.
  * Returns 0 for sizes kda_chunk_fwd would reject. */
 size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int N, int dk, int dv,
                                     kda_dtype_t dtype);
+
+/* Number of kernels one kda_chunk_fwd call with these sizes launches (for profiling and launch
+ * accounting; the bf16 layer variant kda_chunk_fwd_layer launches as many). 0 for sizes the call
+ * rejects or that launch nothing. */
+int kda_chunk_fwd_kernel_launches(int B, int T, int H, int N, kda_dtype_t dtype);
 
 /* Chunkwise-parallel prefill (chunk of 64 tokens): the recurrence above over
  * every sequence and head, returning every o_t and the final state.
@@ -104,7 +111,12 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int N, int dk, int dv,
  *   workspace  device buffer of kda_chunk_fwd_workspace_size(...) bytes,
  *              workspace_bytes its size. Its status word is cleared by this call.
  * S0 and S_final may alias (in-place continuation); no other buffers may overlap.
- * T = 0 or N = 0 is valid (only S_final = S0 is written). */
+ * T = 0 or N = 0 is valid (only S_final = S0 is written).
+ * For bf16 inputs with at most 64 (sequence, head) pairs and at least 32 chunk slots the two
+ * passes run as a pipeline over up to 16 token ranges: the state scan of one range beside the
+ * preparation of the later ones, on two library-owned streams (created on the first such call per
+ * device) that fork from `stream` and join it again; everything stays ordered on `stream`. Between
+ * ranges the state is carried in S_final (or the workspace when S_final is NULL). */
 kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v,
                            const float *log_alpha, const float *beta,
                            const float *S0, const int32_t *cu_seqlens,

@@ -43,7 +43,7 @@ EXPORTS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
            "kda_workspace_status", "kda_status_string", "kda_version", "kda_chunk_fwd_noalloc",
            "kda_chunk_prep", "kda_chunk_scan", "kda_selftest_wait_timeout",
            "kda_chunk_bwd_workspace_size", "kda_chunk_bwd", "kda_chunk_bwd_phase",
-           "kda_chunk_fwd_noalloc_status")
+           "kda_chunk_fwd_noalloc_status", "kda_chunk_fwd_kernel_launches")
 
 
 class LayerOpts(ctypes.Structure):
@@ -88,6 +88,8 @@ def load():
     P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     lib.kda_chunk_fwd_workspace_size.argtypes = [I, I, I, I, I, I, I]
     lib.kda_chunk_fwd_workspace_size.restype = Z
+    lib.kda_chunk_fwd_kernel_launches.argtypes = [I, I, I, I, I]
+    lib.kda_chunk_fwd_kernel_launches.restype = I
     lib.kda_chunk_fwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P]
     lib.kda_chunk_fwd.restype = I
     lib.kda_decode_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P]
@@ -165,6 +167,12 @@ def _stream(device) -> ctypes.c_void_p:
 def chunk_fwd_workspace_size(B, T, H, N, dk=128, dv=128, dtype=torch.bfloat16) -> int:
     code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
     return int(load().kda_chunk_fwd_workspace_size(B, T, H, N, dk, dv, code))
+
+
+def chunk_fwd_kernel_launches(B, T, H, N, dtype=torch.bfloat16) -> int:
+    """Kernels one ``chunk_fwd`` call with these sizes launches (``kda_chunk_fwd_kernel_launches``)."""
+    code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    return int(load().kda_chunk_fwd_kernel_launches(B, T, H, N, code))
 
 
 def chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, S_final=None,

@@ -39,8 +39,10 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int N, int dk, int dv, 
     if (B < 0 || T < 0 || H <= 0 || N < 0 || dk != kHeadDim || dv != kHeadDim) return 0;
     if (dtype != KDA_F32 && dtype != KDA_BF16) return 0;
     if (dtype == KDA_F32) return kStatusBytes;
-    // bf16: prepared operands of every (chunk slot, head)
-    return kStatusBytes + (size_t)H * (size_t)prep_slots((long long)B * T, N) * kPrepBlockBytes;
+    // bf16: prepared operands of every (chunk slot, head), then the state carried between the token
+    // ranges of the pipelined prefill (when it applies)
+    return kStatusBytes + (size_t)H * (size_t)prep_slots((long long)B * T, N) * kPrepBlockBytes +
+           prefill_carry_bytes((long long)B * T, H, N);
 }
 
 }  // extern "C"
@@ -117,12 +119,7 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v,
     if (N == 0) return KDA_OK;
     const PrefillArgs a = prefill_args(q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final,
                                        B, T, H, N, workspace, workspace_bytes);
-    if (dtype == KDA_BF16) {
-        const int n_slots = (int)prep_slots((long long)B * T, N);
-        cudaError_t e = launch_chunk_prep(a, (unsigned char *)a.scratch, n_slots, st);
-        if (e == cudaSuccess) e = launch_chunk_scan(a, (const unsigned char *)a.scratch, n_slots, out_dtype, st);
-        return map_cuda(e);
-    }
+    if (dtype == KDA_BF16) return map_cuda(run_prefill_bf16(a, out_dtype, st, nullptr, nullptr));
     return map_cuda(launch_chunk_fp32(a, dtype, out_dtype, st));
 }
 
@@ -155,6 +152,14 @@ kda_status_t kda_chunk_scan(const void *v, const float *S0, const int32_t *cu_se
                                        B, T, H, N, workspace, workspace_bytes);
     return map_cuda(launch_chunk_scan(a, (const unsigned char *)a.scratch, (int)prep_slots((long long)B * T, N), out_dtype,
                                       (cudaStream_t)stream));
+}
+
+int kda_chunk_fwd_kernel_launches(int B, int T, int H, int N, kda_dtype_t dtype)
+{
+    if (B < 0 || T < 0 || H <= 0 || N < 0 || (dtype != KDA_F32 && dtype != KDA_BF16)) return 0;
+    if (N == 0) return 0;
+    if (dtype == KDA_F32) return 1;
+    return prefill_launches((long long)B * T, H, N);
 }
 
 size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int N, int dk, int dv)

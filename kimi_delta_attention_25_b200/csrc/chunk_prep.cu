@@ -107,6 +107,7 @@ struct PrepParams {
     const int32_t *cu_seqlens;
     unsigned char *ws;              // chunk blocks, [H][n_slots][kPrepBlockBytes]
     int T, H, N, n_slots;
+    int slot_base;                  // first chunk slot of this launch (the grid covers slots from here)
     long long tokens;               // B * T (rows of q, k, log_alpha; beta has tokens * H entries)
     int prefetch_wave;              // CTAs resident at once; > 0: prefetch that many units ahead
     int32_t *status;
@@ -248,7 +249,7 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
     // head fastest: the CTAs resident at one time cover all heads of a few consecutive chunks, so
     // together they read whole [token][head][channel] rows of q, k and log_alpha (DRAM pages are
     // used in full; with one head per row window each 8 KB row would give up 256 bytes)
-    const int h = (int)(blockIdx.x % (unsigned)p.H), slot = (int)(blockIdx.x / (unsigned)p.H);
+    const int h = (int)(blockIdx.x % (unsigned)p.H), slot = p.slot_base + (int)(blockIdx.x / (unsigned)p.H);
     const int H = p.H;
 
     int64_t tok0;
@@ -284,7 +285,7 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
             const long long nxt = (long long)blockIdx.x + p.prefetch_wave;
             int64_t ptok;
             int pL;
-            if (nxt < (long long)gridDim.x && slot_chunk(p, (int)(nxt / H), &ptok, &pL)) {
+            if (nxt < (long long)gridDim.x && slot_chunk(p, p.slot_base + (int)(nxt / H), &ptok, &pL)) {
                 const int ph = (int)(nxt % H);
                 tma_prefetch_3d(&tm_q, 0, ph, (int)ptok);
                 tma_prefetch_3d(&tm_k, 0, ph, (int)ptok);
@@ -643,7 +644,6 @@ chunk_prep_kernel(PrepParams p, const __grid_constant__ CUtensorMap tm_q, const 
     if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-// Tensor map of a [tokens][H][128] row-major tensor whose box is the 64 token rows of one head.
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -662,25 +662,28 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
+}  // namespace
+
 bool token_rows_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint32_t elem_bytes, int H,
-                    long long tokens)
+                    long long tokens, uint32_t box_cols, bool swizzle128)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)DK, (cuuint64_t)H, (cuuint64_t)tokens};
     const cuuint64_t strides[2] = {(cuuint64_t)DK * elem_bytes, (cuuint64_t)DK * elem_bytes * H};
-    const cuuint32_t box[3] = {(cuuint32_t)DK, 1u, (cuuint32_t)C};
+    const cuuint32_t box[3] = {box_cols, 1u, (cuuint32_t)C};
     const cuuint32_t estr[3] = {1u, 1u, 1u};
     return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+              swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-
 cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slots, cudaStream_t stream,
-                              const GateArgs *gate)
+                              const GateArgs *gate, int slot_lo, int slot_hi)
 {
+    if (slot_hi < 0 || slot_hi > n_slots) slot_hi = n_slots;
+    if (slot_lo < 0) slot_lo = 0;
+    if (slot_lo >= slot_hi) return cudaSuccess;
     PrepParams p;
     p.q = (const __nv_bfloat16 *)a.q; p.k = (const __nv_bfloat16 *)a.k;
     p.log_alpha = a.log_alpha; p.beta = a.beta; p.cu_seqlens = a.cu_seqlens;
@@ -689,6 +692,7 @@ cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slo
     p.dt_bias = fgate ? gate->dt_bias : nullptr;
     p.beta_logits = gate ? (const __nv_bfloat16 *)gate->beta_logits : nullptr;
     p.ws = ws; p.T = a.T; p.H = a.H; p.N = a.N; p.n_slots = n_slots; p.status = a.status;
+    p.slot_base = slot_lo;
     p.tokens = (long long)a.B * a.T;
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -707,7 +711,7 @@ cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slo
     auto kern = fgate ? chunk_prep_kernel<true> : chunk_prep_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)n_slots * (unsigned)a.H);
+    const dim3 grid((unsigned)(slot_hi - slot_lo) * (unsigned)a.H);
     kern<<<grid, NT, SMEM_ALLOC, stream>>>(p, tq, tk, tla);
     return cudaGetLastError();
 }

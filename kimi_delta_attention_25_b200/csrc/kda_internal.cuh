@@ -1,6 +1,7 @@
 // kda_internal.cuh -- shared device helpers and launcher prototypes of libkda.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -169,11 +170,35 @@ struct GateArgs {
     const void *beta_logits;
 };
 
+// Tensor map of a [tokens][H][128] row-major tensor whose box is `box_cols` channels of the 64 token
+// rows of one head, without swizzle or with the 128-byte swizzle (box_cols * elem_bytes = 128).
+bool token_rows_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint32_t elem_bytes, int H,
+                    long long tokens, uint32_t box_cols = kHeadDim, bool swizzle128 = false);
+
 // Two-pass tensor-core chunk path for bf16 q/k/v: prepared operands go through the workspace.
+// (slots [slot_lo, slot_hi) only; slot_hi < 0: to the end)
 cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slots, cudaStream_t stream,
-                              const GateArgs *gate = nullptr);
+                              const GateArgs *gate = nullptr, int slot_lo = 0, int slot_hi = -1);
 cudaError_t launch_chunk_scan(const PrefillArgs &a, const unsigned char *ws, int n_slots,
                               kda_dtype_t out_dtype, cudaStream_t stream, const NormArgs *norm = nullptr);
+// The same pass with one CTA per (sequence, head) over all value columns (chunk_scan_wide.cu), for the
+// chunks whose slots lie in [slot_lo, slot_hi); a range that does not start a sequence starts from
+// S_final, which must then be given.
+cudaError_t launch_chunk_scan_wide(const PrefillArgs &a, const unsigned char *ws, int n_slots,
+                                   kda_dtype_t out_dtype, cudaStream_t stream, const NormArgs *norm,
+                                   long long slot_lo, long long slot_hi);
+
+// The bf16 prefill as kda_chunk_fwd runs it (prefill.cu): with at most kPipeMaxChains (sequence,
+// head) chains and enough chunk slots, a pipeline over token ranges (scan of one range beside the
+// preparation of the next ones), else the two passes one after the other. The pipeline carries the
+// state between ranges in S_final, or in prefill_carry_bytes of workspace after the blocks.
+constexpr int kPipeMaxChains = 64;
+constexpr int kPipeMinSlotsPerRange = 16;
+bool prefill_pipelined(long long tokens, int H, int N);
+size_t prefill_carry_bytes(long long tokens, int H, int N);
+int prefill_launches(long long tokens, int H, int N);   // kernels run_prefill_bf16 launches
+cudaError_t run_prefill_bf16(const PrefillArgs &a, kda_dtype_t out_dtype, cudaStream_t stream,
+                             const GateArgs *gate, const NormArgs *norm);
 
 // Backward pass (chunk_bwd.cu). Gradient pointers and the records of the forward kernel.
 struct BwdArgs {

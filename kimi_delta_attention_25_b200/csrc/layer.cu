@@ -199,11 +199,7 @@ kda_status_t kda_chunk_fwd_layer(const void *q, const void *k, const void *v,
                                  workspace_bytes);
     cudaError_t e = cudaSuccess;
     if (dtype == KDA_BF16) {
-        const int n_slots = (int)prep_slots(tokens, N);
-        e = launch_chunk_prep(a, (unsigned char *)a.scratch, n_slots, st, use_gate ? &gate : nullptr);
-        if (e == cudaSuccess)
-            e = launch_chunk_scan(a, (const unsigned char *)a.scratch, n_slots, out_dtype, st,
-                                  use_norm ? &norm : nullptr);
+        e = run_prefill_bf16(a, out_dtype, st, use_gate ? &gate : nullptr, use_norm ? &norm : nullptr);
         return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
     }
     // fp32 inputs: gates -> fp32 scratch, CUDA-core prefill, norm of its fp32 outputs
