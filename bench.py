@@ -491,7 +491,8 @@ LAYER_BYTES_PER_TOKEN_HEAD = 4 * D * 2 + D * 2 + 2 + D * 2
 def run_layer_step(kda, dev, pk, ws, rank, args, d):
     """The same 128K x 32 prefill as a full KDA layer step: gates produced inside the preparation
     pass from f, A_log, dt_bias and the beta logits, and the gated RMSNorm applied in the scan's
-    output epilogue (4-CTA clusters); bf16 outputs. Timed per pass like the headline step."""
+    output epilogue; bf16 outputs. Timed like the headline step (the public call, and each pass
+    alone)."""
     B, T, H = d["v"].shape[:3]
     lay = K.make_layer_inputs(B, T, H, dtype="bf16", device=dev, seed=5)
     opts = dict(lay, norm_eps=1e-5)
@@ -644,31 +645,34 @@ def run_backward(kda, dev, pk, ws, local, args, d):
 
 
 def run_profile_case(args):
-    """One small invocation for Nsight Compute captures: `prefill` runs kda_chunk_fwd on the
-    first `--tokens` tokens of the 32-head bf16 workload (inputs > L2, a few GB at most) twice;
+    """One small invocation for Nsight Compute captures: `step` runs the headline step (the public
+    call kda_chunk_fwd, full size) `--steps` times; `prefill` runs the two passes kda_chunk_prep and
+    kda_chunk_scan, one full launch each, on the first `--tokens` tokens of the 32-head bf16 workload
+    (inputs > L2, a few GB at most) twice;
     `backward` runs kda_chunk_bwd twice on the same tokens; `decode` runs 8 decode steps of the
     256 x 32 decode workload."""
     import kimi_delta_attention_25_b200 as kda
     kda.load()
     dev = torch.device("cuda", 0)
     if args.profile == "step":
-        # the headline step as timed (two passes, bf16 outputs), full size, `--steps` times
+        # the headline step as timed (the public call, bf16 outputs), full size, `--steps` times
         w = K.WORKLOADS[WORKLOAD]
         d = K.make_prefill(w, device=dev)
         out = torch.empty(w.B, w.T, w.H, D, dtype=torch.bfloat16, device=dev)
         Sf = torch.empty(w.B, w.H, D, D, dtype=torch.float32, device=dev)
         ws = torch.empty(kda.chunk_fwd_workspace_size(w.B, w.T, w.H, w.B), dtype=torch.uint8, device=dev)
         for _ in range(args.steps):
-            kda.chunk_prep(d["q"], d["k"], d["log_alpha"], d["beta"], ws)
-            kda.chunk_scan(d["v"], ws, S0=d["S0"], out=out, S_final=Sf)
+            kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"], out=out, S_final=Sf,
+                          workspace=ws)
         torch.cuda.synchronize()
         assert kda.workspace_status(ws) == kda.KDA_OK
     elif args.profile == "prefill":
         w = K.WORKLOADS[WORKLOAD]
         d = K.make_prefill(w, device=dev, T=args.tokens)
+        ws = torch.empty(kda.chunk_fwd_workspace_size(w.B, args.tokens, w.H, w.B), dtype=torch.uint8, device=dev)
         for _ in range(2):
-            ws = kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"],
-                               out_dtype=torch.bfloat16, return_workspace=True)[2]
+            kda.chunk_prep(d["q"], d["k"], d["log_alpha"], d["beta"], ws)
+            kda.chunk_scan(d["v"], ws, S0=d["S0"], out_dtype=torch.bfloat16)
         torch.cuda.synchronize()
         assert kda.workspace_status(ws) == kda.KDA_OK
     elif args.profile == "backward":

@@ -112,7 +112,7 @@ int kda_chunk_fwd_kernel_launches(int B, int T, int H, int N, kda_dtype_t dtype)
  *              workspace_bytes its size. Its status word is cleared by this call.
  * S0 and S_final may alias (in-place continuation); no other buffers may overlap.
  * T = 0 or N = 0 is valid (only S_final = S0 is written).
- * For bf16 inputs with at most 64 (sequence, head) pairs and at least 32 chunk slots the two
+ * For bf16 inputs with at most 64 (sequence, head) pairs and at least 64 chunk slots the two
  * passes run as a pipeline over up to 16 token ranges: the state scan of one range beside the
  * preparation of the later ones, on two library-owned streams (created on the first such call per
  * device) that fork from `stream` and join it again; everything stays ordered on `stream`. Between
@@ -263,8 +263,7 @@ size_t kda_chunk_fwd_layer_workspace_size(int B, int T, int H, int N, int dk, in
  * log_alpha / beta may be NULL when their producer inputs are given. For bf16 inputs every part
  * is fused: the decay and write gates are produced inside the preparation pass (the fp32
  * log_alpha stream is never written or read), and the output norm runs in the scan's output
- * epilogue, with the four 32-channel CTAs of a head exchanging per-token sums of squares through
- * distributed shared memory (a 4-CTA cluster). fp32 inputs run separate gate and norm passes
+ * epilogue (one CTA holds all value channels of a head). fp32 inputs run separate gate and norm passes
  * around the CUDA-core prefill. Errors as for kda_chunk_fwd; a NULL A_log/dt_bias with gate_f, or
  * a NULL norm_weight with out_gate, or norm_eps < 0 is KDA_ERR_INVALID_ARG. */
 kda_status_t kda_chunk_fwd_layer(const void *q, const void *k, const void *v,

@@ -18,7 +18,7 @@
 // block with one bulk copy:
 //   [0, 32K)    X: W (rows 0-63) and Qt - M W (rows 64-127), two 64-channel halves, K-major
 //   [32K, 48K)  Y: -Tb (rows 0-63) and M Tb (rows 64-127), 64 token columns, K-major
-//   [48K, 64K)  Kend, two halves of 64 tokens x 64 channels (the MN-major A of Kend^T U)
+//   [48K, 64K)  Kend, two halves of 64 tokens x 64 channels (the MN-major B of U^T Kend)
 //   [64K, +512) gamma (fp32)
 // A chunk slot is floor(first_token / 64) + sequence, which is unique per (sequence, chunk) and
 // below floor(total_tokens / 64) + N + 1.

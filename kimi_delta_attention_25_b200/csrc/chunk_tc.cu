@@ -17,7 +17,7 @@
 // f and b are running products of alpha = exp(log_alpha) (forward and backward within the chunk).
 //
 // This single-kernel form needs no workspace beyond the status word, so kda_chunk_fwd_noalloc runs
-// it; kda_chunk_fwd runs the faster two-pass form (chunk_prep.cu, chunk_scan.cu).
+// it; kda_chunk_fwd runs the faster two-pass form (chunk_prep.cu, chunk_scan.cu, prefill.cu).
 //
 // Work split: one CTA per (sequence, head, 32-column block of d_v). The value columns of S evolve
 // independently, so the four blocks of a head never communicate; each recomputes the

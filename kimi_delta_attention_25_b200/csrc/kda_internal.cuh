@@ -24,7 +24,7 @@ constexpr int kMaxGridDim = 65535;    // heads and sequences index grid dimensio
 // are contiguous in the same order in the scan's ring stage, so one bulk copy moves a block.
 constexpr uint32_t kPrepXOff = 0;           // X = [W; Qt - M W], 128 x 128 f16, 32 KiB
 constexpr uint32_t kPrepYOff = 32768;       // Y = [-Tb; M Tb], 128 x 64 f16, 16 KiB
-constexpr uint32_t kPrepKEOff = 49152;      // Kend, 16 KiB
+constexpr uint32_t kPrepKEOff = 49152;      // Kend, 64 x 128 f16 (two 64-channel halves), 16 KiB
 constexpr uint32_t kPrepGammaOff = 65536;   // gamma, 512 B
 constexpr size_t kPrepBlockBytes = 66048;
 
@@ -179,21 +179,19 @@ bool token_rows_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, ui
 // (slots [slot_lo, slot_hi) only; slot_hi < 0: to the end)
 cudaError_t launch_chunk_prep(const PrefillArgs &a, unsigned char *ws, int n_slots, cudaStream_t stream,
                               const GateArgs *gate = nullptr, int slot_lo = 0, int slot_hi = -1);
-cudaError_t launch_chunk_scan(const PrefillArgs &a, const unsigned char *ws, int n_slots,
-                              kda_dtype_t out_dtype, cudaStream_t stream, const NormArgs *norm = nullptr);
-// The same pass with one CTA per (sequence, head) over all value columns (chunk_scan_wide.cu), for the
-// chunks whose slots lie in [slot_lo, slot_hi); a range that does not start a sequence starts from
+// The state scan (chunk_scan.cu), one CTA per (sequence, head), over the chunks whose slots lie in
+// [slot_lo, slot_hi) (slot_hi < 0: to the end); a range that does not start a sequence starts from
 // S_final, which must then be given.
-cudaError_t launch_chunk_scan_wide(const PrefillArgs &a, const unsigned char *ws, int n_slots,
-                                   kda_dtype_t out_dtype, cudaStream_t stream, const NormArgs *norm,
-                                   long long slot_lo, long long slot_hi);
+cudaError_t launch_chunk_scan(const PrefillArgs &a, const unsigned char *ws, int n_slots,
+                              kda_dtype_t out_dtype, cudaStream_t stream, const NormArgs *norm = nullptr,
+                              long long slot_lo = 0, long long slot_hi = -1);
 
 // The bf16 prefill as kda_chunk_fwd runs it (prefill.cu): with at most kPipeMaxChains (sequence,
 // head) chains and enough chunk slots, a pipeline over token ranges (scan of one range beside the
 // preparation of the next ones), else the two passes one after the other. The pipeline carries the
 // state between ranges in S_final, or in prefill_carry_bytes of workspace after the blocks.
 constexpr int kPipeMaxChains = 64;
-constexpr int kPipeMinSlotsPerRange = 16;
+constexpr int kPipeMinSlotsPerRange = 32;
 bool prefill_pipelined(long long tokens, int H, int N);
 size_t prefill_carry_bytes(long long tokens, int H, int N);
 int prefill_launches(long long tokens, int H, int N);   // kernels run_prefill_bf16 launches

@@ -7,8 +7,8 @@
 //   y = o / sqrt(mean_c o_c^2 + eps) * w * sigmoid(g)   over the d_v channels of one head.
 //
 // For bf16 inputs they are fused into the prefill's two passes (chunk_prep.cu forms log_alpha and
-// beta from their inputs as it loads them; chunk_scan.cu normalises in its output epilogue across a
-// 4-CTA cluster) and into the decode kernel. This file holds the entry points and, for fp32 inputs,
+// beta from their inputs as it loads them; chunk_scan.cu normalises in its output epilogue, the
+// four warps of a token group adding their sums of squares) and into the decode kernel. This file holds the entry points and, for fp32 inputs,
 // two stand-alone passes around the CUDA-core prefill: the gates into fp32 scratch, and the norm of
 // the fp32 outputs.
 #include <cuda_runtime.h>

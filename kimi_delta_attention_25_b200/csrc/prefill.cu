@@ -1,7 +1,7 @@
 // prefill.cu -- how kda_chunk_fwd (and its layer variant) runs the two passes of the bf16 prefill.
 //
 // The preparation pass (chunk_prep.cu) is data-parallel over every (chunk, head); the scan
-// (chunk_scan_wide.cu) is one serial chain of chunks per (sequence, head) and holds one SM per chain.
+// (chunk_scan.cu) is one serial chain of chunks per (sequence, head) and holds one SM per chain.
 // With few chains (one long sequence: 32 heads hold 32 of the 148 SMs for the whole scan) the two
 // passes run as a pipeline over token ranges: the scan of range r runs while the preparation of the
 // later ranges fills the other SMs. Each range's scan waits for its own preparation only; a range
@@ -82,7 +82,7 @@ cudaError_t run_prefill_bf16(const PrefillArgs &a_in, kda_dtype_t out_dtype, cud
     unsigned char *blocks = (unsigned char *)a_in.scratch;
     if (!prefill_pipelined(tokens, a_in.H, a_in.N)) {
         cudaError_t e = launch_chunk_prep(a_in, blocks, n_slots, st, gate);
-        if (e == cudaSuccess) e = launch_chunk_scan_wide(a_in, blocks, n_slots, out_dtype, st, norm, 0, n_slots);
+        if (e == cudaSuccess) e = launch_chunk_scan(a_in, blocks, n_slots, out_dtype, st, norm, 0, n_slots);
         return e;
     }
     PrefillArgs a = a_in;
@@ -110,7 +110,7 @@ cudaError_t run_prefill_bf16(const PrefillArgs &a_in, kda_dtype_t out_dtype, cud
     for (int r = 0; r < R && e == cudaSuccess; ++r) {
         e = cudaStreamWaitEvent(ps->scan, ps->prepped[r], 0);
         if (e == cudaSuccess)
-            e = launch_chunk_scan_wide(a, blocks, n_slots, out_dtype, ps->scan, norm, bounds[r], bounds[r + 1]);
+            e = launch_chunk_scan(a, blocks, n_slots, out_dtype, ps->scan, norm, bounds[r], bounds[r + 1]);
     }
     // join: the caller's stream waits for both library streams (on an error too, so that nothing the
     // call enqueued can still run unordered with the caller's later work)
