@@ -27,7 +27,8 @@
 //                update (rows past the chunk's end zeroed): one warp converting a chunk's 16 KB
 //                alone set the chunk period.
 // Per chunk the epilogue warps run U (on the chain), the outputs (beside D7), the state update (on
-// the chain), then the v conversion (beside the next chunk's S1).
+// the chain), then the v conversion (beside the next chunk's S1). With the output norm only the sums
+// of squares run beside D7; the normalised outputs follow the state update.
 //   warp 17      MMA issuer (lane 0).
 //   warp 18      output store (lane 0): a full chunk's bf16 outputs are staged as a [token][value]
 //                tile and leave by two tensor stores; with the output norm it also brings each
@@ -432,6 +433,44 @@ chunk_scan_kernel(WideParams p, const __grid_constant__ CUtensorMap tm_v,
             if (lane == 0) mbar_arrive(&bars[B_VCONV + vs]);
             return true;
         };
+        // one warp's outputs of a chunk: 16 tokens x 32 value columns, to the staging tile (bf16, full
+        // chunk) or straight to global memory
+        auto emit = [&](const float (&o)[16], unsigned char *ost, int64_t tok0, int L) {
+            if (STAGED && L == C) {
+                // pairs of neighbouring value columns: the even lane keeps tokens tk0 + i, the odd
+                // lane tokens tk0 + 8 + (i + 4) % 8 (rows four apart mod 8, so the two row pieces
+                // of one store land in different banks)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int ie = i, io = 8 + ((i + 4) & 7);
+                    const float send = odd ? o[ie] : o[io];
+                    const float got = __shfl_xor_sync(0xffffffffu, send, 1);
+                    const int t = tk0 + (odd ? io : ie);
+                    const uint32_t v2 = odd ? pack_bf16x2(got, o[io]) : pack_bf16x2(o[ie], got);
+                    *reinterpret_cast<uint32_t *>(ost + tile_off(t, j & ~1)) = v2;
+                }
+                fence_proxy_async_smem();
+            } else if constexpr (sizeof(TO) == 4) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const long long oi = ((long long)(tok0 + tk0 + i) * H + h) * DK + j;
+                    if (tk0 + i < L && in_bounds(p.status, oi, 1, p.tokens * H * DK))
+                        reinterpret_cast<float *>(p.out)[oi] = o[i];
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int ie = i, io = 8 + i;
+                    const float send = odd ? o[ie] : o[io];
+                    const float got = __shfl_xor_sync(0xffffffffu, send, 1);
+                    const int t = tk0 + (odd ? io : ie);
+                    const uint32_t v2 = odd ? pack_bf16x2(got, o[io]) : pack_bf16x2(o[ie], got);
+                    const long long oi = ((long long)(tok0 + t) * H + h) * DK + (j & ~1);
+                    if (t < L && in_bounds(p.status, oi, 2, p.tokens * H * DK))
+                        *reinterpret_cast<uint32_t *>(reinterpret_cast<uint16_t *>(p.out) + oi) = v2;
+                }
+            }
+        };
         store_state();
         tc_fence_before();
         __syncwarp();
@@ -463,106 +502,58 @@ chunk_scan_kernel(WideParams p, const __grid_constant__ CUtensorMap tm_v,
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_UREADY]);
             // outputs O^T[j][tk0 + i] = O[tk0 + i][j]
-            bool good = true;
-            {
+            if constexpr (!NORM) {
                 float o[16];
                 tmem_ld16_sync(d5 + 64 + tk0, o);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_D5FREE + d]);
-                if constexpr (NORM) {
-                    // sum over the 32 value rows of this warp, 16 tokens: reduce-scatter by lane bits
-                    // 4, 3, 2, 1, then lane bit 0; lane 2 i ends with token i
-                    float r[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) r[i] = o[i] * o[i];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {         // keep tokens 8 bit4 + i
-                        const bool hi = (lane & 16) != 0;
-                        const float send = hi ? r[i] : r[i + 8];
-                        const float keep = hi ? r[i + 8] : r[i];
-                        r[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {         // keep 8 bit4 + 4 bit3 + i
-                        const bool hi = (lane & 8) != 0;
-                        const float send = hi ? r[i] : r[i + 4];
-                        const float keep = hi ? r[i + 4] : r[i];
-                        r[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        const bool hi = (lane & 4) != 0;
-                        const float send = hi ? r[i] : r[i + 2];
-                        const float keep = hi ? r[i + 2] : r[i];
-                        r[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-                    }
-                    {
-                        const bool hi = (lane & 2) != 0;
-                        const float send = hi ? r[0] : r[1];
-                        const float keep = hi ? r[1] : r[0];
-                        r[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-                    }
-                    r[0] += __shfl_xor_sync(0xffffffffu, r[0], 1);
-                    // the four warps of this token group (q = 0..3) add their sums
-                    float *red = reinterpret_cast<float *>(sm + OFF_RED) + (d * 4 + b) * 64;
-                    if (!odd) red[q * 16 + (lane >> 1)] = r[0];
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars[B_RED + d * 4 + b]);
-                    good = warp_wait(&bars[B_RED + d * 4 + b], (k >> 1) & 1);
-                    const int ti = lane >> 1;
-                    const float ss = red[ti] + red[16 + ti] + red[32 + ti] + red[48 + ti];
-                    const float rinv_mine = rsqrtf(ss * (1.f / DK) + p.eps);
-                    good = good && warp_wait(&bars[B_GATE + d], (k >> 1) & 1);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float ri = __shfl_sync(0xffffffffu, rinv_mine, 2 * i);
-                        const float gv = good ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
-                                                    ost + tile_off(tk0 + i, j)))
-                                              : 0.f;
-                        o[i] = o[i] * ri * wj * sigmoid_fast(gv);
-                    }
-                    __syncwarp();                     // every gate value read before the tile is rewritten
-                } else {
-                    if (STAGED && k >= 2) good = warp_wait(&bars[B_OFREE + d], ((k >> 1) - 1) & 1);
-                }
-                if (!good) { fail(); break; }
-                if (STAGED && L == C) {
-                    // pairs of neighbouring value columns: the even lane keeps tokens tk0 + i, the odd
-                    // lane tokens tk0 + 8 + (i + 4) % 8 (rows four apart mod 8, so the two row pieces
-                    // of one store land in different banks)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int ie = i, io = 8 + ((i + 4) & 7);
-                        const float send = odd ? o[ie] : o[io];
-                        const float got = __shfl_xor_sync(0xffffffffu, send, 1);
-                        const int t = tk0 + (odd ? io : ie);
-                        const uint32_t v2 = odd ? pack_bf16x2(got, o[io]) : pack_bf16x2(o[ie], got);
-                        *reinterpret_cast<uint32_t *>(ost + tile_off(t, j & ~1)) = v2;
-                    }
-                    fence_proxy_async_smem();
-                } else if constexpr (sizeof(TO) == 4) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const long long oi = ((long long)(tok0 + tk0 + i) * H + h) * DK + j;
-                        if (tk0 + i < L && in_bounds(p.status, oi, 1, p.tokens * H * DK))
-                            reinterpret_cast<float *>(p.out)[oi] = o[i];
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int ie = i, io = 8 + i;
-                        const float send = odd ? o[ie] : o[io];
-                        const float got = __shfl_xor_sync(0xffffffffu, send, 1);
-                        const int t = tk0 + (odd ? io : ie);
-                        const uint32_t v2 = odd ? pack_bf16x2(got, o[io]) : pack_bf16x2(o[ie], got);
-                        const long long oi = ((long long)(tok0 + t) * H + h) * DK + (j & ~1);
-                        if (t < L && in_bounds(p.status, oi, 2, p.tokens * H * DK))
-                            *reinterpret_cast<uint32_t *>(reinterpret_cast<uint16_t *>(p.out) + oi) = v2;
-                    }
-                }
+                if (STAGED && k >= 2 && !warp_wait(&bars[B_OFREE + d], ((k >> 1) - 1) & 1)) { fail(); break; }
+                emit(o, ost, tok0, L);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_OST + d]);
+            } else {
+                // the norm's sum of squares now (while D7 runs); the rest after the state update
+                float o[16];
+                tmem_ld16_sync(d5 + 64 + tk0, o);
+                // sum over the 32 value rows of this warp, 16 tokens: reduce-scatter by lane bits
+                // 4, 3, 2, 1, then lane bit 0; lane 2 i ends with token i
+                float r[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) r[i] = o[i] * o[i];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {         // keep tokens 8 bit4 + i
+                    const bool hi = (lane & 16) != 0;
+                    const float send = hi ? r[i] : r[i + 8];
+                    const float keep = hi ? r[i + 8] : r[i];
+                    r[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {         // keep 8 bit4 + 4 bit3 + i
+                    const bool hi = (lane & 8) != 0;
+                    const float send = hi ? r[i] : r[i + 4];
+                    const float keep = hi ? r[i + 4] : r[i];
+                    r[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+                }
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const bool hi = (lane & 4) != 0;
+                    const float send = hi ? r[i] : r[i + 2];
+                    const float keep = hi ? r[i + 2] : r[i];
+                    r[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+                }
+                {
+                    const bool hi = (lane & 2) != 0;
+                    const float send = hi ? r[0] : r[1];
+                    const float keep = hi ? r[1] : r[0];
+                    r[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                }
+                r[0] += __shfl_xor_sync(0xffffffffu, r[0], 1);
+                // the four warps of this token group (q = 0..3) add their sums after the state update
+                float *red = reinterpret_cast<float *>(sm + OFF_RED) + (d * 4 + b) * 64;
+                if (!odd) red[q * 16 + (lane >> 1)] = r[0];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_RED + d * 4 + b]);
             }
             // S^T <- S^T Diag(gamma) + D7^T, then hand the new state to the next chunk's S1
             if (!warp_wait(&bars[B_KFULL + r], (k / NR) & 1)) { fail(); break; }
@@ -585,6 +576,32 @@ chunk_scan_kernel(WideParams p, const __grid_constant__ CUtensorMap tm_v,
             tc_fence_before();
             __syncwarp();
             if (lane == 0) { mbar_arrive(&bars[B_SREADY]); mbar_arrive(&bars[B_KEMPTY + r]); }
+            if constexpr (NORM) {
+                // normalised, gated outputs of chunk k (its D5 half stays untouched until the seed of
+                // chunk k + 2, which waits for the arrival below)
+                const float *red = reinterpret_cast<const float *>(sm + OFF_RED) + (d * 4 + b) * 64;
+                bool good = warp_wait(&bars[B_RED + d * 4 + b], (k >> 1) & 1);
+                const int ti = lane >> 1;
+                const float ss = red[ti] + red[16 + ti] + red[32 + ti] + red[48 + ti];
+                const float rinv_mine = rsqrtf(ss * (1.f / DK) + p.eps);
+                good = good && warp_wait(&bars[B_GATE + d], (k >> 1) & 1);
+                if (!good) { fail(); break; }
+                float o[16];
+                tmem_ld16_sync(d5 + 64 + tk0, o);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_D5FREE + d]);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float ri = __shfl_sync(0xffffffffu, rinv_mine, 2 * i);
+                    const float gv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(ost + tile_off(tk0 + i, j)));
+                    o[i] = o[i] * ri * wj * sigmoid_fast(gv);
+                }
+                __syncwarp();                         // every gate value read before the tile is rewritten
+                emit(o, ost, tok0, L);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_OST + d]);
+            }
             // v of chunk k + 2 while the tensor cores run S1 of chunk k + 1
             if (k + 2 < nk && !convert_v(k + 2)) { fail(); break; }
         }
