@@ -95,10 +95,12 @@ cudaError_t run_prefill_bf16(const PrefillArgs &a_in, kda_dtype_t out_dtype, cud
     cudaError_t e = cudaEventRecord(ps->fork, st);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ps->prep, ps->fork, 0);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ps->scan, ps->fork, 0);
-    // ranges of slots, the first one half as long (it runs without a scan beside it)
+    // ranges of slots: the first half as long (its preparation runs with no scan beside it) and, with
+    // eight ranges or more, the last a quarter as long (its scan runs after every preparation has
+    // finished; with fewer ranges a quarter range is too short to pay for its launch)
     int bounds[kMaxRanges + 1];
     {
-        const double unit = (double)n_slots / (R - 0.5);
+        const double unit = (double)n_slots / (R >= 8 ? R - 1.25 : R - 0.5);
         bounds[0] = 0;
         for (int r = 1; r < R; ++r) bounds[r] = (int)((r - 0.5) * unit);
         bounds[R] = n_slots;

@@ -212,3 +212,26 @@ def test_chunked_calls_refuse_more_heads_or_sequences_than_a_grid_dimension(lib)
         kda.KDA_ERR_UNSUPPORTED
     # the limit itself is accepted by the host checks (this call then stops at its workspace)
     assert _chunk(lib, H=65535) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_chunk_fwd_kernel_launches(lib):
+    """The launch count of the prefill: a pipeline over token ranges (two kernels per range) with at
+    most 64 (sequence, head) chains and at least 64 chunk slots, else the two passes once; one
+    kernel for fp32 inputs."""
+    bf, f32 = 1, 0
+    assert lib.kda_chunk_fwd_kernel_launches(1, 131072, 32, 1, bf) == 32     # 16 ranges
+    assert lib.kda_chunk_fwd_kernel_launches(1, 8192, 16, 1, bf) == 8        # 4 ranges
+    assert lib.kda_chunk_fwd_kernel_launches(1, 262144, 32, 8, bf) == 2      # 256 chains
+    assert lib.kda_chunk_fwd_kernel_launches(1, 2048, 4, 1, bf) == 2         # 34 slots
+    assert lib.kda_chunk_fwd_kernel_launches(1, 100, 2, 1, f32) == 1
+    assert lib.kda_chunk_fwd_kernel_launches(1, 100, 2, 0, bf) == 0
+    assert lib.kda_chunk_fwd_kernel_launches(-1, 100, 2, 1, bf) == 0
+
+
+def test_workspace_holds_the_pipeline_carry(lib):
+    """A pipelined prefill carries the state between token ranges; without S_final it lives in the
+    workspace, after the prepared blocks."""
+    blocks = 256 + 32 * (131072 // 64 + 2) * 66048
+    assert lib.kda_chunk_fwd_workspace_size(1, 131072, 32, 1, 128, 128, 1) == blocks + 32 * 128 * 128 * 4
+    blocks = 256 + 32 * (262144 // 64 + 9) * 66048
+    assert lib.kda_chunk_fwd_workspace_size(1, 262144, 32, 8, 128, 128, 1) == blocks
