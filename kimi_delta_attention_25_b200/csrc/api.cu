@@ -222,18 +222,30 @@ kda_status_t chunk_bwd_impl(unsigned phases, const void *q, const void *k, const
     float *ck_Y = ck_U + hs * kBwdRowsFloats;
 
     cudaError_t e = cudaSuccess;
+    // bf16 inputs take the forward records from the tensor-core passes, which write S and U but not
+    // R (the per-chunk kernel forms it); their prepared blocks sit in the dS' and R areas, which
+    // the reverse scan rewrites and nothing reads until then
+    const bool tc = dtype == KDA_BF16;
     if (phases & 1u) {              // 1. forward sweep with records (outputs not needed)
         PrefillArgs a = prefill_args(q, k, v, log_alpha, beta, S0, cu_seqlens, nullptr, nullptr, B, T, H, N,
                                      workspace, workspace_bytes);
-        a.ck_S = ck_S; a.ck_R = ck_R; a.ck_U = ck_U; a.n_slots = (int)n_slots;
-        e = launch_chunk_fp32(a, dtype, KDA_F32, st);
+        a.ck_S = ck_S; a.ck_U = ck_U; a.n_slots = (int)n_slots;
+        if (tc) {
+            static_assert(kPrepBlockBytes <= (kBwdStateFloats + kBwdRowsFloats) * sizeof(float),
+                          "prepared blocks fit the dS' and R areas");
+            e = launch_chunk_prep(a, (unsigned char *)ck_dS, (int)n_slots, st);
+            if (e == cudaSuccess) e = launch_chunk_scan_records(a, (const unsigned char *)ck_dS, (int)n_slots, st);
+        } else {
+            a.ck_R = ck_R;
+            e = launch_chunk_fp32(a, dtype, KDA_F32, st);
+        }
     }
     BwdArgs b;
     b.q = q; b.k = k; b.v = v; b.dout = dout;
     b.log_alpha = log_alpha; b.beta = beta; b.dS_final = dS_final;
     b.cu_seqlens = cu_seqlens;
     b.dq = dq; b.dk = dk_out; b.dv = dv_out; b.dlog_alpha = dlog_alpha; b.dbeta = dbeta; b.dS0 = dS0;
-    b.ck_S = ck_S; b.ck_R = ck_R; b.ck_U = ck_U; b.ck_dS = ck_dS; b.ck_Y = ck_Y;
+    b.ck_S = ck_S; b.ck_R = tc ? nullptr : ck_R; b.ck_U = ck_U; b.ck_dS = ck_dS; b.ck_Y = ck_Y;
     b.B = B; b.T = T; b.H = H; b.N = N; b.n_slots = (int)n_slots;
     b.status = (int32_t *)workspace;
     if (e == cudaSuccess && (phases & 2u)) e = launch_chunk_bwd_scan(b, dtype, st);   // 2. reverse scan

@@ -20,8 +20,10 @@
 //   dlog_alpha = reverse cumulative sum of dg over the chunk's rows.
 //
 // Three launches (the host calls them in order on one stream):
-//  1. the fp32 forward kernel (chunk_fp32.cu) with records on: the state entering every chunk and
-//     each chunk's R and U, per (head, chunk slot);
+//  1. the forward records: the state entering every chunk and each chunk's R and U, per (head,
+//     chunk slot). For fp32 inputs the fp32 forward kernel (chunk_fp32.cu) writes all three; for
+//     bf16 inputs the tensor-core passes do (chunk_prep.cu, then chunk_scan.cu in record mode),
+//     writing S and U, and kernel 3 forms R = V - Kt S itself;
 //  2. chunk_bwd_scan_kernel: the state gradient, chunk by chunk from the end of each sequence
 //     (one CTA per (sequence, head, 32 value columns); the columns are independent). It writes dV,
 //     dS0, Y and the gradient dS' reaching the end of every chunk;
@@ -227,7 +229,10 @@ struct LocalSmem {
 };
 static_assert((NT_LOC / 32) * DK <= C * LDV, "per-warp column sums must fit the dO block");
 
-template <typename T>
+// COMPUTE_R: no R record (the forward records came from the bf16 state scan, which holds S and U
+// but not R). R enters only dbeta, through sum_v R_rv Y_rv = sum_v V_rv Y_rv - sum_c Kt_rc (Y S^T)_rc;
+// the value block of V takes R's place and Y S^T is the product this kernel forms for dKt anyway.
+template <typename T, bool COMPUTE_R>
 __global__ void __launch_bounds__(NT_LOC, 1)
 chunk_bwd_local_kernel(BwdArgs a)
 {
@@ -310,14 +315,14 @@ chunk_bwd_local_kernel(BwdArgs a)
     const float *gdS = a.ck_dS + rec * kBwdStateFloats;
     const float *gU = a.ck_U + rec * kBwdRowsFloats;
     const float *gY = a.ck_Y + rec * kBwdRowsFloats;
-    const float *gR = a.ck_R + rec * kBwdRowsFloats;
+    const float *gR = COMPUTE_R ? nullptr : a.ck_R + rec * kBwdRowsFloats;
     float dgam_acc = 0.f, ry_acc = 0.f;
     for (int j0 = 0; j0 < DK; j0 += DVB) {
         __syncthreads();
         {
             // 16-byte loads, all in flight before the first store: the state blocks (128 rows of
             // 8 float4, two per thread) and the row blocks (64 rows of 8 float4, one per thread)
-            float4 xs[2], xd[2], xu, xy, xr;
+            float4 xs[2], xd[2], xu, xy, xr = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
                 const int idx = tid + it * NT_LOC, c = idx >> 3, q4 = idx & 7;
@@ -327,8 +332,9 @@ chunk_bwd_local_kernel(BwdArgs a)
             const int r = tid >> 3, q4 = tid & 7;
             xu = __ldg(reinterpret_cast<const float4 *>(gU + (size_t)r * DK + j0) + q4);
             xy = __ldg(reinterpret_cast<const float4 *>(gY + (size_t)r * DK + j0) + q4);
-            xr = __ldg(reinterpret_cast<const float4 *>(gR + (size_t)r * DK + j0) + q4);
+            if constexpr (!COMPUTE_R) xr = __ldg(reinterpret_cast<const float4 *>(gR + (size_t)r * DK + j0) + q4);
             fp32c::load_rows<T, NT_LOC, DVB>(sm.dO, LDV, dout, s, L, H, h, j0, tid);
+            if constexpr (COMPUTE_R) fp32c::load_rows<T, NT_LOC, DVB>(sm.R, LDV, (const T *)a.v, s, L, H, h, j0, tid);
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
                 const int idx = tid + it * NT_LOC, c = idx >> 3, v = (idx & 7) * 4;
@@ -340,7 +346,7 @@ chunk_bwd_local_kernel(BwdArgs a)
             float *du = sm.U + r * LDV + v, *dy = sm.Y + r * LDV + v, *dr = sm.R + r * LDV + v;
             du[0] = xu.x; du[1] = xu.y; du[2] = xu.z; du[3] = xu.w;
             dy[0] = xy.x; dy[1] = xy.y; dy[2] = xy.z; dy[3] = xy.w;
-            dr[0] = xr.x; dr[1] = xr.y; dr[2] = xr.z; dr[3] = xr.w;
+            if constexpr (!COMPUTE_R) { dr[0] = xr.x; dr[1] = xr.y; dr[2] = xr.z; dr[3] = xr.w; }
         }
         __syncthreads();
 #pragma unroll 4
@@ -397,6 +403,10 @@ chunk_bwd_local_kernel(BwdArgs a)
                 dM[r * LDC + i] = (i <= r) ? aM[x][z] : 0.f;
                 dP[r * LDC + i] = sm.beta[r] * da;
                 part[x] += da * sm.P[r * LDC + i];
+            }
+            if constexpr (COMPUTE_R) {        // - sum_c Kt_rc (Y S^T)_rc over this thread's 4 columns
+#pragma unroll
+                for (int z = 0; z < 4; ++z) part[x] -= sm.Kt[r * LD + cb + 32 * z] * aY[x][z];
             }
         }
 #pragma unroll
@@ -500,16 +510,22 @@ cudaError_t launch_scan_typed(const BwdArgs &a, cudaStream_t stream)
     return cudaGetLastError();
 }
 
+template <typename T, bool COMPUTE_R>
+cudaError_t launch_local_variant(const BwdArgs &a, cudaStream_t stream)
+{
+    const size_t smem = sizeof(LocalSmem);
+    cudaError_t e = cudaFuncSetAttribute(chunk_bwd_local_kernel<T, COMPUTE_R>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const long long blocks = (long long)a.n_slots * a.H;
+    chunk_bwd_local_kernel<T, COMPUTE_R><<<(unsigned)blocks, NT_LOC, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t launch_local_typed(const BwdArgs &a, cudaStream_t stream)
 {
-    const size_t smem = sizeof(LocalSmem);
-    cudaError_t e = cudaFuncSetAttribute(chunk_bwd_local_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    const long long blocks = (long long)a.n_slots * a.H;
-    chunk_bwd_local_kernel<T><<<(unsigned)blocks, NT_LOC, smem, stream>>>(a);
-    return cudaGetLastError();
+    return a.ck_R ? launch_local_variant<T, false>(a, stream) : launch_local_variant<T, true>(a, stream);
 }
 
 }  // namespace

@@ -41,6 +41,10 @@
 // sums the squares of its 16 tokens over its 32 value rows with a 16-shuffle reduce-scatter; the four
 // warps of a token group then add their sums through shared memory behind a four-arrival mbarrier.
 //
+// Backward records (REC): instead of outputs, the scan writes what the backward pass needs of the
+// forward one (chunk_bwd.cu): the fp32 state entering every chunk and the chunk's U, per (head, chunk
+// slot), in the layout the CUDA-core forward writes them.
+//
 // Token ranges: a launch may cover only the chunks whose slots lie in [slot_lo, slot_hi). A chunk
 // range that does not start a sequence starts from S_final (the state the previous range left
 // there); every launch leaves its state in S_final.
@@ -126,6 +130,7 @@ struct WideParams {
     int32_t *status;
     const float *norm_w;
     float eps;
+    float *ck_S, *ck_U;             // backward records (REC)
 };
 
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
@@ -147,12 +152,12 @@ __device__ __forceinline__ uint32_t tile_off(int t, int j) {
            ((uint32_t)((((j & 63) >> 3) ^ (t & 7)) & 7) << 4) + (uint32_t)(j & 7) * 2u;
 }
 
-template <typename TO, bool NORM>
+template <typename TO, bool NORM, bool REC>
 __global__ void __launch_bounds__(NT, 1)
 chunk_scan_kernel(WideParams p, const __grid_constant__ CUtensorMap tm_v,
                        const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_gate)
 {
-    constexpr bool STAGED = sizeof(TO) == 2;  // bf16 outputs of full chunks leave by tensor stores
+    constexpr bool STAGED = sizeof(TO) == 2 && !REC;   // bf16 outputs of full chunks leave by tensor stores
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
@@ -487,6 +492,12 @@ chunk_scan_kernel(WideParams p, const __grid_constant__ CUtensorMap tm_v,
             const uint32_t d5 = tmem + lanes + TM_D5 + 128 * d;
             unsigned char *ost = sm + OFF_OST + d * OST_BYTES;   // staging tile of this chunk
             if (warp_abort()) break;
+            const size_t rec = (size_t)h * p.n_slots + (size_t)(first_slot + c_begin + k);
+            if constexpr (REC) {              // the state entering this chunk, [key channel][value]
+                float *dst = p.ck_S + rec * (size_t)(DK * DK) + (size_t)kc0 * DK + j;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) dst[(size_t)i * DK] = S[i];
+            }
             if (!warp_wait(&bars[B_S1], k & 1)) { fail(); break; }
             tc_fence_after();
             {   // U^T = -(D5^T columns tk0..) -> f16 pairs, the A operand of D7
@@ -495,6 +506,11 @@ chunk_scan_kernel(WideParams p, const __grid_constant__ CUtensorMap tm_v,
                 tmem_ld16_sync(d5 + tk0, x);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) pk[i] = pack_f16x2(-x[2 * i], -x[2 * i + 1]);
+                if constexpr (REC) {          // U of this chunk, [token][value]; rows past its end are 0
+                    float *dst = p.ck_U + rec * (size_t)(C * DK) + (size_t)tk0 * DK + j;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) dst[(size_t)i * DK] = -x[i];
+                }
                 tmem_st8u(tmem + lanes + TM_U + 8 * b, pk);
                 tmem_st_wait();
             }
@@ -502,7 +518,11 @@ chunk_scan_kernel(WideParams p, const __grid_constant__ CUtensorMap tm_v,
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_UREADY]);
             // outputs O^T[j][tk0 + i] = O[tk0 + i][j]
-            if constexpr (!NORM) {
+            if constexpr (REC) {              // records only: no outputs
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_D5FREE + d]);
+            } else if constexpr (!NORM) {
                 float o[16];
                 tmem_ld16_sync(d5 + 64 + tk0, o);
                 tc_fence_before();
@@ -618,7 +638,7 @@ chunk_scan_kernel(WideParams p, const __grid_constant__ CUtensorMap tm_v,
     if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-template <typename TO, bool NORM>
+template <typename TO, bool NORM, bool REC = false>
 cudaError_t launch_typed(const PrefillArgs &a, const unsigned char *ws, int n_slots, const NormArgs *norm,
                          long long slot_lo, long long slot_hi, cudaStream_t stream)
 {
@@ -630,18 +650,20 @@ cudaError_t launch_typed(const PrefillArgs &a, const unsigned char *ws, int n_sl
     p.slot_lo = slot_lo; p.slot_hi = slot_hi;
     p.norm_w = norm ? norm->weight : nullptr;
     p.eps = norm ? norm->eps : 0.f;
+    p.ck_S = a.ck_S; p.ck_U = a.ck_U;
     if (a.N == 0) return cudaSuccess;
     // with no token at all no CTA touches a tensor map (every sequence is empty); the maps stay zero
     CUtensorMap tv = {}, to = {}, tg = {};
     if (p.tokens > 0) {
         if (!token_rows_map(&tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, p.tokens, 64, true))
             return cudaErrorNotSupported;
-        if (sizeof(TO) == 2 && !token_rows_map(&to, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, p.tokens, 64, true))
+        if (sizeof(TO) == 2 && !REC &&
+            !token_rows_map(&to, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, p.tokens, 64, true))
             return cudaErrorNotSupported;
         if (NORM && !token_rows_map(&tg, norm->gate, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, p.tokens, 64, true))
             return cudaErrorNotSupported;
     }
-    auto kern = chunk_scan_kernel<TO, NORM>;
+    auto kern = chunk_scan_kernel<TO, NORM, REC>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     kern<<<dim3(a.H, a.N), NT, SMEM_ALLOC, stream>>>(p, tv, to, tg);
@@ -663,6 +685,13 @@ cudaError_t launch_chunk_scan(const PrefillArgs &a, const unsigned char *ws, int
     if (out_dtype == KDA_BF16)
         return launch_typed<__nv_bfloat16, false>(a, ws, n_slots, nullptr, slot_lo, slot_hi, stream);
     return launch_typed<float, false>(a, ws, n_slots, nullptr, slot_lo, slot_hi, stream);
+}
+
+cudaError_t launch_chunk_scan_records(const PrefillArgs &a, const unsigned char *ws, int n_slots,
+                                      cudaStream_t stream)
+{
+    if (!a.ck_S || !a.ck_U) return cudaErrorInvalidValue;
+    return launch_typed<float, false, true>(a, ws, n_slots, nullptr, 0, n_slots, stream);
 }
 
 }  // namespace kda

@@ -186,6 +186,11 @@ cudaError_t launch_chunk_scan(const PrefillArgs &a, const unsigned char *ws, int
                               kda_dtype_t out_dtype, cudaStream_t stream, const NormArgs *norm = nullptr,
                               long long slot_lo = 0, long long slot_hi = -1);
 
+// The same scan writing the backward pass's forward records (a.ck_S: the state entering every chunk,
+// a.ck_U: each chunk's U; both per (head, chunk slot)) instead of outputs.
+cudaError_t launch_chunk_scan_records(const PrefillArgs &a, const unsigned char *ws, int n_slots,
+                                      cudaStream_t stream);
+
 // The bf16 prefill as kda_chunk_fwd runs it (prefill.cu): with at most kPipeMaxChains (sequence,
 // head) chains and enough chunk slots, a pipeline over token ranges (scan of one range beside the
 // preparation of the next ones), else the two passes one after the other. The pipeline carries the
