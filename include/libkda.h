@@ -157,7 +157,8 @@ kda_status_t kda_chunk_scan(const void *v, const float *S0, const int32_t *cu_se
  * input, given its gradients with respect to every output o_t and to the final states.
  * The pages print no backward pass (training uses the chunk mode: lpnh.cn article, sec. 5);
  * these are the chain rule through the recurrence above, computed through the same chunk
- * form (chunk 64) in fp32 arithmetic on CUDA cores, for either input dtype.
+ * form (chunk 64). The gradients are fp32 arithmetic on CUDA cores for either input dtype; for
+ * bf16 inputs the forward records come from the tensor-core forward passes.
  *
  *   q, k, v, log_alpha, beta, S0, cu_seqlens, B, T, H, N, dk, dv, dtype:
  *              exactly as passed to kda_chunk_fwd (the forward is recomputed here).
@@ -168,8 +169,9 @@ kda_status_t kda_chunk_scan(const void *v, const float *S0, const int32_t *cu_se
  *   dbeta      [B, T, H]      float32 (written)
  *   dS0        [N, H, dk, dv] float32 (written: dL/dS0), or NULL (not computed).
  *   workspace  device buffer of kda_chunk_bwd_workspace_size(...) bytes (fp32 records
- *              of the forward and of the reverse sweep: 224 KiB per chunk slot and head,
- *              see kda_chunk_fwd_workspace_size for chunk slots). Its status word is
+ *              of the forward and of the reverse sweep and the reverse sweep's prepared
+ *              operands: 385 KiB per chunk slot and head, see kda_chunk_fwd_workspace_size
+ *              for chunk slots). Its status word is
  *              cleared by this call; cu_seqlens is checked on the device as for
  *              kda_chunk_fwd.
  * Gradient buffers must not overlap each other or the inputs. Every pointer except S0,
@@ -191,8 +193,10 @@ kda_status_t kda_chunk_bwd(const void *q, const void *k, const void *v,
  * running the phases of different batches on different streams), with the arguments of
  * kda_chunk_bwd and the same checks:
  *   phase 0  the forward sweep, recording into the workspace the state entering every chunk
- *            and each chunk's R = V - Kt S and U; clears the workspace status word first;
- *   phase 1  the reverse scan of the state gradient: writes dv_out and dS0, and records Y and
+ *            and each chunk's U (and, for fp32 inputs, R = V - Kt S); clears the workspace
+ *            status word first;
+ *   phase 1  the reverse scan of the state gradient: a data-parallel pass forms every chunk's
+ *            state-independent operands, then the scan writes dv_out and dS0, and records Y and
  *            the gradient reaching the end of every chunk;
  *   phase 2  every other gradient (dq, dk_out, dlog_alpha, dbeta), chunk by chunk.
  * Each phase reads what the earlier ones recorded, so they must run in this order on the same

@@ -24,9 +24,11 @@
 //     chunk slot). For fp32 inputs the fp32 forward kernel (chunk_fp32.cu) writes all three; for
 //     bf16 inputs the tensor-core passes do (chunk_prep.cu, then chunk_scan.cu in record mode),
 //     writing S and U, and kernel 3 forms R = V - Kt S itself;
-//  2. chunk_bwd_scan_kernel: the state gradient, chunk by chunk from the end of each sequence
-//     (one CTA per (sequence, head, 32 value columns); the columns are independent). It writes dV,
-//     dS0, Y and the gradient dS' reaching the end of every chunk;
+//  2. the state gradient, chunk by chunk from the end of each sequence, in two kernels:
+//     chunk_bwd_prep_kernel (data-parallel, one CTA per (chunk slot, head)) forms every chunk's
+//     state-independent operands (below), and chunk_bwd_rscan_kernel (one CTA per (sequence,
+//     head, 32 value columns); the columns are independent) runs the two state products per
+//     chunk and writes dV, dS0, Y and the gradient dS' reaching the end of every chunk;
 //  3. chunk_bwd_local_kernel: everything else, one CTA per (chunk slot, head), no chunk-to-chunk
 //     dependence (data-parallel over the whole grid).
 // Rows past a chunk's end are zero-filled (log_alpha = 0, k = q = v = dO = 0), which leaves every
@@ -45,159 +47,310 @@ constexpr int LDC = C + 1;       // padded row stride of the 64 x 64 tiles
 constexpr int LDV = DVB + 1;     // padded row stride of the 32-column blocks
 
 // ------------------------------------------------------------------------------------------
-// 2. reverse scan of the state gradient
+// 2a. backward preparation (data-parallel): the state-independent operands of the reverse scan
 // ------------------------------------------------------------------------------------------
-constexpr int NT_SCAN = 256;
+// With T = (I + A)^{-1}, the reverse scan's two lines become Y = Y0 + Kp dS' and
+// dS = Diag(gamma) dS' + G0 - Bk^T Y, where per chunk
+//   Kp = T^T Ke (64 x 128),  Y0 = T^T M^T dO (64 x 128),  G0 = Qt^T dO (128 x 128),  Bk = diag(beta) Kt,
+// none of which depends on the state gradient. One CTA per (chunk slot, head) forms them.
+constexpr int NT_BP = 512;
+constexpr size_t kBwdSmallFloats = 256;   // gamma (128) then beta (64) of a chunk, per (head, slot)
 
-struct ScanSmem {
-    float Kt[C * LD];
-    float Kh[C * LD];
-    float Qt[C * LD];
-    float Ke[C * LD];
-    float dS[DK * DVB];
+constexpr int LDB = DK + 4;      // row stride of the 64 x 128 tiles: 16-byte aligned rows, 4-bank skew
+struct BprepSmem {
+    float Kt[C * LDB];       // Kt, then Bk
+    float Qt[C * LDB];       // Qt, then M^T dO -> Y0 (solved in place)
+    float Kh[C * LDB];
+    float Ke[C * LDB];       // Ke -> Kp (solved in place)
+    float dO[C * LDB];
     float A[C * LDC];
     float M[C * LDC];
-    float dO[C * DVB];
-    float Y[C * DVB];        // dU, then Y in place
-    float gam[DK];
     float beta[C];
+    float gam[DK];
 };
 
 template <typename T>
-__global__ void __launch_bounds__(NT_SCAN, 1)
-chunk_bwd_scan_kernel(BwdArgs a)
+__global__ void __launch_bounds__(NT_BP, 1)
+chunk_bwd_prep_kernel(BwdArgs a)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    ScanSmem &sm = *reinterpret_cast<ScanSmem *>(smem_raw);
+    BprepSmem &sm = *reinterpret_cast<BprepSmem *>(smem_raw);
+    const int tid = threadIdx.x;
+    const int H = a.H;
+    const int h = (int)(blockIdx.x % (unsigned)H), slot = (int)(blockIdx.x / (unsigned)H);
+    int n, L;
+    int64_t s;
+    if (!slot_to_chunk(a.cu_seqlens, a.N, a.T, slot, &n, &s, &L)) return;
+    const size_t rec = (size_t)h * a.n_slots + (size_t)slot;
+    if (!in_bounds(a.status, s, L, (long long)a.B * a.T) ||
+        !in_bounds(a.status, (long long)rec, 1, (long long)H * a.n_slots))
+        return;
+    fp32c::load_rows<T, NT_BP, DK>(sm.Kt, LDB, (const T *)a.k, s, L, H, h, 0, tid);
+    fp32c::load_rows<T, NT_BP, DK>(sm.Qt, LDB, (const T *)a.q, s, L, H, h, 0, tid);
+    fp32c::load_rows<float, NT_BP, DK>(sm.Kh, LDB, a.log_alpha, s, L, H, h, 0, tid);
+    fp32c::load_rows<T, NT_BP, DK>(sm.dO, LDB, (const T *)a.dout, s, L, H, h, 0, tid);
+    if (tid < C) sm.beta[tid] = (tid < L) ? a.beta[(size_t)(s + tid) * H + h] : 0.f;
+    __syncthreads();
+    {   // decay: Kt = K e^g, Qt = Q e^g, Kh = K e^-g, Ke = K e^(g_last - g)
+        const float gl = fp32c::decay_prefix<NT_BP>(sm.Kh, LDB, tid);
+        constexpr int RP = C / (NT_BP / DK);
+        const int c = tid % DK, r0 = (tid / DK) * RP;
+        if (tid < DK) sm.gam[c] = expf(gl);
+        if (tid < DK && !(gl >= kMinChunkLogDecay)) set_status(a.status, KDA_ERR_UNSUPPORTED);
+#pragma unroll 4
+        for (int r = r0; r < r0 + RP; ++r) {
+            const float gr = sm.Kh[r * LDB + c], kk = sm.Kt[r * LDB + c];
+            const float e = expf(gr);
+            sm.Kt[r * LDB + c] = kk * e;
+            sm.Qt[r * LDB + c] *= e;
+            sm.Kh[r * LDB + c] = kk * expf(-gr);
+            sm.Ke[r * LDB + c] = kk * expf(gl - gr);
+        }
+    }
+    __syncthreads();
+    {   // A = StrictLower(diag(beta) Kt Kh^T) (threads 0-255), M = tril(Qt Kh^T) (256-511); 4x4 tiles
+        const bool isM = tid >= 256;
+        const int t = tid & 255, rb = t / 16, ib = t % 16;
+        const float *X = isM ? sm.Qt : sm.Kt;
+        float acc[4][4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+            for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
+        if (ib <= rb) {
+            for (int c = 0; c < DK; ++c) {
+                float xr[4], kh[4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) { xr[x] = X[(4 * rb + x) * LDB + c]; kh[x] = sm.Kh[(4 * ib + x) * LDB + c]; }
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) acc[x][y] += xr[x] * kh[y];
+            }
+        }
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+            for (int y = 0; y < 4; ++y) {
+                const int r = 4 * rb + x, i = 4 * ib + y;
+                if (isM) sm.M[r * LDC + i] = (i <= r) ? acc[x][y] : 0.f;
+                else sm.A[r * LDC + i] = (i < r) ? sm.beta[r] * acc[x][y] : 0.f;
+            }
+    }
+    __syncthreads();
+    {   // G0 = Qt^T dO: thread -> key channels 4 (tid / 16) .. + 3, value columns 8 (tid % 16) .. + 7
+        const int c0 = 4 * (tid >> 4), j0 = 8 * (tid & 15);
+        float acc[4][8];
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+            for (int y = 0; y < 8; ++y) acc[x][y] = 0.f;
+        for (int r = 0; r < C; ++r) {
+            const float4 q4 = *reinterpret_cast<const float4 *>(sm.Qt + r * LDB + c0);
+            const float4 o0 = *reinterpret_cast<const float4 *>(sm.dO + r * LDB + j0);
+            const float4 o1 = *reinterpret_cast<const float4 *>(sm.dO + r * LDB + j0 + 4);
+            const float qt[4] = {q4.x, q4.y, q4.z, q4.w};
+            const float o[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int y = 0; y < 8; ++y) acc[x][y] += qt[x] * o[y];
+        }
+        float *g0 = a.ck_G0 + rec * kBwdStateFloats;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            float4 *dst = reinterpret_cast<float4 *>(g0 + (size_t)(c0 + x) * DK + j0);
+            dst[0] = make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
+            dst[1] = make_float4(acc[x][4], acc[x][5], acc[x][6], acc[x][7]);
+        }
+    }
+    __syncthreads();                      // Qt is dead
+    {   // M^T dO into Qt's place: thread -> rows 4 (tid / 32) .. + 3, columns 4 (tid % 32) .. + 3
+        const int r0 = 4 * (tid >> 5), j0 = 4 * (tid & 31);
+        float acc[4][4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+            for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
+        for (int i = r0; i < C; ++i) {
+            float m[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) m[x] = sm.M[i * LDC + r0 + x];       // M^T[r][i] = M[i][r]
+            const float4 o4 = *reinterpret_cast<const float4 *>(sm.dO + i * LDB + j0);
+            const float o[4] = {o4.x, o4.y, o4.z, o4.w};
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) acc[x][y] += m[x] * o[y];
+        }
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+            for (int y = 0; y < 4; ++y) sm.Qt[(r0 + x) * LDB + j0 + y] = acc[x][y];
+    }
+    // Bk = diag(beta) Kt (Kt is not needed any more) and the chunk's gamma and beta
+    for (int idx = tid; idx < C * DK; idx += NT_BP) {
+        const int r = idx / DK, c = idx % DK;
+        a.ck_Bk[rec * kBwdRowsFloats + idx] = sm.beta[r] * sm.Kt[r * LDB + c];
+    }
+    if (tid < DK) a.ck_gb[rec * kBwdSmallFloats + tid] = sm.gam[tid];
+    else if (tid < DK + C) a.ck_gb[rec * kBwdSmallFloats + tid] = sm.beta[tid - DK];
+    __syncthreads();
+    // (I + A)^T X = B for B = M^T dO (in Qt) and B = Ke, 16-row blocks from the last: the block minus
+    // the solved rows below it (all threads), then back substitution inside the block (a thread per
+    // column, 128 columns of each matrix)
+#pragma unroll 1
+    for (int b = 3; b >= 0; --b) {
+        if (b < 3) {
+            for (int idx = tid; idx < 2 * 16 * DK; idx += NT_BP) {
+                float *X = (idx < 16 * DK) ? sm.Qt : sm.Ke;
+                const int e = idx % (16 * DK), r = 16 * b + e / DK, j = e % DK;
+                float v = X[r * LDB + j];
+                for (int i = 16 * (b + 1); i < C; ++i) v -= sm.A[i * LDC + r] * X[i * LDB + j];
+                X[r * LDB + j] = v;
+            }
+        }
+        __syncthreads();
+        if (tid < 2 * DK) {
+            float *X = (tid < DK) ? sm.Qt : sm.Ke;
+            const int j = tid % DK;
+            float y[16];
+#pragma unroll
+            for (int r = 15; r >= 0; --r) {
+                float v = X[(16 * b + r) * LDB + j];
+#pragma unroll
+                for (int i = r + 1; i < 16; ++i) v -= sm.A[(16 * b + i) * LDC + 16 * b + r] * y[i];
+                y[r] = v;
+                X[(16 * b + r) * LDB + j] = v;
+            }
+        }
+        __syncthreads();
+    }
+    for (int idx = tid; idx < C * DK; idx += NT_BP) {
+        const int r = idx / DK, c = idx % DK;
+        a.ck_Y0[rec * kBwdRowsFloats + idx] = sm.Qt[r * LDB + c];
+        a.ck_Kp[rec * kBwdRowsFloats + idx] = sm.Ke[r * LDB + c];
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// 2b. reverse scan of the state gradient on the prepared operands
+// ------------------------------------------------------------------------------------------
+// Per chunk, from the last: record dS' (the gradient reaching the chunk's end), Y = Y0 + Kp dS',
+// dV = diag(beta) Y, record Y, dS = Diag(gamma) dS' + G0 - Bk^T Y. One CTA per (sequence, head,
+// 32 value columns); the next chunk's operands are copied in (cp.async, two buffers) while this
+// one is computed.
+constexpr int NT_RS = 256;
+constexpr int LDP = DK + 4;      // row stride of the 64 x 128 operand tiles (16-byte aligned rows)
+
+struct RscanBuf {
+    float Kp[C * LDP];
+    float Bk[C * LDP];
+    float Y0[C * DVB];
+    float G0[DK * DVB];
+    float gb[kBwdSmallFloats];
+};
+struct RscanSmem {
+    RscanBuf buf[2];
+    float dS[DK * DVB];
+    float Y[C * DVB];
+};
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+template <typename T>
+__global__ void __launch_bounds__(NT_RS, 1)
+chunk_bwd_rscan_kernel(BwdArgs a)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    RscanSmem &sm = *reinterpret_cast<RscanSmem *>(smem_raw);
     const int tid = threadIdx.x;
     const int j0 = blockIdx.x * DVB;
     const int h = blockIdx.y;
     const int n = blockIdx.z;
     const int H = a.H;
-    const T *q = (const T *)a.q;
-    const T *k = (const T *)a.k;
-    const T *dout = (const T *)a.dout;
-
     int64_t t0, t1;
     if (!sequence_span(a.cu_seqlens, n, a.N, a.T, &t0, &t1, a.status)) return;
-
     const size_t sbase = ((size_t)n * H + h) * DK * DK;
     if (!in_bounds(a.status, (long long)sbase, DK * DK, (long long)a.N * H * DK * DK)) return;
-    for (int idx = tid; idx < DK * DVB; idx += NT_SCAN) {
+    for (int idx = tid; idx < DK * DVB; idx += NT_RS) {
         const int c = idx / DVB, j = idx % DVB;
         sm.dS[idx] = a.dS_final ? a.dS_final[sbase + (size_t)c * DK + j0 + j] : 0.f;
     }
-
     const int64_t n_chunks = (t1 - t0 + C - 1) / C;
+    auto record_of = [&](int64_t ci) { return (size_t)h * a.n_slots + (size_t)chunk_slot(t0 + ci * C, n); };
+    // copy the prepared operands of chunk ci into buffer b (16-byte pieces, 11 or 12 per thread)
+    auto fetch = [&](int64_t ci, int b) {
+        const size_t rec = record_of(ci);
+        RscanBuf &B = sm.buf[b];
+        const float *kp = a.ck_Kp + rec * kBwdRowsFloats, *bk = a.ck_Bk + rec * kBwdRowsFloats;
+        for (int idx = tid; idx < C * (DK / 4); idx += NT_RS) {
+            const int r = idx / (DK / 4), q = idx % (DK / 4);
+            cp_async16(B.Kp + r * LDP + 4 * q, kp + (size_t)r * DK + 4 * q);
+            cp_async16(B.Bk + r * LDP + 4 * q, bk + (size_t)r * DK + 4 * q);
+        }
+        const float *y0 = a.ck_Y0 + rec * kBwdRowsFloats + j0, *g0 = a.ck_G0 + rec * kBwdStateFloats + j0;
+        for (int idx = tid; idx < C * (DVB / 4); idx += NT_RS) {
+            const int r = idx / (DVB / 4), q = idx % (DVB / 4);
+            cp_async16(B.Y0 + r * DVB + 4 * q, y0 + (size_t)r * DK + 4 * q);
+        }
+        for (int idx = tid; idx < DK * (DVB / 4); idx += NT_RS) {
+            const int c = idx / (DVB / 4), q = idx % (DVB / 4);
+            cp_async16(B.G0 + c * DVB + 4 * q, g0 + (size_t)c * DK + 4 * q);
+        }
+        if (tid < (int)(kBwdSmallFloats / 4)) cp_async16(B.gb + 4 * tid, a.ck_gb + rec * kBwdSmallFloats + 4 * tid);
+        cp_async_commit();
+    };
+    if (n_chunks > 0) fetch(n_chunks - 1, 0);
     for (int64_t ci = n_chunks - 1; ci >= 0; --ci) {
+        const int b = (int)((n_chunks - 1 - ci) & 1);
         const int64_t s = t0 + ci * C;
         const int L = (t1 - s < C) ? (int)(t1 - s) : C;
-        const size_t rec = (size_t)h * a.n_slots + (size_t)chunk_slot(s, n);
+        const size_t rec = record_of(ci);
         if (!in_bounds(a.status, s, L, (long long)a.B * a.T) ||
             !in_bounds(a.status, (long long)rec, 1, (long long)H * a.n_slots))
             break;
+        __syncthreads();                  // the other buffer is free (its chunk is done)
+        if (ci > 0) { fetch(ci - 1, b ^ 1); cp_async_wait1(); } else { cp_async_wait0(); }
+        // record dS' (the gradient reaching this chunk's end) while the operands are in use
+        fp32c::store_block32<NT_RS>(a.ck_dS + rec * kBwdStateFloats + j0, DK, sm.dS, DK, tid);
         __syncthreads();
-        // ---- load the chunk (k -> Kt, q -> Qt, log_alpha -> Kh, dO block) and record dS'
-        fp32c::load_chunk<T, NT_SCAN>(sm.Kt, sm.Qt, sm.Kh, LD, sm.dO, q, k, a.log_alpha, dout, s, L, H, h, j0, tid);
-        if (tid < C) sm.beta[tid] = (tid < L) ? a.beta[(size_t)(s + tid) * H + h] : 0.f;
-        fp32c::store_block32<NT_SCAN>(a.ck_dS + rec * kBwdStateFloats + j0, DK, sm.dS, DK, tid);
-        __syncthreads();
-
-        // ---- cumulative log-decay (all threads, in row parts), then the decay-scaled operands
-        {
-            const float gl = fp32c::decay_prefix<NT_SCAN>(sm.Kh, LD, tid);
-            constexpr int RP = C / (NT_SCAN / DK);
-            const int c = tid % DK, r0 = (tid / DK) * RP;
-            if (tid < DK) sm.gam[c] = expf(gl);
-            if (tid < DK && !(gl >= kMinChunkLogDecay)) set_status(a.status, KDA_ERR_UNSUPPORTED);
-#pragma unroll 4
-            for (int r = r0; r < r0 + RP; ++r) {
-                const float gr = sm.Kh[r * LD + c];
-                const float kk = sm.Kt[r * LD + c];
-                const float e = expf(gr);
-                sm.Kt[r * LD + c] = kk * e;
-                sm.Qt[r * LD + c] *= e;
-                sm.Kh[r * LD + c] = kk * expf(-gr);
-                sm.Ke[r * LD + c] = kk * expf(gl - gr);
-            }
-        }
-        __syncthreads();
-
-        // ---- A = StrictLower(diag(beta) Kt Kh^T), M = tril(Qt Kh^T); 4x4 register tiles
-        {
-            const int rb = tid / 16, ib = tid % 16;
-            float accA[4][4], accM[4][4];
-#pragma unroll
-            for (int x = 0; x < 4; ++x)
-#pragma unroll
-                for (int y = 0; y < 4; ++y) { accA[x][y] = 0.f; accM[x][y] = 0.f; }
-            if (ib <= rb) {
-                for (int c = 0; c < DK; ++c) {
-                    float kt[4], qt[4], kh[4];
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        kt[x] = sm.Kt[(4 * rb + x) * LD + c];
-                        qt[x] = sm.Qt[(4 * rb + x) * LD + c];
-                        kh[x] = sm.Kh[(4 * ib + x) * LD + c];
-                    }
-#pragma unroll
-                    for (int x = 0; x < 4; ++x)
-#pragma unroll
-                        for (int y = 0; y < 4; ++y) {
-                            accA[x][y] += kt[x] * kh[y];
-                            accM[x][y] += qt[x] * kh[y];
-                        }
-                }
-            }
-#pragma unroll
-            for (int x = 0; x < 4; ++x)
-#pragma unroll
-                for (int y = 0; y < 4; ++y) {
-                    const int r = 4 * rb + x, i = 4 * ib + y;
-                    sm.A[r * LDC + i] = (i < r) ? sm.beta[r] * accA[x][y] : 0.f;
-                    sm.M[r * LDC + i] = (i <= r) ? accM[x][y] : 0.f;
-                }
-        }
-        __syncthreads();
-
-        // ---- dU = M^T dO + Ke dS': thread -> row r, 8 columns
-        {
+        const RscanBuf &B = sm.buf[b];
+        {   // Y = Y0 + Kp dS': thread -> row tid / 4, 8 columns
             const int r = tid / 4, jg = (tid % 4) * 8;
             float acc[8];
 #pragma unroll
-            for (int x = 0; x < 8; ++x) acc[x] = 0.f;
-            for (int i = r; i < C; ++i) fp32c::axpy<8>(acc, sm.M[i * LDC + r], sm.dO + i * DVB + jg);
-            for (int c = 0; c < DK; ++c) fp32c::axpy<8>(acc, sm.Ke[r * LD + c], sm.dS + c * DVB + jg);
+            for (int x = 0; x < 8; ++x) acc[x] = B.Y0[r * DVB + jg + x];
+#pragma unroll 4
+            for (int c = 0; c < DK; ++c) fp32c::axpy<8>(acc, B.Kp[r * LDP + c], sm.dS + c * DVB + jg);
 #pragma unroll
             for (int x = 0; x < 8; ++x) sm.Y[r * DVB + jg + x] = acc[x];
         }
         __syncthreads();
-
-        // ---- Y = (I + A)^{-T} dU: blocked back substitution in place
-        fp32c::upper_solve_32<NT_SCAN>(sm.A, LDC, sm.Y, tid);
-
-        // ---- dV = diag(beta) Y -> dv (rows < L); Y -> record (all rows)
-        fp32c::store_block32<NT_SCAN>(a.ck_Y + rec * kBwdRowsFloats + j0, DK, sm.Y, C, tid);
-        fp32c::store_block32<NT_SCAN>(a.dv + ((size_t)s * H + h) * DK + j0, (size_t)H * DK, sm.Y, L, tid, sm.beta);
-
-        // ---- dS <- Diag(gamma) dS' + Qt^T dO - Kt^T diag(beta) Y: thread -> key channel c, 16 columns
-        {
+        fp32c::store_block32<NT_RS>(a.ck_Y + rec * kBwdRowsFloats + j0, DK, sm.Y, C, tid);
+        fp32c::store_block32<NT_RS>(a.dv + ((size_t)s * H + h) * DK + j0, (size_t)H * DK, sm.Y, L, tid, B.gb + DK);
+        {   // dS = Diag(gamma) dS' + G0 - Bk^T Y: thread -> key channel tid / 2, 16 columns
             const int c = tid / 2, jh = (tid % 2) * 16;
+            const float gm = B.gb[c];
             float acc[16];
-            const float gm = sm.gam[c];
 #pragma unroll
-            for (int x = 0; x < 16; ++x) acc[x] = gm * sm.dS[c * DVB + jh + x];
-            for (int r = 0; r < C; ++r) {
-                fp32c::axpy<16>(acc, sm.Qt[r * LD + c], sm.dO + r * DVB + jh);
-                fp32c::axpy<16>(acc, -sm.Kt[r * LD + c] * sm.beta[r], sm.Y + r * DVB + jh);
-            }
+            for (int x = 0; x < 16; ++x) acc[x] = gm * sm.dS[c * DVB + jh + x] + B.G0[c * DVB + jh + x];
+#pragma unroll 4
+            for (int r = 0; r < C; ++r) fp32c::axpy<16>(acc, -B.Bk[r * LDP + c], sm.Y + r * DVB + jh);
+            __syncthreads();              // every thread has read dS' (Y step and this one)
 #pragma unroll
             for (int x = 0; x < 16; ++x) sm.dS[c * DVB + jh + x] = acc[x];
         }
     }
+    cp_async_wait0();
     __syncthreads();
     if (a.dS0) {
-        for (int idx = tid; idx < DK * DVB; idx += NT_SCAN) {
+        for (int idx = tid; idx < DK * DVB; idx += NT_RS) {
             const int c = idx / DVB, j = idx % DVB;
             a.dS0[sbase + (size_t)c * DK + j0 + j] = sm.dS[idx];
         }
@@ -500,13 +653,18 @@ chunk_bwd_local_kernel(BwdArgs a)
 }
 
 template <typename T>
-cudaError_t launch_scan_typed(const BwdArgs &a, cudaStream_t stream)
+cudaError_t launch_rscan_typed(const BwdArgs &a, cudaStream_t stream)
 {
-    const size_t smem = sizeof(ScanSmem);
-    cudaError_t e = cudaFuncSetAttribute(chunk_bwd_scan_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(chunk_bwd_prep_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sizeof(BprepSmem));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(chunk_bwd_rscan_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(RscanSmem));
     if (e != cudaSuccess) return e;
-    chunk_bwd_scan_kernel<T><<<dim3(DK / DVB, a.H, a.N), NT_SCAN, smem, stream>>>(a);
+    chunk_bwd_prep_kernel<T><<<(unsigned)((long long)a.n_slots * a.H), NT_BP, sizeof(BprepSmem), stream>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    chunk_bwd_rscan_kernel<T><<<dim3(DK / DVB, a.H, a.N), NT_RS, sizeof(RscanSmem), stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -533,7 +691,9 @@ cudaError_t launch_local_typed(const BwdArgs &a, cudaStream_t stream)
 cudaError_t launch_chunk_bwd_scan(const BwdArgs &a, kda_dtype_t dtype, cudaStream_t stream)
 {
     if (a.N == 0) return cudaSuccess;
-    return dtype == KDA_BF16 ? launch_scan_typed<__nv_bfloat16>(a, stream) : launch_scan_typed<float>(a, stream);
+    if (!a.ck_Kp || !a.ck_Bk || !a.ck_Y0 || !a.ck_G0 || !a.ck_gb) return cudaErrorInvalidValue;
+    // the data-parallel preparation of every chunk's operands, then the reverse scan
+    return dtype == KDA_BF16 ? launch_rscan_typed<__nv_bfloat16>(a, stream) : launch_rscan_typed<float>(a, stream);
 }
 
 cudaError_t launch_chunk_bwd_local(const BwdArgs &a, kda_dtype_t dtype, cudaStream_t stream)

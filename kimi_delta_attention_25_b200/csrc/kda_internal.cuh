@@ -211,6 +211,9 @@ struct BwdArgs {
     float *dq, *dk, *dv, *dlog_alpha, *dbeta, *dS0;
     const float *ck_S, *ck_R, *ck_U;   // from the forward sweep
     float *ck_dS, *ck_Y;               // from the reverse scan
+    // state-independent operands of the reverse scan (per (head, slot)), formed by a data-parallel
+    // pass before it when given: Kp, Bk, Y0 (64 x 128), G0 (128 x 128), gamma and beta (256 floats)
+    float *ck_Kp = nullptr, *ck_Bk = nullptr, *ck_Y0 = nullptr, *ck_G0 = nullptr, *ck_gb = nullptr;
     int B, T, H, N, n_slots;
     int32_t *status;
 };

@@ -169,8 +169,10 @@ def _bwd(lib, **kw):
 
 def test_backward_host_checks(lib):
     need = kda.chunk_bwd_workspace_size(1, 64, 2, 1)
-    # 2 heads x (64 / 64 + 1 + 1) slots x (2 states + 3 row blocks) of fp32, after the status prefix
-    assert need == 256 + 2 * 3 * (2 * 128 * 128 + 3 * 64 * 128) * 4
+    # 2 heads x (64 / 64 + 1 + 1) slots of fp32 records, after the status prefix
+    # per (head, chunk slot): S, dS' (128 x 128); R, U, Y (64 x 128); the reverse scan's prepared
+    # operands Kp, Bk, Y0 (64 x 128), G0 (128 x 128), gamma and beta (256)
+    assert need == 256 + 2 * 3 * (3 * 128 * 128 + 6 * 64 * 128 + 256) * 4
     assert kda.chunk_bwd_workspace_size(1, 64, 2, 1, dk=64) == 0
     # the first failing check decides; none of these reaches a CUDA call
     assert _bwd(lib, dk=64) == kda.KDA_ERR_UNSUPPORTED
