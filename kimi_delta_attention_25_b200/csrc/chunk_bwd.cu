@@ -42,9 +42,10 @@ namespace {
 constexpr int C = kChunk;
 constexpr int DK = kHeadDim;
 constexpr int DVB = 32;          // value columns per block
-constexpr int LD = DK + 1;       // padded row stride of the 64 x 128 operand tiles
-constexpr int LDC = C + 1;       // padded row stride of the 64 x 64 tiles
-constexpr int LDV = DVB + 1;     // padded row stride of the 32-column blocks
+constexpr int LD = DK + 4;       // row stride of the 64 x 128 operand tiles (16-byte aligned rows)
+constexpr int LDC = C + 1;       // padded row stride of the 64 x 64 tiles read by scalar loads
+constexpr int LDC4 = C + 4;      // row stride of the 64 x 64 tiles read as float4
+constexpr int LDV = DVB + 4;     // row stride of the 32-column blocks (16-byte aligned rows)
 
 // ------------------------------------------------------------------------------------------
 // 2a. backward preparation (data-parallel): the state-independent operands of the reverse scan
@@ -108,47 +109,59 @@ chunk_bwd_prep_kernel(BwdArgs a)
         }
     }
     __syncthreads();
-    {   // A = StrictLower(diag(beta) Kt Kh^T) (threads 0-255), M = tril(Qt Kh^T) (256-511); 4x4 tiles
+    {   // A = StrictLower(diag(beta) Kt Kh^T) (threads 0-255), M = tril(Qt Kh^T) (256-511): thread ->
+        // rows rb + 16 x, columns ib + 16 y (x, y < 4), float4 steps along the key channels, so that
+        // the 8 lanes of a shared-memory phase read one X row (a broadcast) and 8 Kh rows that fall
+        // in 8 distinct bank groups (a row stride of 33 groups)
         const bool isM = tid >= 256;
-        const int t = tid & 255, rb = t / 16, ib = t % 16;
+        const int t = tid & 255, rb = t >> 4, ib = t & 15;
         const float *X = isM ? sm.Qt : sm.Kt;
         float acc[4][4];
 #pragma unroll
         for (int x = 0; x < 4; ++x)
 #pragma unroll
             for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
-        if (ib <= rb) {
-            for (int c = 0; c < DK; ++c) {
-                float xr[4], kh[4];
+#pragma unroll 2
+        for (int c = 0; c < DK; c += 4) {
+            float4 xr[4], kh[4];
 #pragma unroll
-                for (int x = 0; x < 4; ++x) { xr[x] = X[(4 * rb + x) * LDB + c]; kh[x] = sm.Kh[(4 * ib + x) * LDB + c]; }
-#pragma unroll
-                for (int x = 0; x < 4; ++x)
-#pragma unroll
-                    for (int y = 0; y < 4; ++y) acc[x][y] += xr[x] * kh[y];
+            for (int x = 0; x < 4; ++x) {
+                xr[x] = *reinterpret_cast<const float4 *>(X + (rb + 16 * x) * LDB + c);
+                kh[x] = *reinterpret_cast<const float4 *>(sm.Kh + (ib + 16 * x) * LDB + c);
             }
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    acc[x][y] += xr[x].x * kh[y].x;
+                    acc[x][y] += xr[x].y * kh[y].y;
+                    acc[x][y] += xr[x].z * kh[y].z;
+                    acc[x][y] += xr[x].w * kh[y].w;
+                }
         }
 #pragma unroll
         for (int x = 0; x < 4; ++x)
 #pragma unroll
             for (int y = 0; y < 4; ++y) {
-                const int r = 4 * rb + x, i = 4 * ib + y;
+                const int r = rb + 16 * x, i = ib + 16 * y;
                 if (isM) sm.M[r * LDC + i] = (i <= r) ? acc[x][y] : 0.f;
                 else sm.A[r * LDC + i] = (i < r) ? sm.beta[r] * acc[x][y] : 0.f;
             }
     }
     __syncthreads();
-    {   // G0 = Qt^T dO: thread -> key channels 4 (tid / 16) .. + 3, value columns 8 (tid % 16) .. + 7
-        const int c0 = 4 * (tid >> 4), j0 = 8 * (tid & 15);
+    {   // G0 = Qt^T dO: thread -> key channels 4 (tid / 16) .. + 3, value columns j0 .. + 3 and
+        // 64 + j0 .. + 3 with j0 = 4 (tid % 16) (8 lanes of a phase: 8 distinct bank groups)
+        const int c0 = 4 * (tid >> 4), j0 = 4 * (tid & 15);
         float acc[4][8];
 #pragma unroll
         for (int x = 0; x < 4; ++x)
 #pragma unroll
             for (int y = 0; y < 8; ++y) acc[x][y] = 0.f;
+#pragma unroll 4
         for (int r = 0; r < C; ++r) {
             const float4 q4 = *reinterpret_cast<const float4 *>(sm.Qt + r * LDB + c0);
             const float4 o0 = *reinterpret_cast<const float4 *>(sm.dO + r * LDB + j0);
-            const float4 o1 = *reinterpret_cast<const float4 *>(sm.dO + r * LDB + j0 + 4);
+            const float4 o1 = *reinterpret_cast<const float4 *>(sm.dO + r * LDB + 64 + j0);
             const float qt[4] = {q4.x, q4.y, q4.z, q4.w};
             const float o[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
 #pragma unroll
@@ -159,9 +172,9 @@ chunk_bwd_prep_kernel(BwdArgs a)
         float *g0 = a.ck_G0 + rec * kBwdStateFloats;
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
-            float4 *dst = reinterpret_cast<float4 *>(g0 + (size_t)(c0 + x) * DK + j0);
-            dst[0] = make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
-            dst[1] = make_float4(acc[x][4], acc[x][5], acc[x][6], acc[x][7]);
+            float *dst = g0 + (size_t)(c0 + x) * DK + j0;
+            *reinterpret_cast<float4 *>(dst) = make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
+            *reinterpret_cast<float4 *>(dst + 64) = make_float4(acc[x][4], acc[x][5], acc[x][6], acc[x][7]);
         }
     }
     __syncthreads();                      // Qt is dead
@@ -189,9 +202,12 @@ chunk_bwd_prep_kernel(BwdArgs a)
             for (int y = 0; y < 4; ++y) sm.Qt[(r0 + x) * LDB + j0 + y] = acc[x][y];
     }
     // Bk = diag(beta) Kt (Kt is not needed any more) and the chunk's gamma and beta
-    for (int idx = tid; idx < C * DK; idx += NT_BP) {
-        const int r = idx / DK, c = idx % DK;
-        a.ck_Bk[rec * kBwdRowsFloats + idx] = sm.beta[r] * sm.Kt[r * LDB + c];
+    for (int idx = tid; idx < C * DK / 4; idx += NT_BP) {
+        const int r = idx / (DK / 4), c = 4 * (idx % (DK / 4));
+        const float bt = sm.beta[r];
+        const float4 k4 = *reinterpret_cast<const float4 *>(sm.Kt + r * LDB + c);
+        *reinterpret_cast<float4 *>(a.ck_Bk + rec * kBwdRowsFloats + 4 * idx) =
+            make_float4(bt * k4.x, bt * k4.y, bt * k4.z, bt * k4.w);
     }
     if (tid < DK) a.ck_gb[rec * kBwdSmallFloats + tid] = sm.gam[tid];
     else if (tid < DK + C) a.ck_gb[rec * kBwdSmallFloats + tid] = sm.beta[tid - DK];
@@ -201,14 +217,20 @@ chunk_bwd_prep_kernel(BwdArgs a)
     // column, 128 columns of each matrix)
 #pragma unroll 1
     for (int b = 3; b >= 0; --b) {
-        if (b < 3) {
-            for (int idx = tid; idx < 2 * 16 * DK; idx += NT_BP) {
-                float *X = (idx < 16 * DK) ? sm.Qt : sm.Ke;
-                const int e = idx % (16 * DK), r = 16 * b + e / DK, j = e % DK;
-                float v = X[r * LDB + j];
-                for (int i = 16 * (b + 1); i < C; ++i) v -= sm.A[i * LDC + r] * X[i * LDB + j];
-                X[r * LDB + j] = v;
+        if (b < 3) {   // thread -> matrix tid / 256, rows r, r + 1 of the block, columns j .. j + 3
+            float *X = (tid < 256) ? sm.Qt : sm.Ke;
+            const int t = tid & 255, r = 16 * b + 2 * (t >> 5), j = 4 * (t & 31);
+            float4 v0 = *reinterpret_cast<const float4 *>(X + r * LDB + j);
+            float4 v1 = *reinterpret_cast<const float4 *>(X + (r + 1) * LDB + j);
+#pragma unroll 4
+            for (int i = 16 * (b + 1); i < C; ++i) {
+                const float a0 = sm.A[i * LDC + r], a1 = sm.A[i * LDC + r + 1];
+                const float4 x = *reinterpret_cast<const float4 *>(X + i * LDB + j);
+                v0.x -= a0 * x.x; v0.y -= a0 * x.y; v0.z -= a0 * x.z; v0.w -= a0 * x.w;
+                v1.x -= a1 * x.x; v1.y -= a1 * x.y; v1.z -= a1 * x.z; v1.w -= a1 * x.w;
             }
+            *reinterpret_cast<float4 *>(X + r * LDB + j) = v0;
+            *reinterpret_cast<float4 *>(X + (r + 1) * LDB + j) = v1;
         }
         __syncthreads();
         if (tid < 2 * DK) {
@@ -226,10 +248,12 @@ chunk_bwd_prep_kernel(BwdArgs a)
         }
         __syncthreads();
     }
-    for (int idx = tid; idx < C * DK; idx += NT_BP) {
-        const int r = idx / DK, c = idx % DK;
-        a.ck_Y0[rec * kBwdRowsFloats + idx] = sm.Qt[r * LDB + c];
-        a.ck_Kp[rec * kBwdRowsFloats + idx] = sm.Ke[r * LDB + c];
+    for (int idx = tid; idx < C * DK / 4; idx += NT_BP) {
+        const int r = idx / (DK / 4), c = 4 * (idx % (DK / 4));
+        *reinterpret_cast<float4 *>(a.ck_Y0 + rec * kBwdRowsFloats + 4 * idx) =
+            *reinterpret_cast<const float4 *>(sm.Qt + r * LDB + c);
+        *reinterpret_cast<float4 *>(a.ck_Kp + rec * kBwdRowsFloats + 4 * idx) =
+            *reinterpret_cast<const float4 *>(sm.Ke + r * LDB + c);
     }
 }
 
@@ -255,6 +279,15 @@ struct RscanSmem {
     float dS[DK * DVB];
     float Y[C * DVB];
 };
+
+// acc + a.x b.x + a.y b.y + a.z b.z + a.w b.w, added in that order
+__device__ __forceinline__ float dot4acc(float acc, const float4 a, const float4 b) {
+    acc += a.x * b.x;
+    acc += a.y * b.y;
+    acc += a.z * b.z;
+    acc += a.w * b.w;
+    return acc;
+}
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src) : "memory");
@@ -367,7 +400,8 @@ struct LocalSmem {
     float Kh[C * LD];        // after the last products: dg
     float Qt[C * LD];
     float E[C * LD];
-    // one 32-column block of the value axis at a time; after the loop: dM and dP (64 x LDC each)
+    // one 32-column block of the value axis at a time; after the loop: dM, dP and their transposes
+    // (64 x LDC4 each)
     float S[DK * LDV];
     float dSn[DK * LDV];
     float dO[C * LDV];       // after the last products: per-warp column sums (16 x 128)
@@ -381,6 +415,7 @@ struct LocalSmem {
     float ry[C];
 };
 static_assert((NT_LOC / 32) * DK <= C * LDV, "per-warp column sums must fit the dO block");
+static_assert(4 * C * LDC4 <= 2 * DK * LDV + 4 * C * LDV, "dM, dP and their transposes must fit the staging area");
 
 // COMPUTE_R: no R record (the forward records came from the bf16 state scan, which holds S and U
 // but not R). R enters only dbeta, through sum_v R_rv Y_rv = sum_v V_rv Y_rv - sum_c Kt_rc (Y S^T)_rc;
@@ -439,13 +474,15 @@ chunk_bwd_local_kernel(BwdArgs a)
         float acc[4][2];
 #pragma unroll
         for (int x = 0; x < 4; ++x) { acc[x][0] = 0.f; acc[x][1] = 0.f; }
-        for (int c = 0; c < DK; ++c) {
-            float kt[4];
+#pragma unroll 2
+        for (int c = 0; c < DK; c += 4) {      // float4 steps: Kt rows broadcast, Kh rows conflict-free
+            float4 kt[4];
 #pragma unroll
-            for (int x = 0; x < 4; ++x) kt[x] = sm.Kt[(4 * rb + x) * LD + c];
-            const float kh0 = sm.Kh[cb * LD + c], kh1 = sm.Kh[(cb + 32) * LD + c];
+            for (int x = 0; x < 4; ++x) kt[x] = *reinterpret_cast<const float4 *>(sm.Kt + (4 * rb + x) * LD + c);
+            const float4 kh0 = *reinterpret_cast<const float4 *>(sm.Kh + cb * LD + c);
+            const float4 kh1 = *reinterpret_cast<const float4 *>(sm.Kh + (cb + 32) * LD + c);
 #pragma unroll
-            for (int x = 0; x < 4; ++x) { acc[x][0] += kt[x] * kh0; acc[x][1] += kt[x] * kh1; }
+            for (int x = 0; x < 4; ++x) { acc[x][0] = dot4acc(acc[x][0], kt[x], kh0); acc[x][1] = dot4acc(acc[x][1], kt[x], kh1); }
         }
 #pragma unroll
         for (int x = 0; x < 4; ++x)
@@ -491,55 +528,67 @@ chunk_bwd_local_kernel(BwdArgs a)
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
                 const int idx = tid + it * NT_LOC, c = idx >> 3, v = (idx & 7) * 4;
-                float *ds = sm.S + c * LDV + v, *dd = sm.dSn + c * LDV + v;
-                ds[0] = xs[it].x; ds[1] = xs[it].y; ds[2] = xs[it].z; ds[3] = xs[it].w;
-                dd[0] = xd[it].x; dd[1] = xd[it].y; dd[2] = xd[it].z; dd[3] = xd[it].w;
+                *reinterpret_cast<float4 *>(sm.S + c * LDV + v) = xs[it];
+                *reinterpret_cast<float4 *>(sm.dSn + c * LDV + v) = xd[it];
             }
             const int v = q4 * 4;
-            float *du = sm.U + r * LDV + v, *dy = sm.Y + r * LDV + v, *dr = sm.R + r * LDV + v;
-            du[0] = xu.x; du[1] = xu.y; du[2] = xu.z; du[3] = xu.w;
-            dy[0] = xy.x; dy[1] = xy.y; dy[2] = xy.z; dy[3] = xy.w;
-            if constexpr (!COMPUTE_R) { dr[0] = xr.x; dr[1] = xr.y; dr[2] = xr.z; dr[3] = xr.w; }
+            *reinterpret_cast<float4 *>(sm.U + r * LDV + v) = xu;
+            *reinterpret_cast<float4 *>(sm.Y + r * LDV + v) = xy;
+            if constexpr (!COMPUTE_R) *reinterpret_cast<float4 *>(sm.R + r * LDV + v) = xr;
         }
         __syncthreads();
-#pragma unroll 4
-        for (int v = 0; v < DVB; ++v) {
-            float o[4], y[4], u[4], sv[4], dv[4], ui[2];
+        // float4 steps along the value axis: the thread's rows of dO, Y, U are broadcasts, the
+        // column rows of S, dS', U fall in 8 distinct bank groups per phase (row stride 9 groups);
+        // two loops, so that fewer operands are live at once
+#pragma unroll 2
+        for (int v = 0; v < DVB; v += 4) {
+            float4 o[4], y[4];
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
-                o[x] = sm.dO[(4 * rb + x) * LDV + v];
-                y[x] = sm.Y[(4 * rb + x) * LDV + v];
-                u[x] = sm.U[(4 * rb + x) * LDV + v];
-                sv[x] = sm.S[(cb + 32 * x) * LDV + v];
-                dv[x] = sm.dSn[(cb + 32 * x) * LDV + v];
+                o[x] = *reinterpret_cast<const float4 *>(sm.dO + (4 * rb + x) * LDV + v);
+                y[x] = *reinterpret_cast<const float4 *>(sm.Y + (4 * rb + x) * LDV + v);
             }
-            ui[0] = sm.U[cb * LDV + v];
-            ui[1] = sm.U[(cb + 32) * LDV + v];
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
+            for (int z = 0; z < 4; ++z) {
+                const float4 sv = *reinterpret_cast<const float4 *>(sm.S + (cb + 32 * z) * LDV + v);
 #pragma unroll
-                for (int z = 0; z < 4; ++z) {
-                    aQ[x][z] += o[x] * sv[z];
-                    aY[x][z] += y[x] * sv[z];
-                    aE[x][z] += u[x] * dv[z];
-                }
+                for (int x = 0; x < 4; ++x) { aQ[x][z] = dot4acc(aQ[x][z], o[x], sv); aY[x][z] = dot4acc(aY[x][z], y[x], sv); }
+            }
 #pragma unroll
-                for (int z = 0; z < 2; ++z) {
-                    aM[x][z] += o[x] * ui[z];
-                    aA[x][z] += y[x] * ui[z];
-                }
+            for (int z = 0; z < 2; ++z) {
+                const float4 ui = *reinterpret_cast<const float4 *>(sm.U + (cb + 32 * z) * LDV + v);
+#pragma unroll
+                for (int x = 0; x < 4; ++x) { aM[x][z] = dot4acc(aM[x][z], o[x], ui); aA[x][z] = dot4acc(aA[x][z], y[x], ui); }
+            }
+        }
+#pragma unroll 2
+        for (int v = 0; v < DVB; v += 4) {
+            float4 u[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) u[x] = *reinterpret_cast<const float4 *>(sm.U + (4 * rb + x) * LDV + v);
+#pragma unroll
+            for (int z = 0; z < 4; ++z) {
+                const float4 dv = *reinterpret_cast<const float4 *>(sm.dSn + (cb + 32 * z) * LDV + v);
+#pragma unroll
+                for (int x = 0; x < 4; ++x) aE[x][z] = dot4acc(aE[x][z], u[x], dv);
             }
         }
         if (tid < DK) {
-            for (int v = 0; v < DVB; ++v) dgam_acc += sm.dSn[tid * LDV + v] * sm.S[tid * LDV + v];
+#pragma unroll
+            for (int v = 0; v < DVB; v += 4)
+                dgam_acc = dot4acc(dgam_acc, *reinterpret_cast<const float4 *>(sm.dSn + tid * LDV + v),
+                                   *reinterpret_cast<const float4 *>(sm.S + tid * LDV + v));
         } else if (tid < DK + C) {
             const int r = tid - DK;
-            for (int v = 0; v < DVB; ++v) ry_acc += sm.R[r * LDV + v] * sm.Y[r * LDV + v];
+#pragma unroll
+            for (int v = 0; v < DVB; v += 4)
+                ry_acc = dot4acc(ry_acc, *reinterpret_cast<const float4 *>(sm.R + r * LDV + v),
+                                 *reinterpret_cast<const float4 *>(sm.Y + r * LDV + v));
         }
     }
     __syncthreads();                                   // the value blocks are dead from here on
-    float *dM = sm.S;                                  // 64 x LDC, aliases the staging area
-    float *dP = sm.S + C * LDC;
+    // dM, dP and their transposes, 64 x LDC4 each, in the staging area
+    float *dM = sm.S, *dP = dM + C * LDC4, *dMT = dP + C * LDC4, *dPT = dMT + C * LDC4;
     if (tid < DK) sm.dgam[tid] = dgam_acc;
     else if (tid < DK + C) sm.ry[tid - DK] = ry_acc;
     {
@@ -553,8 +602,11 @@ chunk_bwd_local_kernel(BwdArgs a)
             for (int z = 0; z < 2; ++z) {
                 const int i = cb + 32 * z;
                 const float da = (i < r) ? -aA[x][z] : 0.f;
-                dM[r * LDC + i] = (i <= r) ? aM[x][z] : 0.f;
-                dP[r * LDC + i] = sm.beta[r] * da;
+                const float mv = (i <= r) ? aM[x][z] : 0.f, pv = sm.beta[r] * da;
+                dM[r * LDC4 + i] = mv;
+                dMT[i * LDC4 + r] = mv;
+                dP[r * LDC4 + i] = pv;
+                dPT[i * LDC4 + r] = pv;
                 part[x] += da * sm.P[r * LDC + i];
             }
             if constexpr (COMPUTE_R) {        // - sum_c Kt_rc (Y S^T)_rc over this thread's 4 columns
@@ -597,16 +649,20 @@ chunk_bwd_local_kernel(BwdArgs a)
                 qt[z] = sm.Qt[i * LD + cb + 32 * z];
                 kt[z] = sm.Kt[i * LD + cb + 32 * z];
             }
+            // the thread's 4 rows r of column i (dQt, dKt) and of row i (dKh): four broadcasts
+            const float4 m_c = *reinterpret_cast<const float4 *>(dMT + i * LDC4 + 4 * rb);   // dM[r][i]
+            const float4 p_c = *reinterpret_cast<const float4 *>(dPT + i * LDC4 + 4 * rb);   // dP[r][i]
+            const float4 m_r = *reinterpret_cast<const float4 *>(dM + i * LDC4 + 4 * rb);    // dM[i][r]
+            const float4 p_r = *reinterpret_cast<const float4 *>(dP + i * LDC4 + 4 * rb);    // dP[i][r]
+            const float m_ri[4] = {m_c.x, m_c.y, m_c.z, m_c.w}, p_ri[4] = {p_c.x, p_c.y, p_c.z, p_c.w};
+            const float m_ir[4] = {m_r.x, m_r.y, m_r.z, m_r.w}, p_ir[4] = {p_r.x, p_r.y, p_r.z, p_r.w};
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
-                const int r = 4 * rb + x;
-                const float m_ri = dM[r * LDC + i], p_ri = dP[r * LDC + i];     // row r: dQt, dKt
-                const float m_ir = dM[i * LDC + r], p_ir = dP[i * LDC + r];     // column r: dKh
 #pragma unroll
                 for (int z = 0; z < 4; ++z) {
-                    dQ[x][z] += m_ri * kh[z];
-                    dKt[x][z] += p_ri * kh[z];
-                    dKh[x][z] += m_ir * qt[z] + p_ir * kt[z];
+                    dQ[x][z] += m_ri[x] * kh[z];
+                    dKt[x][z] += p_ri[x] * kh[z];
+                    dKh[x][z] += m_ir[x] * qt[z] + p_ir[x] * kt[z];
                 }
             }
         }
