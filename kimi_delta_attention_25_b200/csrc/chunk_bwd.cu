@@ -278,6 +278,7 @@ struct RscanSmem {
     RscanBuf buf[2];
     float dS[DK * DVB];
     float Y[C * DVB];
+    float Yp[C * DVB];       // the upper key-channel half's part of Kp dS'
 };
 
 // acc + a.x b.x + a.y b.y + a.z b.z + a.w b.w, added in that order
@@ -354,30 +355,74 @@ chunk_bwd_rscan_kernel(BwdArgs a)
         fp32c::store_block32<NT_RS>(a.ck_dS + rec * kBwdStateFloats + j0, DK, sm.dS, DK, tid);
         __syncthreads();
         const RscanBuf &B = sm.buf[b];
-        {   // Y = Y0 + Kp dS': thread -> row tid / 4, 8 columns
-            const int r = tid / 4, jg = (tid % 4) * 8;
-            float acc[8];
+        {   // Y = Y0 + Kp dS', the key-channel sum in two halves (warps 0-3: c < 64, warps 4-7: the
+            // rest, whose part goes through Yp): thread -> rows rq + 16 x (x < 4), columns 4 jq .. + 3.
+            // Per channel a warp reads 4 Kp values (4 rows in 4 banks) and one 128-byte row of dS'.
+            const int g = tid >> 7, t = tid & 127, rq = t >> 3, jq = t & 7;
+            float acc[4][4];
 #pragma unroll
-            for (int x = 0; x < 8; ++x) acc[x] = B.Y0[r * DVB + jg + x];
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
 #pragma unroll 4
-            for (int c = 0; c < DK; ++c) fp32c::axpy<8>(acc, B.Kp[r * LDP + c], sm.dS + c * DVB + jg);
+            for (int c = 64 * g; c < 64 * g + 64; ++c) {
+                const float4 d4 = *reinterpret_cast<const float4 *>(sm.dS + c * DVB + 4 * jq);
 #pragma unroll
-            for (int x = 0; x < 8; ++x) sm.Y[r * DVB + jg + x] = acc[x];
+                for (int x = 0; x < 4; ++x) {
+                    const float kp = B.Kp[(rq + 16 * x) * LDP + c];
+                    acc[x][0] += kp * d4.x; acc[x][1] += kp * d4.y; acc[x][2] += kp * d4.z; acc[x][3] += kp * d4.w;
+                }
+            }
+            if (g == 1) {
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+                    *reinterpret_cast<float4 *>(sm.Yp + (rq + 16 * x) * DVB + 4 * jq) =
+                        make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
+            }
+            __syncthreads();
+            if (g == 0) {
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int o = (rq + 16 * x) * DVB + 4 * jq;
+                    const float4 y0 = *reinterpret_cast<const float4 *>(B.Y0 + o);
+                    const float4 yp = *reinterpret_cast<const float4 *>(sm.Yp + o);
+                    *reinterpret_cast<float4 *>(sm.Y + o) =
+                        make_float4(y0.x + (acc[x][0] + yp.x), y0.y + (acc[x][1] + yp.y),
+                                    y0.z + (acc[x][2] + yp.z), y0.w + (acc[x][3] + yp.w));
+                }
+            }
         }
         __syncthreads();
         fp32c::store_block32<NT_RS>(a.ck_Y + rec * kBwdRowsFloats + j0, DK, sm.Y, C, tid);
         fp32c::store_block32<NT_RS>(a.dv + ((size_t)s * H + h) * DK + j0, (size_t)H * DK, sm.Y, L, tid, B.gb + DK);
-        {   // dS = Diag(gamma) dS' + G0 - Bk^T Y: thread -> key channel tid / 2, 16 columns
-            const int c = tid / 2, jh = (tid % 2) * 16;
-            const float gm = B.gb[c];
-            float acc[16];
+        {   // dS = Diag(gamma) dS' + G0 - Bk^T Y: thread -> key channels 4 cq .. + 3, columns 4 jq .. + 3
+            const int cq = tid >> 3, jq = tid & 7;
+            float acc[4][4];
 #pragma unroll
-            for (int x = 0; x < 16; ++x) acc[x] = gm * sm.dS[c * DVB + jh + x] + B.G0[c * DVB + jh + x];
+            for (int x = 0; x < 4; ++x) {
+                const int o = (4 * cq + x) * DVB + 4 * jq;
+                const float gm = B.gb[4 * cq + x];
+                const float4 d4 = *reinterpret_cast<const float4 *>(sm.dS + o);
+                const float4 g4 = *reinterpret_cast<const float4 *>(B.G0 + o);
+                acc[x][0] = gm * d4.x + g4.x; acc[x][1] = gm * d4.y + g4.y;
+                acc[x][2] = gm * d4.z + g4.z; acc[x][3] = gm * d4.w + g4.w;
+            }
 #pragma unroll 4
-            for (int r = 0; r < C; ++r) fp32c::axpy<16>(acc, -B.Bk[r * LDP + c], sm.Y + r * DVB + jh);
+            for (int r = 0; r < C; ++r) {
+                const float4 bk = *reinterpret_cast<const float4 *>(B.Bk + r * LDP + 4 * cq);
+                const float4 y4 = *reinterpret_cast<const float4 *>(sm.Y + r * DVB + 4 * jq);
+                const float b4[4] = {bk.x, bk.y, bk.z, bk.w};
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    acc[x][0] -= b4[x] * y4.x; acc[x][1] -= b4[x] * y4.y;
+                    acc[x][2] -= b4[x] * y4.z; acc[x][3] -= b4[x] * y4.w;
+                }
+            }
             __syncthreads();              // every thread has read dS' (Y step and this one)
 #pragma unroll
-            for (int x = 0; x < 16; ++x) sm.dS[c * DVB + jh + x] = acc[x];
+            for (int x = 0; x < 4; ++x)
+                *reinterpret_cast<float4 *>(sm.dS + (4 * cq + x) * DVB + 4 * jq) =
+                    make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
         }
     }
     cp_async_wait0();
