@@ -239,8 +239,11 @@ kda_status_t chunk_bwd_impl(unsigned phases, const void *q, const void *k, const
         if (tc) {
             static_assert(kPrepBlockBytes <= (kBwdStateFloats + kBwdRowsFloats) * sizeof(float),
                           "prepared blocks fit the dS' and R areas");
-            e = launch_chunk_prep(a, (unsigned char *)ck_dS, (int)n_slots, st);
-            if (e == cudaSuccess) e = launch_chunk_scan_records(a, (const unsigned char *)ck_dS, (int)n_slots, st);
+            // the two passes as the forward runs them (pipelined over token ranges when few chains);
+            // the state carried between ranges goes to the G0 area, written only later
+            a.scratch = ck_dS;
+            a.S_final = ck_G0;
+            e = run_prefill_bf16(a, KDA_F32, st, nullptr, nullptr, /*records=*/true);
         } else {
             a.ck_R = ck_R;
             e = launch_chunk_fp32(a, dtype, KDA_F32, st);

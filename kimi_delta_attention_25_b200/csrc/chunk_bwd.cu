@@ -109,73 +109,75 @@ chunk_bwd_prep_kernel(BwdArgs a)
         }
     }
     __syncthreads();
-    {   // A = StrictLower(diag(beta) Kt Kh^T) (threads 0-255), M = tril(Qt Kh^T) (256-511): thread ->
-        // rows rb + 16 x, columns ib + 16 y (x, y < 4), float4 steps along the key channels, so that
-        // the 8 lanes of a shared-memory phase read one X row (a broadcast) and 8 Kh rows that fall
-        // in 8 distinct bank groups (a row stride of 33 groups)
-        const bool isM = tid >= 256;
-        const int t = tid & 255, rb = t >> 4, ib = t & 15;
-        const float *X = isM ? sm.Qt : sm.Kt;
-        float acc[4][4];
+    // G0 (threads 0-255) beside A and M (threads 256-511); per step of the sum a thread tile of
+    // a x b outputs reads a + b values, so the larger tiles take fewer shared-memory wavefronts
+    if (tid < 256) {
+        // G0 = Qt^T dO: thread -> key channels 8 cq .. + 7, value columns 4 jq .. + 3 and 64 + 4 jq ..
+        // + 3 (cq = tid / 16, jq = tid % 16: the 8 lanes of a phase read 8 distinct bank groups of dO)
+        const int cq = tid >> 4, jq = tid & 15;
+        float acc[8][8];
 #pragma unroll
-        for (int x = 0; x < 4; ++x)
-#pragma unroll
-            for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
-#pragma unroll 2
-        for (int c = 0; c < DK; c += 4) {
-            float4 xr[4], kh[4];
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                xr[x] = *reinterpret_cast<const float4 *>(X + (rb + 16 * x) * LDB + c);
-                kh[x] = *reinterpret_cast<const float4 *>(sm.Kh + (ib + 16 * x) * LDB + c);
-            }
-#pragma unroll
-            for (int x = 0; x < 4; ++x)
-#pragma unroll
-                for (int y = 0; y < 4; ++y) {
-                    acc[x][y] += xr[x].x * kh[y].x;
-                    acc[x][y] += xr[x].y * kh[y].y;
-                    acc[x][y] += xr[x].z * kh[y].z;
-                    acc[x][y] += xr[x].w * kh[y].w;
-                }
-        }
-#pragma unroll
-        for (int x = 0; x < 4; ++x)
-#pragma unroll
-            for (int y = 0; y < 4; ++y) {
-                const int r = rb + 16 * x, i = ib + 16 * y;
-                if (isM) sm.M[r * LDC + i] = (i <= r) ? acc[x][y] : 0.f;
-                else sm.A[r * LDC + i] = (i < r) ? sm.beta[r] * acc[x][y] : 0.f;
-            }
-    }
-    __syncthreads();
-    {   // G0 = Qt^T dO: thread -> key channels 4 (tid / 16) .. + 3, value columns j0 .. + 3 and
-        // 64 + j0 .. + 3 with j0 = 4 (tid % 16) (8 lanes of a phase: 8 distinct bank groups)
-        const int c0 = 4 * (tid >> 4), j0 = 4 * (tid & 15);
-        float acc[4][8];
-#pragma unroll
-        for (int x = 0; x < 4; ++x)
+        for (int x = 0; x < 8; ++x)
 #pragma unroll
             for (int y = 0; y < 8; ++y) acc[x][y] = 0.f;
-#pragma unroll 4
+#pragma unroll 2
         for (int r = 0; r < C; ++r) {
-            const float4 q4 = *reinterpret_cast<const float4 *>(sm.Qt + r * LDB + c0);
-            const float4 o0 = *reinterpret_cast<const float4 *>(sm.dO + r * LDB + j0);
-            const float4 o1 = *reinterpret_cast<const float4 *>(sm.dO + r * LDB + 64 + j0);
-            const float qt[4] = {q4.x, q4.y, q4.z, q4.w};
+            const float4 qa = *reinterpret_cast<const float4 *>(sm.Qt + r * LDB + 8 * cq);
+            const float4 qb = *reinterpret_cast<const float4 *>(sm.Qt + r * LDB + 8 * cq + 4);
+            const float4 o0 = *reinterpret_cast<const float4 *>(sm.dO + r * LDB + 4 * jq);
+            const float4 o1 = *reinterpret_cast<const float4 *>(sm.dO + r * LDB + 64 + 4 * jq);
+            const float qt[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
             const float o[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
 #pragma unroll
-            for (int x = 0; x < 4; ++x)
+            for (int x = 0; x < 8; ++x)
 #pragma unroll
                 for (int y = 0; y < 8; ++y) acc[x][y] += qt[x] * o[y];
         }
         float *g0 = a.ck_G0 + rec * kBwdStateFloats;
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            float *dst = g0 + (size_t)(c0 + x) * DK + j0;
+        for (int x = 0; x < 8; ++x) {
+            float *dst = g0 + (size_t)(8 * cq + x) * DK + 4 * jq;
             *reinterpret_cast<float4 *>(dst) = make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
             *reinterpret_cast<float4 *>(dst + 64) = make_float4(acc[x][4], acc[x][5], acc[x][6], acc[x][7]);
         }
+    } else {
+        // [A; M] from the rows of [Kt; Qt] times Kh^T, A = StrictLower(diag(beta) Kt Kh^T),
+        // M = tril(Qt Kh^T): thread -> rows rb + 16 x of [Kt; Qt] (x < 8: Kt for x < 4, Qt after),
+        // columns ib + 16 y (y < 4); float4 steps along the key channels, so that the 8 lanes of a
+        // phase read one X row (a broadcast) and 8 Kh rows in 8 distinct bank groups (a row stride
+        // of 33 groups)
+        const int t = tid - 256, rb = t >> 4, ib = t & 15;
+        float acc[8][4];
+#pragma unroll
+        for (int x = 0; x < 8; ++x)
+#pragma unroll
+            for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < DK; c += 4) {
+            float4 kh[4];
+#pragma unroll
+            for (int y = 0; y < 4; ++y) kh[y] = *reinterpret_cast<const float4 *>(sm.Kh + (ib + 16 * y) * LDB + c);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+                const float *X = x < 4 ? sm.Kt : sm.Qt;
+                const float4 xr = *reinterpret_cast<const float4 *>(X + (rb + 16 * (x & 3)) * LDB + c);
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    acc[x][y] += xr.x * kh[y].x;
+                    acc[x][y] += xr.y * kh[y].y;
+                    acc[x][y] += xr.z * kh[y].z;
+                    acc[x][y] += xr.w * kh[y].w;
+                }
+            }
+        }
+#pragma unroll
+        for (int x = 0; x < 8; ++x)
+#pragma unroll
+            for (int y = 0; y < 4; ++y) {
+                const int r = rb + 16 * (x & 3), i = ib + 16 * y;
+                if (x >= 4) sm.M[r * LDC + i] = (i <= r) ? acc[x][y] : 0.f;
+                else sm.A[r * LDC + i] = (i < r) ? sm.beta[r] * acc[x][y] : 0.f;
+            }
     }
     __syncthreads();                      // Qt is dead
     {   // M^T dO into Qt's place: thread -> rows 4 (tid / 32) .. + 3, columns 4 (tid % 32) .. + 3

@@ -688,10 +688,11 @@ cudaError_t launch_chunk_scan(const PrefillArgs &a, const unsigned char *ws, int
 }
 
 cudaError_t launch_chunk_scan_records(const PrefillArgs &a, const unsigned char *ws, int n_slots,
-                                      cudaStream_t stream)
+                                      cudaStream_t stream, long long slot_lo, long long slot_hi)
 {
     if (!a.ck_S || !a.ck_U) return cudaErrorInvalidValue;
-    return launch_typed<float, false, true>(a, ws, n_slots, nullptr, 0, n_slots, stream);
+    if (slot_hi < 0) slot_hi = n_slots;
+    return launch_typed<float, false, true>(a, ws, n_slots, nullptr, slot_lo, slot_hi, stream);
 }
 
 }  // namespace kda

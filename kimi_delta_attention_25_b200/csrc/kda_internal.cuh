@@ -187,21 +187,23 @@ cudaError_t launch_chunk_scan(const PrefillArgs &a, const unsigned char *ws, int
                               long long slot_lo = 0, long long slot_hi = -1);
 
 // The same scan writing the backward pass's forward records (a.ck_S: the state entering every chunk,
-// a.ck_U: each chunk's U; both per (head, chunk slot)) instead of outputs.
+// a.ck_U: each chunk's U; both per (head, chunk slot)) instead of outputs; the same slot ranges.
 cudaError_t launch_chunk_scan_records(const PrefillArgs &a, const unsigned char *ws, int n_slots,
-                                      cudaStream_t stream);
+                                      cudaStream_t stream, long long slot_lo = 0, long long slot_hi = -1);
 
 // The bf16 prefill as kda_chunk_fwd runs it (prefill.cu): with at most kPipeMaxChains (sequence,
 // head) chains and enough chunk slots, a pipeline over token ranges (scan of one range beside the
 // preparation of the next ones), else the two passes one after the other. The pipeline carries the
-// state between ranges in S_final, or in prefill_carry_bytes of workspace after the blocks.
+// state between ranges in S_final, or in prefill_carry_bytes of workspace after the blocks. With
+// records, the scans write the backward's forward records (launch_chunk_scan_records) instead of
+// outputs.
 constexpr int kPipeMaxChains = 64;
 constexpr int kPipeMinSlotsPerRange = 32;
 bool prefill_pipelined(long long tokens, int H, int N);
 size_t prefill_carry_bytes(long long tokens, int H, int N);
 int prefill_launches(long long tokens, int H, int N);   // kernels run_prefill_bf16 launches
 cudaError_t run_prefill_bf16(const PrefillArgs &a, kda_dtype_t out_dtype, cudaStream_t stream,
-                             const GateArgs *gate, const NormArgs *norm);
+                             const GateArgs *gate, const NormArgs *norm, bool records = false);
 
 // Backward pass (chunk_bwd.cu). Gradient pointers and the records of the forward kernel.
 struct BwdArgs {

@@ -51,6 +51,9 @@ PipeStreams *pipe_streams()
 }
 
 // token ranges of the pipeline over n_slots chunk slots
+// chunk slots of a prefill's workspace
+int n_slots_of(const PrefillArgs &a) { return (int)prep_slots((long long)a.B * a.T, a.N); }
+
 int pipe_ranges(int n_slots)
 {
     const int R = n_slots / kPipeMinSlotsPerRange;
@@ -75,14 +78,18 @@ size_t prefill_carry_bytes(long long tokens, int H, int N)
 }
 
 cudaError_t run_prefill_bf16(const PrefillArgs &a_in, kda_dtype_t out_dtype, cudaStream_t st,
-                             const GateArgs *gate, const NormArgs *norm)
+                             const GateArgs *gate, const NormArgs *norm, bool records)
 {
+    auto scan = [&](const PrefillArgs &a, cudaStream_t s, long long lo, long long hi) {
+        return records ? launch_chunk_scan_records(a, (const unsigned char *)a.scratch, n_slots_of(a), s, lo, hi)
+                       : launch_chunk_scan(a, (const unsigned char *)a.scratch, n_slots_of(a), out_dtype, s, norm, lo, hi);
+    };
     const long long tokens = (long long)a_in.B * a_in.T;
     const int n_slots = (int)prep_slots(tokens, a_in.N);
     unsigned char *blocks = (unsigned char *)a_in.scratch;
     if (!prefill_pipelined(tokens, a_in.H, a_in.N)) {
         cudaError_t e = launch_chunk_prep(a_in, blocks, n_slots, st, gate);
-        if (e == cudaSuccess) e = launch_chunk_scan(a_in, blocks, n_slots, out_dtype, st, norm, 0, n_slots);
+        if (e == cudaSuccess) e = scan(a_in, st, 0, n_slots);
         return e;
     }
     PrefillArgs a = a_in;
@@ -111,8 +118,7 @@ cudaError_t run_prefill_bf16(const PrefillArgs &a_in, kda_dtype_t out_dtype, cud
     }
     for (int r = 0; r < R && e == cudaSuccess; ++r) {
         e = cudaStreamWaitEvent(ps->scan, ps->prepped[r], 0);
-        if (e == cudaSuccess)
-            e = launch_chunk_scan(a, blocks, n_slots, out_dtype, ps->scan, norm, bounds[r], bounds[r + 1]);
+        if (e == cudaSuccess) e = scan(a, ps->scan, bounds[r], bounds[r + 1]);
     }
     // join: the caller's stream waits for both library streams (on an error too, so that nothing the
     // call enqueued can still run unordered with the caller's later work)

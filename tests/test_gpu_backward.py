@@ -86,6 +86,21 @@ def test_varlen_with_empty_sequences(dtype):
     _run(d, TOL[K.to_dtype(dtype)])
 
 
+def test_packed_sequences_across_token_ranges():
+    """Few (sequence, head) chains and enough chunks: the forward records come from the two passes
+    pipelined over token ranges, with sequences that start, end or lie inside a range and the state
+    carried between ranges; gradients against the oracle on two of the four heads."""
+    lens = [1000, 0, 3000, 64, 5000, 70]
+    cu = torch.tensor(np.cumsum([0] + lens), dtype=torch.int32)
+    w = K.Workload("bwd_packed", B=1, T=int(cu[-1]), H=4, dtype="bf16", s0_std=0.1)
+    d = K.make_prefill(w, seed=39)
+    d["S0"] = 0.1 * torch.randn(len(lens), 4, 128, 128, generator=torch.Generator().manual_seed(6))
+    d["cu_seqlens"] = cu
+    d = _with_output_grads(d, seed=12)
+    assert kda.chunk_fwd_kernel_launches(1, int(cu[-1]), 4, len(lens), torch.bfloat16) > 2   # pipelined
+    _run(d, TOL[torch.bfloat16], heads=[0, 3])
+
+
 def test_zero_state_and_no_state_gradients():
     w = K.Workload("bwd_nostate", B=1, T=200, H=2, dtype="bf16")
     d = _with_output_grads(K.make_prefill(w, seed=34), seed=5, with_dSf=False)
