@@ -463,6 +463,7 @@ struct LocalSmem {
 };
 static_assert((NT_LOC / 32) * DK <= C * LDV, "per-warp column sums must fit the dO block");
 static_assert(4 * C * LDC4 <= 2 * DK * LDV + 4 * C * LDV, "dM, dP and their transposes must fit the staging area");
+static_assert((NT_LOC / DK) * 16 == C, "the reverse sum over rows takes quarters of 16 rows");
 
 // COMPUTE_R: no R record (the forward records came from the bf16 state scan, which holds S and U
 // but not R). R enters only dbeta, through sum_v R_rv Y_rv = sum_v V_rv Y_rv - sum_c Kt_rc (Y S^T)_rc;
@@ -487,11 +488,33 @@ chunk_bwd_local_kernel(BwdArgs a)
     const T *q = (const T *)a.q;
     const T *k = (const T *)a.k;
     const T *dout = (const T *)a.dout;
+    const float *gS = a.ck_S + rec * kBwdStateFloats;
+    const float *gdS = a.ck_dS + rec * kBwdStateFloats;
+    const float *gU = a.ck_U + rec * kBwdRowsFloats;
+    const float *gY = a.ck_Y + rec * kBwdRowsFloats;
+    const float *gR = COMPUTE_R ? nullptr : a.ck_R + rec * kBwdRowsFloats;
+    // asks L2 for the rows of value block jp (32 columns) ahead of its loads: one row segment per
+    // thread (128 of S, 128 of dS', 64 each of U, Y, dO and V or R; token rows past L skipped)
+    auto prefetch_block = [&](int jp) {
+        const void *ptr = nullptr;
+        if (tid < 128) ptr = gS + (size_t)tid * DK + jp;
+        else if (tid < 256) ptr = gdS + (size_t)(tid - 128) * DK + jp;
+        else if (tid < 320) ptr = gU + (size_t)(tid - 256) * DK + jp;
+        else if (tid < 384) ptr = gY + (size_t)(tid - 320) * DK + jp;
+        else if (tid < 448) {
+            if (tid - 384 < L) ptr = dout + ((size_t)(s + tid - 384) * H + h) * DK + jp;
+        } else if (tid - 448 < L) {
+            if constexpr (COMPUTE_R) ptr = (const T *)a.v + ((size_t)(s + tid - 448) * H + h) * DK + jp;
+            else ptr = gR + (size_t)(tid - 448) * DK + jp;
+        }
+        if (ptr) asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+    };
 
     // ---- load q, k, log_alpha (zero past L), beta; then g = cumsum(log_alpha) in row parts
     fp32c::load_rows<T, NT_LOC, DK>(sm.Kt, LD, k, s, L, H, h, 0, tid);
     fp32c::load_rows<T, NT_LOC, DK>(sm.Qt, LD, q, s, L, H, h, 0, tid);
     fp32c::load_rows<float, NT_LOC, DK>(sm.E, LD, a.log_alpha, s, L, H, h, 0, tid);
+    prefetch_block(0);
     if (tid < C) sm.beta[tid] = (tid < L) ? a.beta[(size_t)(s + tid) * H + h] : 0.f;
     if (tid < DK) sm.dgam[tid] = 0.f;
     if (tid < C) sm.ry[tid] = 0.f;
@@ -548,11 +571,6 @@ chunk_bwd_local_kernel(BwdArgs a)
         for (int y = 0; y < 4; ++y) { aQ[x][y] = 0.f; aY[x][y] = 0.f; aE[x][y] = 0.f; }
         aM[x][0] = aM[x][1] = aA[x][0] = aA[x][1] = 0.f;
     }
-    const float *gS = a.ck_S + rec * kBwdStateFloats;
-    const float *gdS = a.ck_dS + rec * kBwdStateFloats;
-    const float *gU = a.ck_U + rec * kBwdRowsFloats;
-    const float *gY = a.ck_Y + rec * kBwdRowsFloats;
-    const float *gR = COMPUTE_R ? nullptr : a.ck_R + rec * kBwdRowsFloats;
     float dgam_acc = 0.f, ry_acc = 0.f;
     for (int j0 = 0; j0 < DK; j0 += DVB) {
         __syncthreads();
@@ -584,6 +602,7 @@ chunk_bwd_local_kernel(BwdArgs a)
             if constexpr (!COMPUTE_R) *reinterpret_cast<float4 *>(sm.R + r * LDV + v) = xr;
         }
         __syncthreads();
+        if (j0 + DVB < DK) prefetch_block(j0 + DVB);
         // float4 steps along the value axis: the thread's rows of dO, Y, U are broadcasts, the
         // column rows of S, dS', U fall in 8 distinct bank groups per phase (row stride 9 groups);
         // two loops, so that fewer operands are live at once
@@ -743,12 +762,21 @@ chunk_bwd_local_kernel(BwdArgs a)
     __syncthreads();
     // ---- dlog_alpha: reverse cumulative sum over rows, the last row also carrying the terms of
     //      g_{L-1} (through Ke and gamma)
-    if (tid < DK) {
-        const int c = tid;
-        float dgl = 0.f;
-        for (int w = 0; w < NT_LOC / 32; ++w) dgl += sm.dO[w * DK + c];
-        float run = dgl + sm.dgam[c] * sm.gam[c];
-        for (int r = C - 1; r >= 0; --r) {
+    //      on all threads: 4 quarters of 16 rows per channel, each quarter's sum first
+    {
+        const int c = tid & (DK - 1), qd = tid / DK;
+        float part = 0.f;
+#pragma unroll
+        for (int r = 16 * qd; r < 16 * qd + 16; ++r) part += sm.Kh[r * LD + c];
+        float *qsum = sm.S;                            // free again (it held dM)
+        qsum[qd * DK + c] = part;
+        float run = 0.f;
+        for (int w = 0; w < NT_LOC / 32; ++w) run += sm.dO[w * DK + c];
+        run += sm.dgam[c] * sm.gam[c];
+        __syncthreads();
+        for (int q2 = NT_LOC / DK - 1; q2 > qd; --q2) run += qsum[q2 * DK + c];
+#pragma unroll 4
+        for (int r = 16 * qd + 15; r >= 16 * qd; --r) {
             run += sm.Kh[r * LD + c];
             if (r < L) a.dlog_alpha[((size_t)(s + r) * H + h) * DK + c] = run;
         }
