@@ -170,7 +170,7 @@ kda_status_t kda_chunk_scan(const void *v, const float *S0, const int32_t *cu_se
  *   dS0        [N, H, dk, dv] float32 (written: dL/dS0), or NULL (not computed).
  *   workspace  device buffer of kda_chunk_bwd_workspace_size(...) bytes (fp32 records
  *              of the forward and of the reverse sweep and the reverse sweep's prepared
- *              operands: 385 KiB per chunk slot and head, see kda_chunk_fwd_workspace_size
+ *              operands: 401 KiB per chunk slot and head, see kda_chunk_fwd_workspace_size
  *              for chunk slots). Its status word is
  *              cleared by this call; cu_seqlens is checked on the device as for
  *              kda_chunk_fwd.

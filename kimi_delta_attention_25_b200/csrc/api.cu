@@ -165,8 +165,10 @@ int kda_chunk_fwd_kernel_launches(int B, int T, int H, int N, kda_dtype_t dtype)
 size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int N, int dk, int dv)
 {
     if (B < 0 || T < 0 || H <= 0 || N < 0 || dk != kHeadDim || dv != kHeadDim) return 0;
-    // S, dS'; R, U, Y; then the reverse scan's prepared operands Kp, Bk, Y0; G0; gamma and beta
-    const size_t per = 2 * kBwdStateFloats + 3 * kBwdRowsFloats + 3 * kBwdRowsFloats + kBwdStateFloats + 256;
+    // S, dS'; R, U, Y; then the reverse scan's prepared operands Kp, Bk, Y0; G0; gamma and beta;
+    // P for the per-chunk kernel
+    const size_t per = 2 * kBwdStateFloats + 3 * kBwdRowsFloats + 3 * kBwdRowsFloats + kBwdStateFloats + 256 +
+                       kBwdTriFloats;
     return kStatusBytes + (size_t)H * (size_t)prep_slots((long long)B * T, N) * per * sizeof(float);
 }
 
@@ -226,6 +228,7 @@ kda_status_t chunk_bwd_impl(unsigned phases, const void *q, const void *k, const
     float *ck_Y0 = ck_Bk + hs * kBwdRowsFloats;
     float *ck_G0 = ck_Y0 + hs * kBwdRowsFloats;
     float *ck_gb = ck_G0 + hs * kBwdStateFloats;
+    float *ck_P = ck_gb + hs * 256;
 
     cudaError_t e = cudaSuccess;
     // bf16 inputs take the forward records from the tensor-core passes, which write S and U but not
@@ -255,7 +258,7 @@ kda_status_t chunk_bwd_impl(unsigned phases, const void *q, const void *k, const
     b.cu_seqlens = cu_seqlens;
     b.dq = dq; b.dk = dk_out; b.dv = dv_out; b.dlog_alpha = dlog_alpha; b.dbeta = dbeta; b.dS0 = dS0;
     b.ck_S = ck_S; b.ck_R = tc ? nullptr : ck_R; b.ck_U = ck_U; b.ck_dS = ck_dS; b.ck_Y = ck_Y;
-    b.ck_Kp = ck_Kp; b.ck_Bk = ck_Bk; b.ck_Y0 = ck_Y0; b.ck_G0 = ck_G0; b.ck_gb = ck_gb;
+    b.ck_Kp = ck_Kp; b.ck_Bk = ck_Bk; b.ck_Y0 = ck_Y0; b.ck_G0 = ck_G0; b.ck_gb = ck_gb; b.ck_P = ck_P;
     b.B = B; b.T = T; b.H = H; b.N = N; b.n_slots = (int)n_slots;
     b.status = (int32_t *)workspace;
     if (e == cudaSuccess && (phases & 2u)) e = launch_chunk_bwd_scan(b, dtype, st);   // 2. reverse scan

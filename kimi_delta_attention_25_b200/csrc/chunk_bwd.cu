@@ -26,7 +26,8 @@
 //     writing S and U, and kernel 3 forms R = V - Kt S itself;
 //  2. the state gradient, chunk by chunk from the end of each sequence, in two kernels:
 //     chunk_bwd_prep_kernel (data-parallel, one CTA per (chunk slot, head)) forms every chunk's
-//     state-independent operands (below), and chunk_bwd_rscan_kernel (one CTA per (sequence,
+//     state-independent operands (below) and the per-chunk kernel's StrictLower(Kt Kh^T), and
+//     chunk_bwd_rscan_kernel (one CTA per (sequence,
 //     head, 32 value columns); the columns are independent) runs the two state products per
 //     chunk and writes dV, dS0, Y and the gradient dS' reaching the end of every chunk;
 //  3. chunk_bwd_local_kernel: everything else, one CTA per (chunk slot, head), no chunk-to-chunk
@@ -170,13 +171,18 @@ chunk_bwd_prep_kernel(BwdArgs a)
                 }
             }
         }
+        float *gP = a.ck_P + rec * kBwdTriFloats;   // P = StrictLower(Kt Kh^T) for the per-chunk kernel
 #pragma unroll
         for (int x = 0; x < 8; ++x)
 #pragma unroll
             for (int y = 0; y < 4; ++y) {
                 const int r = rb + 16 * (x & 3), i = ib + 16 * y;
-                if (x >= 4) sm.M[r * LDC + i] = (i <= r) ? acc[x][y] : 0.f;
-                else sm.A[r * LDC + i] = (i < r) ? sm.beta[r] * acc[x][y] : 0.f;
+                if (x >= 4) {
+                    sm.M[r * LDC + i] = (i <= r) ? acc[x][y] : 0.f;
+                } else {
+                    sm.A[r * LDC + i] = (i < r) ? sm.beta[r] * acc[x][y] : 0.f;
+                    gP[r * C + i] = (i < r) ? acc[x][y] : 0.f;
+                }
             }
     }
     __syncthreads();                      // Qt is dead
@@ -455,7 +461,6 @@ struct LocalSmem {
     float U[C * LDV];
     float Y[C * LDV];
     float R[C * LDV];
-    float P[C * LDC];        // Kt Kh^T (strictly lower part used)
     float beta[C];
     float gam[DK];
     float dgam[DK];
@@ -493,6 +498,7 @@ chunk_bwd_local_kernel(BwdArgs a)
     const float *gU = a.ck_U + rec * kBwdRowsFloats;
     const float *gY = a.ck_Y + rec * kBwdRowsFloats;
     const float *gR = COMPUTE_R ? nullptr : a.ck_R + rec * kBwdRowsFloats;
+    const float *gP = a.ck_P + rec * kBwdTriFloats;   // StrictLower(Kt Kh^T), from the preparation pass
     // asks L2 for the rows of value block jp (32 columns) ahead of its loads: one row segment per
     // thread (128 of S, 128 of dS', 64 each of U, Y, dO and V or R; token rows past L skipped)
     auto prefetch_block = [&](int jp) {
@@ -515,6 +521,7 @@ chunk_bwd_local_kernel(BwdArgs a)
     fp32c::load_rows<T, NT_LOC, DK>(sm.Qt, LD, q, s, L, H, h, 0, tid);
     fp32c::load_rows<float, NT_LOC, DK>(sm.E, LD, a.log_alpha, s, L, H, h, 0, tid);
     prefetch_block(0);
+    if (tid < (int)(kBwdTriFloats / 32)) asm volatile("prefetch.global.L2 [%0];" ::"l"(gP + 32 * tid));
     if (tid < C) sm.beta[tid] = (tid < L) ? a.beta[(size_t)(s + tid) * H + h] : 0.f;
     if (tid < DK) sm.dgam[tid] = 0.f;
     if (tid < C) sm.ry[tid] = 0.f;
@@ -539,29 +546,6 @@ chunk_bwd_local_kernel(BwdArgs a)
 
     // thread tile: rows 4 rb .. 4 rb + 3 (rb = warp), key columns lane + 32 x, token columns lane + 32 x
     const int rb = warp, cb = lane;
-    // ---- P = Kt Kh^T, strictly lower part
-    {
-        float acc[4][2];
-#pragma unroll
-        for (int x = 0; x < 4; ++x) { acc[x][0] = 0.f; acc[x][1] = 0.f; }
-#pragma unroll 2
-        for (int c = 0; c < DK; c += 4) {      // float4 steps: Kt rows broadcast, Kh rows conflict-free
-            float4 kt[4];
-#pragma unroll
-            for (int x = 0; x < 4; ++x) kt[x] = *reinterpret_cast<const float4 *>(sm.Kt + (4 * rb + x) * LD + c);
-            const float4 kh0 = *reinterpret_cast<const float4 *>(sm.Kh + cb * LD + c);
-            const float4 kh1 = *reinterpret_cast<const float4 *>(sm.Kh + (cb + 32) * LD + c);
-#pragma unroll
-            for (int x = 0; x < 4; ++x) { acc[x][0] = dot4acc(acc[x][0], kt[x], kh0); acc[x][1] = dot4acc(acc[x][1], kt[x], kh1); }
-        }
-#pragma unroll
-        for (int x = 0; x < 4; ++x)
-#pragma unroll
-            for (int y = 0; y < 2; ++y) {
-                const int r = 4 * rb + x, i = cb + 32 * y;
-                sm.P[r * LDC + i] = (i < r) ? acc[x][y] : 0.f;
-            }
-    }
 
     // ---- sums over the value axis, 32 columns at a time
     float aQ[4][4], aY[4][4], aE[4][4], aM[4][2], aA[4][2];
@@ -673,7 +657,7 @@ chunk_bwd_local_kernel(BwdArgs a)
                 dMT[i * LDC4 + r] = mv;
                 dP[r * LDC4 + i] = pv;
                 dPT[i * LDC4 + r] = pv;
-                part[x] += da * sm.P[r * LDC + i];
+                part[x] += da * __ldg(gP + r * C + i);
             }
             if constexpr (COMPUTE_R) {        // - sum_c Kt_rc (Y S^T)_rc over this thread's 4 columns
 #pragma unroll
@@ -822,7 +806,7 @@ cudaError_t launch_local_typed(const BwdArgs &a, cudaStream_t stream)
 cudaError_t launch_chunk_bwd_scan(const BwdArgs &a, kda_dtype_t dtype, cudaStream_t stream)
 {
     if (a.N == 0) return cudaSuccess;
-    if (!a.ck_Kp || !a.ck_Bk || !a.ck_Y0 || !a.ck_G0 || !a.ck_gb) return cudaErrorInvalidValue;
+    if (!a.ck_Kp || !a.ck_Bk || !a.ck_Y0 || !a.ck_G0 || !a.ck_gb || !a.ck_P) return cudaErrorInvalidValue;
     // the data-parallel preparation of every chunk's operands, then the reverse scan
     return dtype == KDA_BF16 ? launch_rscan_typed<__nv_bfloat16>(a, stream) : launch_rscan_typed<float>(a, stream);
 }
@@ -830,6 +814,7 @@ cudaError_t launch_chunk_bwd_scan(const BwdArgs &a, kda_dtype_t dtype, cudaStrea
 cudaError_t launch_chunk_bwd_local(const BwdArgs &a, kda_dtype_t dtype, cudaStream_t stream)
 {
     if (a.N == 0 || a.n_slots == 0) return cudaSuccess;
+    if (!a.ck_P) return cudaErrorInvalidValue;
     return dtype == KDA_BF16 ? launch_local_typed<__nv_bfloat16>(a, stream) : launch_local_typed<float>(a, stream);
 }
 

@@ -109,6 +109,7 @@ struct PrefillArgs {
 // Backward-pass record sizes (floats) per (head, chunk slot).
 constexpr size_t kBwdStateFloats = (size_t)kHeadDim * kHeadDim;   // 128 x 128
 constexpr size_t kBwdRowsFloats = (size_t)kChunk * kHeadDim;       // 64 x 128
+constexpr size_t kBwdTriFloats = (size_t)kChunk * kChunk;          // 64 x 64
 
 // The chunk slot of a chunk starting at absolute token s in sequence n (unique per chunk, below
 // prep_slots(total_tokens, N)).
@@ -214,8 +215,10 @@ struct BwdArgs {
     const float *ck_S, *ck_R, *ck_U;   // from the forward sweep
     float *ck_dS, *ck_Y;               // from the reverse scan
     // state-independent operands of the reverse scan (per (head, slot)), formed by a data-parallel
-    // pass before it when given: Kp, Bk, Y0 (64 x 128), G0 (128 x 128), gamma and beta (256 floats)
+    // pass before it when given: Kp, Bk, Y0 (64 x 128), G0 (128 x 128), gamma and beta (256 floats);
+    // the same pass leaves P = StrictLower(Kt Kh^T) (64 x 64) for the per-chunk kernel
     float *ck_Kp = nullptr, *ck_Bk = nullptr, *ck_Y0 = nullptr, *ck_G0 = nullptr, *ck_gb = nullptr;
+    float *ck_P = nullptr;
     int B, T, H, N, n_slots;
     int32_t *status;
 };

@@ -172,7 +172,7 @@ def test_backward_host_checks(lib):
     # 2 heads x (64 / 64 + 1 + 1) slots of fp32 records, after the status prefix
     # per (head, chunk slot): S, dS' (128 x 128); R, U, Y (64 x 128); the reverse scan's prepared
     # operands Kp, Bk, Y0 (64 x 128), G0 (128 x 128), gamma and beta (256)
-    assert need == 256 + 2 * 3 * (3 * 128 * 128 + 6 * 64 * 128 + 256) * 4
+    assert need == 256 + 2 * 3 * (3 * 128 * 128 + 6 * 64 * 128 + 256 + 64 * 64) * 4
     assert kda.chunk_bwd_workspace_size(1, 64, 2, 1, dk=64) == 0
     # the first failing check decides; none of these reaches a CUDA call
     assert _bwd(lib, dk=64) == kda.KDA_ERR_UNSUPPORTED
