@@ -57,15 +57,14 @@ PREFILL_FLOPS_PER_TOKEN_HEAD = 6 * D * D + 5 * C * D + C * C // 3
 # (TRI = a 64 x 64 triangle times 128 columns, FULL = 64 x 128 x 128, 2 flops per multiply-add):
 #   forward records: A, the solve for U (TRI each); Kt S, Ke^T U (FULL each) (for bf16 inputs the
 #                    forward's tensor-core passes do this work; the count is the fp32 design's)
-#   state gradient:  A, M, M^T dO, the solves for Y0 and Kp (TRI); Qt^T dO, then per chunk of the
-#                    reverse scan Kp dS' and Bk^T Y (FULL)
-#   per chunk:       Kt Kh^T, dO U^T, Y U^T, dM Kh, dP Kh, dM^T Qt, dP^T Kt (TRI); dO S^T, Y S^T,
-#                    U dS'^T (FULL)
+#   state gradient:  A (with Kt Kh^T, kept for the per-chunk kernel), M, M^T dO, the solves for Y0
+#                    and Kp (TRI); Qt^T dO, then per chunk of the reverse scan Kp dS' and Bk^T Y (FULL)
+#   per chunk:       dO U^T, Y U^T, dM Kh, dP Kh, dM^T Qt, dP^T Kt (TRI); dO S^T, Y S^T, U dS'^T (FULL)
 BWD_TRI = C * C // 2 * D * 2
 BWD_FULL = C * D * D * 2
 BWD_FLOPS_PER_CHUNK_HEAD = {"bwd_forward_records": 2 * BWD_TRI + 2 * BWD_FULL,
                             "bwd_scan": 5 * BWD_TRI + 3 * BWD_FULL,
-                            "bwd_local": 7 * BWD_TRI + 3 * BWD_FULL}
+                            "bwd_local": 6 * BWD_TRI + 3 * BWD_FULL}
 # algorithmic HBM bytes per token*head: q, k, v, dout bf16 and log_alpha, beta read; dq, dk, dv,
 # dlog_alpha, dbeta fp32 written
 BWD_BYTES_PER_TOKEN_HEAD = 4 * D * 2 + D * 4 + 4 + 4 * D * 4 + 4
