@@ -158,7 +158,9 @@ kda_status_t kda_chunk_scan(const void *v, const float *S0, const int32_t *cu_se
  * The pages print no backward pass (training uses the chunk mode: lpnh.cn article, sec. 5);
  * these are the chain rule through the recurrence above, computed through the same chunk
  * form (chunk 64). The gradients are fp32 arithmetic on CUDA cores for either input dtype; for
- * bf16 inputs the forward records come from the tensor-core forward passes.
+ * bf16 inputs the forward records come from the tensor-core forward passes, run as
+ * kda_chunk_fwd runs them (pipelined over token ranges on the library's two streams when there
+ * are few (sequence, head) chains; the call stays ordered on `stream`).
  *
  *   q, k, v, log_alpha, beta, S0, cu_seqlens, B, T, H, N, dk, dv, dtype:
  *              exactly as passed to kda_chunk_fwd (the forward is recomputed here).
